@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Decode throughput of the ReplaySSM path on one SSM layer (B200).
+
+One bench step is one window of L decode tokens for the whole batch: L calls of
+replay_step, one of which folds the buffer into the checkpoint (every row of the hot
+path: append, decay scan, k.q products, output-only reads of S0, the fused flush).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica of the batch on its own GPU (sequences
+are independent; there is no collective on the data path) and the timing is the max
+over ranks. Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import gen  # noqa: E402
+
+METRIC = "decode tokens/s per SSM layer at batch 256, L=16 (1 B200); achieved HBM GB/s vs peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
+# window) from an ncu capture, and the hash of the kernel sources it was taken on. When
+# the sources change the figure no longer applies and is reported as null.
+NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None}
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_decode_replay_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def algorithmic_bytes_per_token(s: gen.Shape) -> dict:
+    """Bytes a decoded token must move, per sequence (steady state, lazy flush once per
+    window of L tokens):
+      replay: state (L+1)/L * H*P*N*4 (L-1 output-only reads + one fused read+write),
+              buffer re-reads (L+1)/2 * E, new inputs q + E, entry write E, output 4*H*P,
+              with E = G*N*s + H*P*s + 8*H (one entry: k, v, Delta, a);
+      eager:  state 2 * H*P*N*4 (read + write), inputs q + E, output 4*H*P."""
+    sio = s.io_bytes
+    E = s.G * s.N * sio + s.H * s.P * sio + 8 * s.H
+    q = s.G * s.N * sio
+    y = 4 * s.H * s.P
+    state = s.H * s.P * s.N * 4
+    if s.ckpt == "f32_fp8read":
+        copy = s.H * s.P * (s.N + 4)  # e4m3 codes + per-row scales
+        replay_state = ((s.L - 1) * copy + 2 * state + copy) / s.L
+    else:
+        replay_state = (s.L + 1) / s.L * state
+    replay = replay_state + (s.L + 1) / 2 * E + (q + E) + E + y
+    eager = 2 * state + q + E + y
+    return {"replay": replay, "eager": eager, "replay_state": replay_state, "eager_state": 2 * state}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (the slowest rank sets the time)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons of one GPU with nvidia-smi while running."""
+
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:  # noqa: BLE001
+            pass
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        rows = [r for r in rows if len(r) == len(self.FIELDS) and (self.uuid is None or r[0] == self.uuid)]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_oracle_rate(shape: gen.Shape, budget_s: float, windows_per_seq: int = 1):
+    """Tokens/s of the CPU oracle (float64, one thread) on sequences of the workload's
+    shape: each sample is one sequence, all heads, `windows_per_seq` windows of L steps
+    (one flush each). Runs whole samples until `budget_s` seconds have passed."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import replay_oracle as ro
+
+    one = shape.replace(B=1)
+    S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))
+    steps = windows_per_seq * shape.L
+    xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()} for t in range(steps)]
+    tokens, elapsed, samples = 0, 0.0, 0
+    with threadpool_limits(1):
+        while elapsed < budget_s or samples == 0:
+            t0 = time.perf_counter()
+            seq = ro.ReplayBatch(S0, shape.G, shape.L)
+            for x in xs:
+                seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
+            elapsed += time.perf_counter() - t0
+            tokens += steps
+            samples += 1
+    return tokens / elapsed, samples, steps, elapsed
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local):
+    import linear_attention_decode_replay_b200 as lar
+
+    shape = gen.SHAPES[args.workload]
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = lar.Config(batch=shape.B, heads=shape.H, groups=shape.G, P=shape.P, N=shape.N, L=shape.L,
+                     max_pos=1, io=shape.io, ckpt=shape.ckpt)
+    L, B = shape.L, shape.B
+    bufs = lar.alloc_buffers(cfg, device)
+    S0 = gen.initial_state(shape, device=device)
+    bufs["S0"].copy_(S0)
+    r = lar.Replay(cfg, bufs)
+    window = [gen.step_inputs(shape, t, device=device) for t in range(L)]
+    y = torch.empty(B, shape.H, shape.P, device=device)
+
+    def one_window():
+        for x in window:
+            r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+
+    for _ in range(args.warmup):
+        one_window()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start.record(stream)
+    i = 0
+    for _ in range(K):
+        for x in window:
+            ev[i][0].record(stream)
+            r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+            ev[i][1].record(stream)
+            i += 1
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), world, device)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    avg_launch_ms = max_over_ranks(sum(launch_ms) / len(launch_ms), world, device)
+    status = r.check_status()
+    if status:
+        raise RuntimeError(f"device status bits {status} after the timed region")
+
+    bpt = algorithmic_bytes_per_token(shape)
+    bytes_per_launch = bpt["replay"] * B  # one launch decodes one token of every sequence
+    achieved_gbs = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    traffic = None
+    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_hash():
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+
+    tokens = world * B * L * K
+    value = tokens / (elapsed_ms * 1e-3)
+
+    # ---- the in-house eager kernel on the same inputs (state read + written every token)
+    S = S0.clone()
+    Ke = max(3, K // 4)
+    for _ in range(2):
+        for x in window:
+            lar.eager_step(cfg, S, x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        for x in window:
+            lar.eager_step(cfg, S, x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world, device)
+    del S
+
+    # ---- end to end through the public API: pinned host inputs in, y back to the host
+    host_in = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in window]
+    dev_in = {k: torch.empty_like(v) for k, v in window[0].items()}
+    host_y = torch.empty(B, shape.H, shape.P).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values()) * L
+    d2h = host_y.numel() * host_y.element_size() * L
+    Kx = max(3, min(K, 100))
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(Kx):
+        for hx in host_in:
+            for k in dev_in:
+                dev_in[k].copy_(hx[k], non_blocking=True)
+            r.step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dt"], dev_in["a"], y=y)
+            host_y.copy_(y, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / Kx, world, device)
+    r.close()
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": shape.name, "batch": B, "heads": shape.H, "groups": shape.G, "P": shape.P,
+                   "N": shape.N, "L": L, "io": shape.io, "ckpt": shape.ckpt,
+                   "step": f"one window = {L} replay_step launches x {B} sequences",
+                   "global_batch": B * world, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (checkpoint %d MiB per GPU)" % (B * shape.H * shape.P * shape.N * 4 >> 20)},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": achieved_gbs / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "replay_kernel (replay_step)", "avg_launch_us": avg_launch_ms * 1e3,
+                     "algorithmic_bytes_per_launch": bytes_per_launch},
+        "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * L,
+        "clocks": clk,
+        "eager": {"value": world * B * L / (eager_ms * 1e-3), "unit": UNIT, "ms_per_step": eager_ms,
+                  "kernel": "replay_kernel (eager_step)",
+                  "achieved_gbs": bpt["eager"] * B * L / (eager_ms * 1e-3) / 1e9},
+        "speedup_vs_eager": value / (world * B * L / (eager_ms * 1e-3)),
+        "state_bytes_per_token": {"replay": bpt["replay_state"], "eager": bpt["eager_state"],
+                                  "cut": bpt["eager_state"] / bpt["replay_state"]},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, samples, steps, secs = cpu_oracle_rate(shape, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                  "sample": f"{samples} x (1 sequence x {shape.H} heads x {steps} steps) of "
+                                            f"{shape.name}, float64 numpy, {secs:.1f} s"}
+    return result
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    shape = gen.SHAPES[args.workload]
+    from threadpoolctl import threadpool_limits
+
+    from oracle import replay_oracle as ro
+
+    one = shape.replace(B=1)
+    S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))
+    xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()}
+          for t in range(shape.L)]
+
+    def step():
+        seq = ro.ReplayBatch(S0, shape.G, shape.L)
+        for x in xs + xs[:1]:  # one window plus the step that folds it
+            seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
+
+    with threadpool_limits(1):
+        for _ in range(args.warmup):
+            step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        secs = time.perf_counter() - t0
+    tokens = (shape.L + 1) * args.steps
+    value = tokens / secs
+    sample = f"each step: 1 sequence x {shape.H} heads x {shape.L + 1} decode steps of {shape.name}"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": shape.name, "batch": shape.B, "heads": shape.H, "groups": shape.G, "P": shape.P,
+                   "N": shape.N, "L": shape.L, "io": shape.io, "ckpt": shape.ckpt},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1500, help="timed windows of L decode steps")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mamba2_b256", choices=sorted(k for k in gen.SHAPES if k != "tiny"))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, rank, world)
+        else:
+            out = run_ours(args, rank, world, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * replay.h -- C ABI of the ReplaySSM decode path for scalar-decay (Mamba-2-style) SSM
+ * layers on NVIDIA B200 (sm_100a).
+ *
+ * The method (blog "ReplaySSM: Cachear Inputs, No Estado", sections "Forma resumen",
+ * "Forma historia", the two routes, "Decodificacion estandar", "Rollback",
+ * "Paralelismo"; abstract of arXiv 2610.13778 "ReplaySSM: Cache SSM Inputs, Not State";
+ * video page "The SSM Layer Nobody Made Fast (Until Now): ReplaySSM Explained", key
+ * takeaways): instead of reading and writing the recurrent state
+ *     S_t = a_t S_{t-1} + Delta_t v_t k_t^T,   y_t = S_t q_t
+ * at every decode step, each sequence keeps a checkpoint S0 and a buffer of its inputs
+ * (k_j, v_j, Delta_j, a_j) since S0. Most steps take the output-only route
+ *     y_t = abar_t (S0 q_t) + sum_j s_{j,t} v_j (k_j^T q_t),
+ *     abar_t = prod_{i<=t} a_i,   s_{j,t} = Delta_j prod_{j<i<=t} a_i,
+ * and once per window of L tokens a flush folds the buffer into the checkpoint,
+ *     S0 <- abar S0 + sum_j s_j v_j k_j^T.
+ * Speculative verification scores several positions output-only with a causal mask,
+ * rollback only moves the buffer pointer, and an optional FP8 e4m3 copy of S0 (one FP32
+ * scale per row) serves the outputs while the flush updates an FP32 master.
+ *
+ * Conventions for every call below:
+ *  - All pointers named "device" point to device memory owned by the caller; the
+ *    library never allocates device memory. A replay_ctx holds host metadata only.
+ *  - Work is queued asynchronously on the given stream. Only replay_read_counts and
+ *    replay_check_status synchronise (that stream only).
+ *  - Invalid arguments return a negative replay_status at once and queue nothing.
+ *    Errors found on the device are OR-ed into the caller's status word; read them
+ *    with replay_check_status. No kernel traps.
+ *  - Layouts are dense, row-major, batch-major. Shapes use B = batch, H = heads,
+ *    G = k/q groups (H % G == 0; head h uses group h / (H/G)), P = v-dim, N = k-dim,
+ *    L = window, cap = replay_ring_capacity(cfg). "io" is the replay_config.io dtype.
+ *  - A replay_ctx is not thread-safe; calls on one context must be serialised.
+ */
+#ifndef REPLAY_H
+#define REPLAY_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* replay_stream_t;
+
+typedef enum {
+  REPLAY_OK = 0,
+  REPLAY_EINVAL = -1,      /* bad size, null pointer, unsupported combination */
+  REPLAY_EALIGN = -2,      /* a pointer misses its required alignment */
+  REPLAY_ECUDA = -3,       /* a CUDA runtime call failed (launch, copy, attribute) */
+  REPLAY_EPENDING = -4,    /* a verify is pending: call replay_rollback first */
+  REPLAY_ENOPENDING = -5,  /* replay_rollback without a pending verify */
+  REPLAY_EDEVICE = -6,     /* the device status word is non-zero (see replay_check_status) */
+  REPLAY_ENOMEM = -7       /* host allocation of the context failed */
+} replay_status;
+
+typedef enum { REPLAY_F32 = 0, REPLAY_BF16 = 1 } replay_dtype;
+
+typedef enum {
+  REPLAY_CKPT_F32 = 0,         /* outputs and flushes use the FP32 checkpoint */
+  REPLAY_CKPT_F32_FP8READ = 1  /* outputs read an FP8 e4m3 copy; flushes update the FP32
+                                  master and re-quantise the copy (abstract: separate
+                                  state precisions; video takeaways: dual precision) */
+} replay_ckpt;
+
+/* Device-detected error bits OR-ed into the status word. */
+#define REPLAY_DEV_WAIT_TIMEOUT 1 /* a pipeline wait gave up after ~2 s (results invalid) */
+#define REPLAY_DEV_POINTER 2      /* a buffer pointer word was out of range */
+#define REPLAY_DEV_ROLLBACK 4     /* n_keep outside [0, n_pos]; that sequence kept none */
+
+typedef struct {
+  int32_t batch;   /* B >= 1 */
+  int32_t heads;   /* H >= 1 */
+  int32_t groups;  /* G >= 1, H % G == 0 (k and q are shared by the H/G heads of a group) */
+  int32_t P;       /* v-dim: multiple of 8, 8..256 */
+  int32_t N;       /* k-dim: 16, 32, 64 or 128 */
+  int32_t L;       /* window: buffer entries between checkpoint flushes, 1..64 */
+  int32_t max_pos; /* largest n_pos of replay_verify, 1..8 and <= L (1 = plain decode) */
+  int32_t io;      /* replay_dtype of q, k, v and of the ring of k, v */
+  int32_t ckpt;    /* replay_ckpt */
+} replay_config;
+
+/* Caller-owned device buffers of one decode layer. All 16-byte aligned except counts and
+ * status (4-byte). P*N*4 bytes per head must not exceed 65536. */
+typedef struct {
+  float* S0;         /* [B][H][P][N] FP32 checkpoint (master); row p of N floats contiguous */
+  uint8_t* S0_fp8;   /* [B][H][P][N] e4m3 read copy (ckpt = REPLAY_CKPT_F32_FP8READ, else NULL) */
+  float* S0_scale;   /* [B][H][P] FP32 per-row scale of the copy (same condition) */
+  void* ring_k;      /* [B][G][cap][N] io: buffered k entries */
+  void* ring_v;      /* [B][H][cap][P] io: buffered v entries */
+  float* ring_dt;    /* [B][H][cap] buffered Delta */
+  float* ring_a;     /* [B][H][cap] buffered decay a */
+  int32_t* counts;   /* [2][B] buffer pointer words, double-buffered (the library alternates
+                        halves each call so that no launch reads what it writes) */
+  int32_t* status;   /* [1] device error word (REPLAY_DEV_* bits) */
+} replay_buffers;
+
+typedef struct replay_ctx replay_ctx;
+
+/* Entries the ring arrays must hold per (sequence, head): L + max_pos rounded up to a
+ * multiple of 4. A flush and the appends of the same call touch disjoint slots, so heads
+ * that share a k/q group can run in any order. Returns a negative replay_status on a
+ * bad config. */
+int32_t replay_ring_capacity(const replay_config* cfg);
+
+/* Validates cfg and bufs, zeroes both halves of counts (every buffer empty) and the
+ * status word, and for REPLAY_CKPT_F32_FP8READ fills S0_fp8 / S0_scale from S0 (per-row
+ * e4m3, scale = amax/448). S0 must already hold the initial checkpoint. On success
+ * *out receives a context owned by the caller (free with replay_destroy). */
+int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_stream_t stream,
+                replay_ctx** out);
+
+/* One decode token per sequence (blog "Decodificacion estandar"). Per sequence: if its
+ * buffer already holds L entries, fold them into the checkpoint first, in the same launch
+ * (the state is read once and written once); append (k, v, Delta, a); write
+ *   y = abar (S q) + sum_j s_j v_j (k_j^T q)
+ * over the buffer, S being the stored checkpoint (or its FP8 copy times the row scales)
+ * or the fresh fold.
+ *   q, k:  device [B][G][N] io        v: device [B][H][P] io
+ *   dt, a: device [B][H] FP32         y: device [B][H][P] FP32 (written)
+ *   flushed: device [B] uint8 (written: 1 where this call folded) or NULL.
+ * Returns REPLAY_EPENDING while a verify awaits its rollback. */
+int replay_step(replay_ctx* ctx, const void* q, const void* k, const void* v, const float* dt,
+                const float* a, float* y, uint8_t* flushed, replay_stream_t stream);
+
+/* Output-only verification of n_pos speculative positions (blog "Paralelismo";
+ * abstract: output-only verification without intermediate states). Per sequence with c
+ * committed entries: if c + n_pos > L, fold the c entries first (same launch); then the
+ * n_pos entries are written to the ring tentatively and position s gets
+ *   y_s = abar_{c+s} (S q_s) + sum_{j <= c+s} s_{j,c+s} v_j (k_j^T q_s)
+ * (causal: position s sees the buffer up to its own entry). 1 <= n_pos <= min(L, max_pos).
+ *   q, k:  device [B][n_pos][G][N] io     v: device [B][n_pos][H][P] io
+ *   dt, a: device [B][n_pos][H] FP32      y: device [B][n_pos][H][P] FP32 (written)
+ *   flushed: device [B] uint8 or NULL.
+ * Must be followed by replay_rollback before the next step, verify or flush. */
+int replay_verify(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k, const void* v,
+                  const float* dt, const float* a, float* y, uint8_t* flushed,
+                  replay_stream_t stream);
+
+/* Resolves the pending verify (blog "Rollback (deshacer)"; video takeaways: rollback is a
+ * pointer move): sequence b keeps the first n_keep[b] of the n_pos tentative entries
+ * (device int32 [B], values in [0, n_pos]); the rest are dropped by moving the buffer end
+ * back, O(1) per sequence, no state traffic. A value outside the range sets
+ * REPLAY_DEV_ROLLBACK and keeps none for that sequence. */
+int replay_rollback(replay_ctx* ctx, const int32_t* n_keep, replay_stream_t stream);
+
+/* Folds the buffer of every sequence with mask[b] != 0 (device uint8 [B]; NULL = all)
+ * into the checkpoint (state route) and empties it; also refreshes the FP8 copy. */
+int replay_flush(replay_ctx* ctx, const uint8_t* mask, replay_stream_t stream);
+
+/* Copies the committed entry count of every sequence to host_counts (host int32 [B]);
+ * synchronises the stream. */
+int replay_read_counts(replay_ctx* ctx, int32_t* host_counts, replay_stream_t stream);
+
+/* Reads the device status word (synchronises the stream). Returns REPLAY_OK if it is
+ * zero, else REPLAY_EDEVICE; *host_bits (may be NULL) receives the REPLAY_DEV_* bits. */
+int replay_check_status(replay_ctx* ctx, int32_t* host_bits, replay_stream_t stream);
+
+/* Frees the host context (the caller's device buffers are untouched). NULL is a no-op. */
+void replay_destroy(replay_ctx* ctx);
+
+/* Baseline: one eager decode step (blog "Forma resumen"), S <- a S + Delta v k^T and
+ * y = S q, the FP32 state read and written in place. cfg supplies B, H, G, P, N, io
+ * (L, max_pos and ckpt are ignored).
+ *   S: device [B][H][P][N] FP32 (updated)   q, k: device [B][G][N] io   v: [B][H][P] io
+ *   dt, a: device [B][H] FP32               y: device [B][H][P] FP32 (written) */
+int eager_step(const replay_config* cfg, float* S, const void* q, const void* k, const void* v,
+               const float* dt, const float* a, float* y, replay_stream_t stream);
+
+/* Baseline: eager step on a state kept only in FP8 e4m3 with a per-row FP32 scale (a
+ * shared low-precision checkpoint, whose rounding enters every later update; abstract
+ * and video takeaways): dequantise, update, y from the updated FP32 values, re-quantise.
+ *   S8: device [B][H][P][N] e4m3 (updated)   scale: device [B][H][P] FP32 (updated)
+ *   other arguments as eager_step. */
+int eager_step_fp8(const replay_config* cfg, uint8_t* S8, float* scale, const void* q,
+                   const void* k, const void* v, const float* dt, const float* a, float* y,
+                   replay_stream_t stream);
+
+/* Per-row e4m3 quantisation used for the FP8 read copy: for each row of n FP32 values,
+ * scale = amax/448 (1 for an all-zero row) and code = e4m3(x * (448/amax)) with the
+ * product rounded to FP32, round-to-nearest-even, saturating to +-448.
+ *   x: device [rows][n] FP32   codes: device [rows][n] uint8   scale: device [rows] FP32
+ *   n: 16, 32, 64 or 128. */
+int replay_quantize_rows_e4m3(const float* x, int64_t rows, int32_t n, uint8_t* codes,
+                              float* scale, replay_stream_t stream);
+
+/* Static text for a replay_status code. */
+const char* replay_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REPLAY_H */

@@ -1,0 +1,417 @@
+// Host side of the C ABI declared in include/replay.h: argument validation, the shared-
+// memory layout of the replay kernel, the double-buffered pointer words, the pending-
+// verify protocol, and launches on the caller's stream. No device memory is allocated.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "../../include/replay.h"
+#include "replay_device.cuh"
+#include "replay_launch.h"
+
+using replay::KParams;
+
+struct replay_ctx {
+  replay_config cfg;
+  replay_buffers bufs;
+  int cap;
+  int parity;   // which half of counts holds the current pointer words
+  int pending;  // n_pos of an unresolved verify, 0 if none
+  int device;
+  int num_sms;
+  KParams kp_step, kp_verify, kp_flush;  // prebuilt launch layouts (pointers filled per call)
+  int verify_ok;                          // kp_verify was built (max_pos > 1)
+};
+
+namespace {
+
+constexpr int kHeaderBytes = 256;  // 2 * kMaxStages mbarriers + abort flag
+
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate_config(const replay_config* c, bool needs_window) {
+  if (!c) return REPLAY_EINVAL;
+  if (c->batch < 1 || c->heads < 1 || c->groups < 1 || c->heads % c->groups) return REPLAY_EINVAL;
+  if (c->P < 8 || c->P > 256 || c->P % 8) return REPLAY_EINVAL;
+  if (c->N != 16 && c->N != 32 && c->N != 64 && c->N != 128) return REPLAY_EINVAL;
+  if ((int64_t)c->P * c->N * 4 > 65536) return REPLAY_EINVAL;
+  if (c->io != REPLAY_F32 && c->io != REPLAY_BF16) return REPLAY_EINVAL;
+  if ((int64_t)c->batch * c->heads > INT32_MAX / 2) return REPLAY_EINVAL;
+  if (needs_window) {
+    if (c->L < 1 || c->L > 64) return REPLAY_EINVAL;
+    if (c->max_pos < 1 || c->max_pos > replay::kMaxPos || c->max_pos > c->L) return REPLAY_EINVAL;
+    if (c->ckpt != REPLAY_CKPT_F32 && c->ckpt != REPLAY_CKPT_F32_FP8READ) return REPLAY_EINVAL;
+  }
+  return REPLAY_OK;
+}
+
+int ring_capacity(const replay_config& c) { return round_up(c.L + c.max_pos, 4); }
+
+struct DeviceInfo {
+  int device, num_sms, smem_optin;
+};
+
+int device_info(DeviceInfo* d) {
+  if (cudaGetDevice(&d->device) != cudaSuccess) return REPLAY_ECUDA;
+  if (cudaDeviceGetAttribute(&d->num_sms, cudaDevAttrMultiProcessorCount, d->device) != cudaSuccess)
+    return REPLAY_ECUDA;
+  if (cudaDeviceGetAttribute(&d->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, d->device) != cudaSuccess)
+    return REPLAY_ECUDA;
+  return REPLAY_OK;
+}
+
+// Shared-memory layout of one launch mode. nq_alloc = query slots per stage, jmax =
+// entries a stage holds (buffer + new), lfold = most entries one unit folds.
+int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, int cap, int smem_optin) {
+  std::memset(p, 0, sizeof(*p));
+  const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
+  const int P = c.P, N = c.N;
+  int jmax, nq_alloc, lfold, ring;
+  if (mode == replay::kModeReplay) {
+    jmax = c.L + c.max_pos;
+    nq_alloc = c.max_pos;
+    lfold = c.L;
+    ring = cap;
+  } else if (mode == replay::kModeFlush) {
+    jmax = c.L;
+    nq_alloc = 0;
+    lfold = c.L;
+    ring = cap;
+  } else {
+    jmax = 1;
+    nq_alloc = 1;
+    lfold = 1;
+    ring = 0;
+  }
+  const int tile = fp8_eager ? round_up(P * N + P * 4, 16) : P * N * 4;
+  p->off_k = round_up(tile, 16);
+  p->off_v = p->off_k + round_up(jmax * N * s_io, 16);
+  p->off_q = p->off_v + round_up(jmax * P * s_io, 16);
+  p->off_dtr = p->off_q + round_up(nq_alloc * N * s_io, 16);
+  p->off_ar = p->off_dtr + round_up(ring * 4, 16);
+  p->off_dtn = p->off_ar + round_up(ring * 4, 16);
+  p->off_an = p->off_dtn + replay::kMaxPos * 4;
+  p->off_meta = p->off_an + replay::kMaxPos * 4;
+  p->stage_bytes = round_up(p->off_meta + 16, 128);
+
+  p->jw = round_up(c.L + c.max_pos + 1, 4);
+  p->fp = round_up(lfold, replay::kFoldChunk);
+  p->ws_w = 0;
+  p->ws_kq = p->ws_w + replay::kMaxPos * p->jw * 4;
+  p->ws_alpha = p->ws_kq + replay::kMaxPos * p->jw * 4;
+  p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
+  p->ws_wt = round_up(p->ws_sig + (p->jw + 4) * 4, 16);
+  p->ws_bt = p->ws_wt + P * p->fp * 4;
+  const int ws_bytes = round_up(p->ws_bt + replay::kMaxPos * P * 4, 128);
+  p->ws_off = kHeaderBytes;
+  p->stages_off = round_up(kHeaderBytes + ws_bytes, 128);
+  const int avail = smem_optin - p->stages_off;
+  int ns = avail / p->stage_bytes;
+  if (ns > replay::kMaxStages) ns = replay::kMaxStages;
+  if (ns < 2) return REPLAY_EINVAL;
+  p->num_stages = ns;
+  p->smem_bytes = p->stages_off + ns * p->stage_bytes;
+
+  p->B = c.batch;
+  p->H = c.heads;
+  p->G = c.groups;
+  p->P = P;
+  p->N = N;
+  p->L = c.L;
+  p->cap = cap;
+  p->hpg = c.heads / c.groups;
+  p->num_units = c.batch * c.heads;
+  return REPLAY_OK;
+}
+
+cudaError_t launch_main(const KParams& p, const replay_config& c, int ckpt, int mode, int nq, int num_sms,
+                        cudaStream_t s) {
+  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  switch (c.N) {
+    case 16: return replay::launch_replay_n16(p, c.io, ckpt, mode, nq, grid, s);
+    case 32: return replay::launch_replay_n32(p, c.io, ckpt, mode, nq, grid, s);
+    case 64: return replay::launch_replay_n64(p, c.io, ckpt, mode, nq, grid, s);
+    case 128: return replay::launch_replay_n128(p, c.io, ckpt, mode, nq, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+void set_state(KParams* p, const replay_ctx* ctx) {
+  p->S = ctx->bufs.S0;
+  p->S8 = ctx->bufs.S0_fp8;
+  p->Sscale = ctx->bufs.S0_scale;
+  p->ring_k = ctx->bufs.ring_k;
+  p->ring_v = ctx->bufs.ring_v;
+  p->ring_dt = ctx->bufs.ring_dt;
+  p->ring_a = ctx->bufs.ring_a;
+  p->counts_in = ctx->bufs.counts + (size_t)ctx->parity * ctx->cfg.batch;
+  p->counts_out = ctx->bufs.counts + (size_t)(1 - ctx->parity) * ctx->cfg.batch;
+  p->status = ctx->bufs.status;
+}
+
+int check_inputs(const void* q, const void* k, const void* v, const float* dt, const float* a, const float* y) {
+  if (!q || !k || !v || !dt || !a || !y) return REPLAY_EINVAL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return REPLAY_EALIGN;
+  if (!aligned(dt, 4) || !aligned(a, 4) || !aligned(y, 4)) return REPLAY_EALIGN;
+  return REPLAY_OK;
+}
+
+int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const void* k, const void* v,
+                const float* dt, const float* a, float* y, uint8_t* flushed, cudaStream_t s) {
+  KParams p = (n_pos > 1) ? ctx->kp_verify : ctx->kp_step;
+  set_state(&p, ctx);
+  p.n_pos = n_pos;
+  p.commit = commit;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.dt = dt;
+  p.a = a;
+  p.y = y;
+  p.flushed = flushed;
+  const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
+  if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos > 1 ? replay::kMaxPos : 1, ctx->num_sms, s) !=
+      cudaSuccess)
+    return REPLAY_ECUDA;
+  ctx->parity ^= 1;
+  return REPLAY_OK;
+}
+
+int eager_call(const replay_config* cfg, float* S, uint8_t* S8, float* scale, const void* q, const void* k,
+               const void* v, const float* dt, const float* a, float* y, cudaStream_t s) {
+  replay_config c = *cfg;
+  c.L = 1;
+  c.max_pos = 1;
+  c.ckpt = REPLAY_CKPT_F32;
+  int rc = validate_config(&c, true);
+  if (rc) return rc;
+  if ((rc = check_inputs(q, k, v, dt, a, y))) return rc;
+  const bool fp8 = S8 != nullptr;
+  if (fp8) {
+    if (!scale) return REPLAY_EINVAL;
+    if (!aligned(S8, 16) || !aligned(scale, 16)) return REPLAY_EALIGN;
+  } else {
+    if (!S) return REPLAY_EINVAL;
+    if (!aligned(S, 16)) return REPLAY_EALIGN;
+  }
+  DeviceInfo d;
+  if ((rc = device_info(&d))) return rc;
+  KParams p;
+  if ((rc = build_layout(&p, c, replay::kModeEager, fp8 ? 1 : 0, 0, d.smem_optin))) return rc;
+  p.S = S;
+  p.S8 = S8;
+  p.Sscale = scale;
+  p.n_pos = 1;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.dt = dt;
+  p.a = a;
+  p.y = y;
+  p.status = nullptr;
+  if (launch_main(p, c, fp8 ? replay::kCkptFp8 : replay::kCkptF32, replay::kModeEager, 1, d.num_sms, s) !=
+      cudaSuccess)
+    return REPLAY_ECUDA;
+  return REPLAY_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t replay_ring_capacity(const replay_config* cfg) {
+  const int rc = validate_config(cfg, true);
+  if (rc) return rc;
+  return ring_capacity(*cfg);
+}
+
+int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_stream_t stream, replay_ctx** out) {
+  if (!out) return REPLAY_EINVAL;
+  *out = nullptr;
+  int rc = validate_config(cfg, true);
+  if (rc) return rc;
+  if (!bufs || !bufs->S0 || !bufs->ring_k || !bufs->ring_v || !bufs->ring_dt || !bufs->ring_a || !bufs->counts ||
+      !bufs->status)
+    return REPLAY_EINVAL;
+  const bool fp8 = cfg->ckpt == REPLAY_CKPT_F32_FP8READ;
+  if (fp8 && (!bufs->S0_fp8 || !bufs->S0_scale)) return REPLAY_EINVAL;
+  if (!aligned(bufs->S0, 16) || !aligned(bufs->ring_k, 16) || !aligned(bufs->ring_v, 16) ||
+      !aligned(bufs->ring_dt, 16) || !aligned(bufs->ring_a, 16) || !aligned(bufs->counts, 4) ||
+      !aligned(bufs->status, 4))
+    return REPLAY_EALIGN;
+  if (fp8 && (!aligned(bufs->S0_fp8, 16) || !aligned(bufs->S0_scale, 16))) return REPLAY_EALIGN;
+
+  DeviceInfo d;
+  if ((rc = device_info(&d))) return rc;
+  replay_ctx* ctx = new (std::nothrow) replay_ctx;
+  if (!ctx) return REPLAY_ENOMEM;
+  std::memset(ctx, 0, sizeof(*ctx));
+  ctx->cfg = *cfg;
+  ctx->bufs = *bufs;
+  if (!fp8) {
+    ctx->bufs.S0_fp8 = nullptr;
+    ctx->bufs.S0_scale = nullptr;
+  }
+  ctx->cap = ring_capacity(*cfg);
+  ctx->device = d.device;
+  ctx->num_sms = d.num_sms;
+  replay_config one = *cfg;
+  one.max_pos = 1;
+  if ((rc = build_layout(&ctx->kp_step, one, replay::kModeReplay, 0, ctx->cap, d.smem_optin)) ||
+      (rc = build_layout(&ctx->kp_flush, *cfg, replay::kModeFlush, 0, ctx->cap, d.smem_optin))) {
+    delete ctx;
+    return rc;
+  }
+  if (cfg->max_pos > 1) {
+    if ((rc = build_layout(&ctx->kp_verify, *cfg, replay::kModeReplay, 0, ctx->cap, d.smem_optin))) {
+      delete ctx;
+      return rc;
+    }
+    ctx->verify_ok = 1;
+  }
+  // the step layout was built with max_pos = 1 but indexes the same ring (capacity cap)
+  ctx->kp_step.cap = ctx->cap;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(bufs->counts, 0, sizeof(int32_t) * 2 * (size_t)cfg->batch, s) != cudaSuccess ||
+      cudaMemsetAsync(bufs->status, 0, sizeof(int32_t), s) != cudaSuccess) {
+    delete ctx;
+    return REPLAY_ECUDA;
+  }
+  if (fp8) {
+    const long long rows = (long long)cfg->batch * cfg->heads * cfg->P;
+    const long long passes = (rows + (256 / (cfg->N / 4)) - 1) / (256 / (cfg->N / 4));
+    const int grid = (int)(passes < (long long)d.num_sms * 8 ? passes : (long long)d.num_sms * 8);
+    if (replay::launch_quantize_rows(bufs->S0, rows, cfg->N, bufs->S0_fp8, bufs->S0_scale, grid, s) !=
+        cudaSuccess) {
+      delete ctx;
+      return REPLAY_ECUDA;
+    }
+  }
+  *out = ctx;
+  return REPLAY_OK;
+}
+
+int replay_step(replay_ctx* ctx, const void* q, const void* k, const void* v, const float* dt, const float* a,
+                float* y, uint8_t* flushed, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  int rc = check_inputs(q, k, v, dt, a, y);
+  if (rc) return rc;
+  return replay_call(ctx, 1, 1, q, k, v, dt, a, y, flushed, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int replay_verify(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k, const void* v, const float* dt,
+                  const float* a, float* y, uint8_t* flushed, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  if (n_pos < 1 || n_pos > ctx->cfg.max_pos || n_pos > ctx->cfg.L) return REPLAY_EINVAL;
+  int rc = check_inputs(q, k, v, dt, a, y);
+  if (rc) return rc;
+  if (n_pos > 1 && !ctx->verify_ok) return REPLAY_EINVAL;
+  rc = replay_call(ctx, n_pos, 0, q, k, v, dt, a, y, flushed, reinterpret_cast<cudaStream_t>(stream));
+  if (rc == REPLAY_OK) ctx->pending = n_pos;
+  return rc;
+}
+
+int replay_rollback(replay_ctx* ctx, const int32_t* n_keep, replay_stream_t stream) {
+  if (!ctx || !n_keep) return REPLAY_EINVAL;
+  if (!ctx->pending) return REPLAY_ENOPENDING;
+  if (!aligned(n_keep, 4)) return REPLAY_EALIGN;
+  const int B = ctx->cfg.batch;
+  const int32_t* cin = ctx->bufs.counts + (size_t)ctx->parity * B;
+  int32_t* cout = ctx->bufs.counts + (size_t)(1 - ctx->parity) * B;
+  if (replay::launch_rollback(cin, cout, n_keep, B, ctx->pending, ctx->bufs.status,
+                              reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return REPLAY_ECUDA;
+  ctx->parity ^= 1;
+  ctx->pending = 0;
+  return REPLAY_OK;
+}
+
+int replay_flush(replay_ctx* ctx, const uint8_t* mask, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  KParams p = ctx->kp_flush;
+  set_state(&p, ctx);
+  p.mask = mask;
+  const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
+  if (launch_main(p, ctx->cfg, ckpt, replay::kModeFlush, 0, ctx->num_sms, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return REPLAY_ECUDA;
+  ctx->parity ^= 1;
+  return REPLAY_OK;
+}
+
+int replay_read_counts(replay_ctx* ctx, int32_t* host_counts, replay_stream_t stream) {
+  if (!ctx || !host_counts) return REPLAY_EINVAL;
+  const int B = ctx->cfg.batch;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host_counts, ctx->bufs.counts + (size_t)ctx->parity * B, sizeof(int32_t) * B,
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return REPLAY_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return REPLAY_ECUDA;
+  for (int b = 0; b < B; ++b) host_counts[b] &= 0xFFFF;
+  return REPLAY_OK;
+}
+
+int replay_check_status(replay_ctx* ctx, int32_t* host_bits, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t bits = 0;
+  if (cudaMemcpyAsync(&bits, ctx->bufs.status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return REPLAY_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return REPLAY_ECUDA;
+  if (host_bits) *host_bits = bits;
+  return bits ? REPLAY_EDEVICE : REPLAY_OK;
+}
+
+void replay_destroy(replay_ctx* ctx) { delete ctx; }
+
+int eager_step(const replay_config* cfg, float* S, const void* q, const void* k, const void* v, const float* dt,
+               const float* a, float* y, replay_stream_t stream) {
+  if (!cfg) return REPLAY_EINVAL;
+  return eager_call(cfg, S, nullptr, nullptr, q, k, v, dt, a, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int eager_step_fp8(const replay_config* cfg, uint8_t* S8, float* scale, const void* q, const void* k, const void* v,
+                   const float* dt, const float* a, float* y, replay_stream_t stream) {
+  if (!cfg || !S8) return REPLAY_EINVAL;
+  return eager_call(cfg, nullptr, S8, scale, q, k, v, dt, a, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int replay_quantize_rows_e4m3(const float* x, int64_t rows, int32_t n, uint8_t* codes, float* scale,
+                              replay_stream_t stream) {
+  if (!x || !codes || !scale || rows < 0) return REPLAY_EINVAL;
+  if (n != 16 && n != 32 && n != 64 && n != 128) return REPLAY_EINVAL;
+  if (!aligned(x, 16) || !aligned(codes, 4) || !aligned(scale, 4)) return REPLAY_EALIGN;
+  if (rows == 0) return REPLAY_OK;
+  DeviceInfo d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  const long long rpb = 256 / (n / 4);
+  const long long passes = (rows + rpb - 1) / rpb;
+  const int grid = (int)(passes < (long long)d.num_sms * 8 ? passes : (long long)d.num_sms * 8);
+  if (replay::launch_quantize_rows(x, rows, n, codes, scale, grid, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return REPLAY_ECUDA;
+  return REPLAY_OK;
+}
+
+const char* replay_strerror(int code) {
+  switch (code) {
+    case REPLAY_OK: return "ok";
+    case REPLAY_EINVAL: return "invalid argument";
+    case REPLAY_EALIGN: return "misaligned pointer";
+    case REPLAY_ECUDA: return "CUDA runtime error";
+    case REPLAY_EPENDING: return "a verify is pending: call replay_rollback first";
+    case REPLAY_ENOPENDING: return "no verify is pending";
+    case REPLAY_EDEVICE: return "device reported an error (see the status bits)";
+    case REPLAY_ENOMEM: return "host allocation failed";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

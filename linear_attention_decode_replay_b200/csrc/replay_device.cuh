@@ -1,0 +1,216 @@
+// Device-side building blocks for the replay decode kernels (sm_100a):
+// mbarrier and bulk-copy (TMA) wrappers written as inline PTX, bounded waits that
+// report a timeout through the status word instead of trapping, segment reductions
+// over the lanes that share one state row, and FP8 e4m3 / BF16 conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace replay {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kMaxPos = 8;                       // query positions per verify call
+constexpr int kMaxStages = 8;
+constexpr int kFoldChunk = 8;                    // buffer entries folded per register pass
+constexpr int kRowsPerThread = 8;                // state rows one thread covers per row group
+constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
+
+// status word bits (device-detected errors; the host reads them with replay_check_status)
+constexpr int32_t kErrWaitTimeout = 1 << 0;   // an mbarrier wait gave up
+constexpr int32_t kErrPointer = 1 << 1;       // a buffer pointer word was out of range
+constexpr int32_t kErrRollback = 1 << 2;      // n_keep outside [0, n_pos]
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with the given parity to complete; gives up after about two
+// seconds and returns false (the caller records kErrWaitTimeout and winds down).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+}
+
+// ---------------------------------------------------------------- bulk copy (TMA, 1-D)
+// Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte aligned),
+// completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- consumer-only barriers
+// Named barrier 1 spans the consumer warps only (the producer warp never joins it).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+// Barrier with an AND-vote across the consumer threads.
+__device__ __forceinline__ bool consumer_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kConsumerThreads)
+      : "memory");
+  return r != 0;
+}
+
+// ---------------------------------------------------------------- conversions
+template <typename IO>
+struct IoT;
+template <>
+struct IoT<float> {
+  static constexpr int bytes = 4;
+  __device__ __forceinline__ static float4 load4(const void* p) {
+    return *reinterpret_cast<const float4*>(p);
+  }
+  __device__ __forceinline__ static float load1(const void* p) { return *reinterpret_cast<const float*>(p); }
+};
+template <>
+struct IoT<__nv_bfloat16> {
+  static constexpr int bytes = 2;
+  __device__ __forceinline__ static float4 load4(const void* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const float2 a = __bfloat1622float2(lo);
+    const float2 b = __bfloat1622float2(hi);
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
+  __device__ __forceinline__ static float load1(const void* p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+  }
+};
+
+// four e4m3 codes (byte i = element i) -> four floats
+__device__ __forceinline__ float4 e4m3x4_to_float4(uint32_t w) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+// one float -> e4m3 code, round to nearest even, saturating to +-448
+__device__ __forceinline__ uint32_t float_to_e4m3(float x) {
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+// quantise four values of one row with that row's inverse scale; byte i = element i
+__device__ __forceinline__ uint32_t quant4_e4m3(float4 x, float inv) {
+  return float_to_e4m3(__fmul_rn(x.x, inv)) | (float_to_e4m3(__fmul_rn(x.y, inv)) << 8) |
+         (float_to_e4m3(__fmul_rn(x.z, inv)) << 16) | (float_to_e4m3(__fmul_rn(x.w, inv)) << 24);
+}
+// row scale and its inverse from the row's largest magnitude (1 and 1 for a zero row)
+__device__ __forceinline__ void e4m3_row_scale(float amax, float& scale, float& inv) {
+  if (amax > 0.f) {
+    scale = __fdiv_rn(amax, 448.f);
+    inv = __fdiv_rn(448.f, amax);
+  } else {
+    scale = 1.f;
+    inv = 1.f;
+  }
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+__device__ __forceinline__ float amax4(float4 a) {
+  return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+}
+
+// ---------------------------------------------------------------- segment reductions
+// Sum over the TPR lanes of an aligned lane segment (all lanes get the total).
+template <int TPR>
+__device__ __forceinline__ float seg_allsum(float v) {
+#pragma unroll
+  for (int off = TPR / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+template <int TPR>
+__device__ __forceinline__ float seg_allmax(float v) {
+#pragma unroll
+  for (int off = TPR / 2; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// Transposing reduction: each lane of a TPR-lane segment holds R partial sums (one per
+// row it covers); afterwards lane l holds complete row sums for R/TPR rows (or one row,
+// replicated over TPR/R lanes, when R < TPR). Costs about R + log2(TPR) shuffles
+// instead of R * log2(TPR). `base` returns the index of the first row held in v[0].
+template <int R, int OFF>
+struct SegTranspose {
+  __device__ __forceinline__ static void run(float* v, int lane, int& base) {
+    if constexpr (OFF >= 1) {
+      if constexpr (R > 1) {
+        constexpr int H = R / 2;
+        const bool up = (lane & OFF) != 0;
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+          const float send = up ? v[i] : v[i + H];
+          const float keep = up ? v[i + H] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+        }
+        if (up) base += H;
+        SegTranspose<H, OFF / 2>::run(v, lane, base);
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+        SegTranspose<1, OFF / 2>::run(v, lane, base);
+      }
+    }
+  }
+};
+template <int R, int TPR>
+struct SegReduce {
+  static constexpr int kHeld = (R >= TPR) ? R / TPR : 1;  // row sums each lane ends with
+  // returns true for the lanes that should write their v[0..kHeld)
+  __device__ __forceinline__ static bool run(float* v, int lane, int& base) {
+    base = 0;
+    SegTranspose<R, TPR / 2>::run(v, lane, base);
+    if constexpr (R >= TPR) {
+      return true;
+    } else {
+      return (lane & (TPR / R - 1)) == 0;
+    }
+  }
+};
+
+}  // namespace replay

@@ -1,0 +1,61 @@
+// Instantiates the replay kernel for one k-dim (REPLAY_N) and provides its launcher.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "replay_kernel.cuh"
+#include "replay_launch.h"
+
+#ifndef REPLAY_N
+#error "define REPLAY_N before including replay_instances.cuh"
+#endif
+
+namespace replay {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+template <typename IO, int CKPT, int MODE, int NQ>
+cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
+  auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ>;
+  // the dynamic shared-memory opt-in is per function and device; remember the largest set
+  static int configured[kMaxDevices] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices || configured[dev] < p.smem_bytes) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) configured[dev] = p.smem_bytes;
+  }
+  kern<<<grid, kThreads, p.smem_bytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename IO, int CKPT>
+cudaError_t launch_mode(const KParams& p, int mode, int nq, int grid, cudaStream_t s) {
+  if (mode == kModeReplay) {
+    return nq > 1 ? launch_one<IO, CKPT, kModeReplay, kMaxPos>(p, grid, s)
+                  : launch_one<IO, CKPT, kModeReplay, 1>(p, grid, s);
+  }
+  if (mode == kModeFlush) return launch_one<IO, CKPT, kModeFlush, 0>(p, grid, s);
+  return launch_one<IO, CKPT, kModeEager, 1>(p, grid, s);
+}
+
+template <typename IO>
+cudaError_t launch_ckpt(const KParams& p, int ckpt, int mode, int nq, int grid, cudaStream_t s) {
+  return ckpt == kCkptFp8 ? launch_mode<IO, kCkptFp8>(p, mode, nq, grid, s)
+                          : launch_mode<IO, kCkptF32>(p, mode, nq, grid, s);
+}
+
+}  // namespace
+
+#define REPLAY_CAT2(a, b) a##b
+#define REPLAY_CAT(a, b) REPLAY_CAT2(a, b)
+cudaError_t REPLAY_CAT(launch_replay_n, REPLAY_N)(const KParams& p, int io, int ckpt, int mode, int nq, int grid,
+                                                   cudaStream_t s) {
+  return io == 1 ? launch_ckpt<__nv_bfloat16>(p, ckpt, mode, nq, grid, s)
+                 : launch_ckpt<float>(p, ckpt, mode, nq, grid, s);
+}
+
+}  // namespace replay

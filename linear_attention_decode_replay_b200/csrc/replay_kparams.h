@@ -1,0 +1,43 @@
+// Launch parameters shared by the host launcher and the replay kernel.
+#pragma once
+
+#include <stdint.h>
+
+namespace replay {
+
+enum { kModeReplay = 0, kModeFlush = 1, kModeEager = 2 };
+enum { kCkptF32 = 0, kCkptFp8 = 1 };
+
+struct KParams {
+  // sizes
+  int32_t B, H, G, P, N, L, cap, n_pos, hpg, num_units;
+  int32_t commit;  // replay: 1 = step (new entries committed), 0 = verify (tentative)
+  // this call's inputs and outputs
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* dt;
+  const float* a;
+  float* y;
+  uint8_t* flushed;
+  const uint8_t* mask;
+  // state (checkpoint or eager state)
+  float* S;
+  uint8_t* S8;
+  float* Sscale;
+  void* ring_k;
+  void* ring_v;
+  float* ring_dt;
+  float* ring_a;
+  const int32_t* counts_in;
+  int32_t* counts_out;
+  int32_t* status;
+  // shared-memory layout, bytes
+  int32_t num_stages, stage_bytes, stages_off, ws_off;
+  int32_t off_k, off_v, off_q, off_dtr, off_ar, off_dtn, off_an, off_meta;  // within a stage
+  int32_t ws_w, ws_kq, ws_alpha, ws_sig, ws_wt, ws_bt;                      // within the workspace
+  int32_t jw, fp;  // workspace row strides (entries per query row, fold entries per state row)
+  int32_t smem_bytes;
+};
+
+}  // namespace replay

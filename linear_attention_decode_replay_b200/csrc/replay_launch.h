@@ -1,0 +1,22 @@
+// Internal launch entry points, one per supported k-dim N (one translation unit each).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "replay_kparams.h"
+
+namespace replay {
+
+// mode: kModeReplay / kModeFlush / kModeEager; ckpt: kCkptF32 / kCkptFp8;
+// io: 0 = FP32, 1 = BF16; nq: query registers (1, or kMaxPos for multi-position verify)
+cudaError_t launch_replay_n16(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
+cudaError_t launch_replay_n32(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
+cudaError_t launch_replay_n64(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
+cudaError_t launch_replay_n128(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
+
+cudaError_t launch_quantize_rows(const float* x, long long rows, int n, unsigned char* codes, float* scale,
+                                 int grid, cudaStream_t s);
+cudaError_t launch_rollback(const int* counts_in, int* counts_out, const int* n_keep, int B, int n_pos,
+                            int* status, cudaStream_t s);
+
+}  // namespace replay

@@ -200,6 +200,7 @@ class ReplaySeq:
         self.pending = None  # (base, n_pos) of an unresolved verify
         self.state_reads = 0
         self.state_writes = 0
+        self._read_copy = None  # dequantised FP8 copy, kept until the next flush
         if ckpt == "f32_fp8read":
             self.codes, self.scale = quantize_rows_e4m3(self.S0)
 
@@ -231,6 +232,7 @@ class ReplaySeq:
             self.S0 = state_route(self.S0, abar, s, vb, kb)
             if self.ckpt == "f32_fp8read":
                 self.codes, self.scale = quantize_rows_e4m3(self.S0)
+                self._read_copy = None
             self.state_reads += 1
             self.state_writes += 1
         self.k, self.v, self.dt, self.a = [], [], [], []
@@ -242,7 +244,9 @@ class ReplaySeq:
         if self.ckpt == "f32" or from_master:
             S_read = self.S0
         else:
-            S_read = dequantize_rows_e4m3(self.codes, self.scale)
+            if self._read_copy is None:
+                self._read_copy = dequantize_rows_e4m3(self.codes, self.scale)
+            S_read = self._read_copy
         return output_only(S_read, abar, s, vb, kb, np.asarray(q, np.float64)[self.group_of_head])
 
     def step(self, q, k, v, dt, a):

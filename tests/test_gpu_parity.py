@@ -1,0 +1,224 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element on the same
+seeded inputs: small shapes in full, the full-size workloads on sampled sequences."""
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_harness as hx
+import linear_attention_decode_replay_b200 as lar
+from linear_attention_decode_replay_b200 import _abi
+from oracle import replay_oracle as ro
+from workloads import gen
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+
+def _check_decode(rep, tol=hx.TOL_F32):
+    assert rep.max_err <= tol, (rep.max_err, int(np.argmax(rep.per_step)))
+    assert rep.flags_equal, "flush flags differ from the oracle's schedule"
+    assert rep.counts_equal, "buffer counts differ from the oracle's"
+    assert rep.ckpt_err <= tol, rep.ckpt_err
+
+
+# ------------------------------------------------------------------ FP8 quantiser, bit-exact
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128])
+def test_quantize_rows_bit_exact(n):
+    g = torch.Generator(device="cuda").manual_seed(1234 + n)
+    rows = 4096
+    mags = torch.exp2(torch.randint(-30, 30, (rows, 1), generator=g, device="cuda").float())
+    x = torch.randn(rows, n, generator=g, device="cuda") * mags
+    x[7] = 0.0                       # all-zero row
+    x[9, :] = 0.0
+    x[9, 3] = -2.5                   # single non-zero
+    x[11] = torch.linspace(-448, 448, n, device="cuda")  # values on codes and between
+    x[13] = 1e-30 * torch.randn(n, generator=g, device="cuda")  # tiny magnitudes
+    codes, scale = lar.quantize_rows_e4m3(x)
+    want_codes, want_scale = ro.quantize_rows_e4m3(x.cpu().numpy())
+    np.testing.assert_array_equal(scale.cpu().numpy(), want_scale)
+    np.testing.assert_array_equal(codes.cpu().numpy(), want_codes)
+
+
+# ------------------------------------------------------------------ small shapes, every output
+
+def test_tiny_replay_matches_oracle_every_step():
+    rep = hx.run_decode(gen.SHAPES["tiny"], 32, np.arange(2))
+    _check_decode(rep)
+
+
+def test_tiny_eager_matches_oracle_every_step():
+    rep = hx.run_eager(gen.SHAPES["tiny"], 32, np.arange(2))
+    assert rep.max_err <= hx.TOL_F32 and rep.ckpt_err <= hx.TOL_F32, (rep.max_err, rep.ckpt_err)
+
+
+RAGGED = [
+    # groups shared by heads, ragged window, ring wrap-around, FP32 I/O
+    gen.Shape("r1", B=3, H=4, G=2, P=24, N=32, L=5, io="f32", seed=11),
+    # BF16 I/O, three heads per group, P not a multiple of the rows one pass covers
+    gen.Shape("r2", B=5, H=6, G=2, P=40, N=64, L=7, io="bf16", seed=12),
+    # several row groups with a ragged tail (N = 128: 64 rows per group)
+    gen.Shape("r3", B=2, H=3, G=3, P=136, N=128, L=6, io="bf16", seed=13),
+    # window of one: every step folds the previous token
+    gen.Shape("r4", B=2, H=2, G=2, P=8, N=16, L=1, io="f32", seed=14),
+    # one head, one group, prefill-shaped checkpoint
+    gen.Shape("r5", B=4, H=1, G=1, P=64, N=128, L=16, io="bf16", s0="prefill", seed=15),
+]
+
+
+@pytest.mark.parametrize("shape", RAGGED, ids=[s.name for s in RAGGED])
+def test_ragged_shapes_match_oracle(shape):
+    steps = 3 * shape.L + 4
+    rep = hx.run_decode(shape, steps, np.arange(shape.B))
+    _check_decode(rep)
+
+
+@pytest.mark.parametrize("shape", RAGGED[:3], ids=[s.name for s in RAGGED[:3]])
+def test_ragged_eager_matches_oracle(shape):
+    rep = hx.run_eager(shape, 9, np.arange(shape.B))
+    assert rep.max_err <= hx.TOL_F32 and rep.ckpt_err <= hx.TOL_F32, (rep.max_err, rep.ckpt_err)
+
+
+SPEC = [
+    gen.Shape("s1", B=4, H=4, G=2, P=16, N=32, L=8, io="bf16", max_pos=5, seed=21),
+    gen.Shape("s2", B=3, H=2, G=2, P=24, N=16, L=5, io="f32", max_pos=5, seed=22),
+    gen.Shape("s3", B=2, H=2, G=1, P=64, N=128, L=16, io="bf16", max_pos=8, seed=23),
+]
+
+
+@pytest.mark.parametrize("shape", SPEC, ids=[s.name for s in SPEC])
+def test_verify_rollback_match_oracle(shape):
+    rep = hx.run_spec(shape, 14, np.arange(shape.B), steps_after=shape.L + 2)
+    _check_decode(rep)
+
+
+@pytest.mark.parametrize("n_pos", [1, 2, 3])
+def test_verify_with_fewer_positions(n_pos):
+    shape = gen.Shape("s4", B=3, H=2, G=2, P=16, N=64, L=6, io="f32", max_pos=4, seed=24)
+    rep = hx.run_spec(shape, 9, np.arange(shape.B), n_pos=n_pos, steps_after=3)
+    _check_decode(rep)
+
+
+def test_fp8_read_copy_small():
+    shape = gen.Shape("f1", B=3, H=2, G=2, P=32, N=64, L=4, io="f32", ckpt="f32_fp8read", seed=31)
+    rep = hx.run_decode(shape, 21, np.arange(shape.B), fp8_emulation=True)
+    assert rep.max_err <= hx.TOL_FP8, rep.max_err
+    assert rep.max_err_fp8_emul <= 1e-3, rep.max_err_fp8_emul
+    assert rep.flags_equal and rep.counts_equal
+    assert rep.ckpt_err <= hx.TOL_F32  # the master never sees FP8 rounding
+
+
+def test_fp8_init_copy_bit_exact():
+    shape = gen.Shape("f2", B=2, H=3, G=3, P=16, N=128, L=4, io="bf16", ckpt="f32_fp8read", seed=32)
+    cfg, bufs, r, S0 = hx.setup(shape)
+    torch.cuda.synchronize()
+    codes, scale = ro.quantize_rows_e4m3(S0.cpu().numpy())
+    np.testing.assert_array_equal(bufs["S0_fp8"].cpu().numpy(), codes)
+    np.testing.assert_array_equal(bufs["S0_scale"].cpu().numpy(), scale)
+    r.close()
+
+
+def test_eager_fp8_small():
+    shape = gen.Shape("f3", B=2, H=2, G=2, P=32, N=64, L=4, io="f32", seed=33)
+    rep = hx.run_eager(shape, 12, np.arange(shape.B), fp8=True)
+    assert rep.max_err <= 1e-3, rep.max_err
+
+
+# ------------------------------------------------------------------ protocol and error paths
+
+def test_flush_mask_folds_only_selected_sequences():
+    shape = gen.Shape("m1", B=4, H=2, G=1, P=16, N=32, L=8, io="f32", seed=41)
+    cfg, bufs, r, S0 = hx.setup(shape)
+    rows = np.arange(shape.B)
+    ref = ro.ReplayBatch(gen.to_numpy64(S0), shape.G, shape.L)
+    for t in range(5):
+        x = gen.step_inputs(shape, t, device="cuda")
+        r.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
+        xs = {k: gen.to_numpy64(v) for k, v in x.items()}
+        ref.step(xs["q"], xs["k"], xs["v"], xs["dt"], xs["a"])
+    mask = torch.tensor([1, 0, 1, 0], dtype=torch.uint8, device="cuda")
+    r.flush(mask)
+    ref.flush(mask.cpu().numpy())
+    assert r.read_counts() == [0, 5, 0, 5] == list(ref.counts)
+    assert ro.relative_error(gen.to_numpy64(bufs["S0"]), ref.checkpoints()) <= hx.TOL_F32
+    for t in range(5, 12):  # decoding continues correctly from the mixed state
+        x = gen.step_inputs(shape, t, device="cuda")
+        y = r.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
+        xs = {k: gen.to_numpy64(v) for k, v in x.items()}
+        y_ref, _ = ref.step(xs["q"], xs["k"], xs["v"], xs["dt"], xs["a"])
+        assert ro.relative_error(gen.to_numpy64(y), y_ref) <= hx.TOL_F32
+    assert r.read_counts() == list(ref.counts)
+    assert r.check_status() == 0
+    del rows
+
+
+def test_protocol_errors():
+    shape = gen.Shape("e1", B=2, H=2, G=2, P=16, N=16, L=4, io="f32", max_pos=3, seed=42)
+    cfg, bufs, r, S0 = hx.setup(shape)
+    x = gen.step_inputs(shape, 0, device="cuda")
+    with pytest.raises(lar.ReplayError) as e:
+        r.rollback(torch.ones(2, dtype=torch.int32, device="cuda"))
+    assert e.value.code == _abi.REPLAY_ENOPENDING
+    xv = gen.verify_inputs(shape, 0, 3, device="cuda")
+    r.verify(xv["q"], xv["k"], xv["v"], xv["dt"], xv["a"])
+    for call in (lambda: r.step(x["q"], x["k"], x["v"], x["dt"], x["a"]),
+                 lambda: r.verify(xv["q"], xv["k"], xv["v"], xv["dt"], xv["a"]),
+                 lambda: r.flush()):
+        with pytest.raises(lar.ReplayError) as e:
+            call()
+        assert e.value.code == _abi.REPLAY_EPENDING
+    # an out-of-range n_keep is reported on the device and keeps none of the drafts
+    r.rollback(torch.tensor([2, 7], dtype=torch.int32, device="cuda"))
+    assert r.read_counts() == [2, 0]
+    assert r.check_status() == lar.DEV_ROLLBACK
+    xv4 = gen.verify_inputs(shape, 1, 4, device="cuda")
+    with pytest.raises(lar.ReplayError) as e:
+        r.verify(xv4["q"], xv4["k"], xv4["v"], xv4["dt"], xv4["a"])
+    assert e.value.code == _abi.REPLAY_EINVAL
+    r.close()
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_mamba2_b256_decode_sampled():
+    """B=256, H=64, P=64, N=128, L=16, BF16 I/O, FP32 checkpoint, 512 steps (32
+    windows): 8 sampled sequences against the oracle every step, counts and flush
+    flags of all 256 sequences bit-exact."""
+    shape = gen.SHAPES["mamba2_b256"]
+    rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 8))
+    _check_decode(rep)
+    assert rep.max_err <= hx.TOL_BF16
+
+
+def test_mamba2_b256_fp8_sampled():
+    """Dual precision at full size over 2048 steps: FP8 read copy vs the unquantised
+    oracle (6e-2), vs the oracle's FP8 emulation, and the shared-FP8 eager error beside it."""
+    shape = gen.SHAPES["mamba2_b256_fp8"]
+    rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 3), fp8_emulation=True,
+                        shared_fp8=True)
+    assert rep.max_err <= hx.TOL_FP8, rep.max_err
+    assert rep.max_err_fp8_emul <= 1e-2, rep.max_err_fp8_emul
+    assert rep.flags_equal and rep.counts_equal
+    assert rep.ckpt_err <= hx.TOL_F32
+    print(f"fp8 read err {rep.max_err:.3e}  vs emulation {rep.max_err_fp8_emul:.3e}  "
+          f"shared-fp8 eager err {rep.max_err_shared_fp8:.3e}")
+
+
+def test_mamba2_b256_spec_sampled():
+    """Verify (5 positions) + rollback (accepted ~ U{0..4}) for 256 rounds at full size."""
+    shape = gen.SHAPES["mamba2_b256_spec"]
+    rep = hx.run_spec(shape, shape.steps, hx.sample_rows(shape.B, 6))
+    _check_decode(rep)
+
+
+SWEEP = [s for s in gen.sweep_shapes() if (s.B, s.L) in ((1, 4), (16, 32), (1024, 16), (64, 8))]
+
+
+@pytest.mark.parametrize("shape", SWEEP, ids=[s.name for s in SWEEP])
+def test_sweep_points_sampled(shape):
+    steps = 2 * shape.L + 3
+    rep = hx.run_decode(shape, steps, hx.sample_rows(shape.B, 3))
+    _check_decode(rep)
+    eag = hx.run_eager(shape, 3, hx.sample_rows(shape.B, 3))
+    assert eag.max_err <= hx.TOL_F32

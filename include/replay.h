@@ -74,7 +74,7 @@ typedef struct {
   int32_t groups;  /* G >= 1, H % G == 0 (k and q are shared by the H/G heads of a group) */
   int32_t P;       /* v-dim: multiple of 8, 8..256 */
   int32_t N;       /* k-dim: 16, 32, 64 or 128 */
-  int32_t L;       /* window: buffer entries between checkpoint flushes, 1..64 */
+  int32_t L;       /* window: buffer entries between checkpoint flushes, 1..32 */
   int32_t max_pos; /* largest n_pos of replay_verify, 1..8 and <= L (1 = plain decode) */
   int32_t io;      /* replay_dtype of q, k, v and of the ring of k, v */
   int32_t ckpt;    /* replay_ckpt */

@@ -27,7 +27,8 @@ struct replay_ctx {
 
 namespace {
 
-constexpr int kHeaderBytes = 256;  // 2 * kMaxStages mbarriers + abort flag
+constexpr int kHeaderBytes = 256;  // the kernel's mbarriers and abort flag
+constexpr int kGroups = 2;         // consumer groups per CTA (must match the launcher)
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -41,7 +42,7 @@ int validate_config(const replay_config* c, bool needs_window) {
   if (c->io != REPLAY_F32 && c->io != REPLAY_BF16) return REPLAY_EINVAL;
   if ((int64_t)c->batch * c->heads > INT32_MAX / 2) return REPLAY_EINVAL;
   if (needs_window) {
-    if (c->L < 1 || c->L > 64) return REPLAY_EINVAL;
+    if (c->L < 1 || c->L > replay::kMaxWindow) return REPLAY_EINVAL;
     if (c->max_pos < 1 || c->max_pos > replay::kMaxPos || c->max_pos > c->L) return REPLAY_EINVAL;
     if (c->ckpt != REPLAY_CKPT_F32 && c->ckpt != REPLAY_CKPT_F32_FP8READ) return REPLAY_EINVAL;
   }
@@ -97,17 +98,18 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->off_meta = p->off_an + replay::kMaxPos * 4;
   p->stage_bytes = round_up(p->off_meta + 16, 128);
 
-  p->jw = round_up(c.L + c.max_pos + 1, 4);
+  // one workspace per consumer group: decay weights and k.q of the outputs
+  // [kMaxPos][kMaxWindow] each, alpha[kMaxPos], fold weights [kMaxWindow] + abar, and the
+  // fold weights times v, [P][fp]
   p->fp = round_up(lfold, replay::kFoldChunk);
   p->ws_w = 0;
-  p->ws_kq = p->ws_w + replay::kMaxPos * p->jw * 4;
-  p->ws_alpha = p->ws_kq + replay::kMaxPos * p->jw * 4;
+  p->ws_kq = p->ws_w + replay::kMaxPos * replay::kMaxWindow * 4;
+  p->ws_alpha = p->ws_kq + replay::kMaxPos * replay::kMaxWindow * 4;
   p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
-  p->ws_wt = round_up(p->ws_sig + (p->jw + 4) * 4, 16);
-  p->ws_bt = p->ws_wt + P * p->fp * 4;
-  const int ws_bytes = round_up(p->ws_bt + replay::kMaxPos * P * 4, 128);
+  p->ws_wt = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
+  p->ws_group_bytes = round_up(p->ws_wt + P * p->fp * 4, 128);
   p->ws_off = kHeaderBytes;
-  p->stages_off = round_up(kHeaderBytes + ws_bytes, 128);
+  p->stages_off = round_up(p->ws_off + kGroups * p->ws_group_bytes, 128);
   const int avail = smem_optin - p->stages_off;
   int ns = avail / p->stage_bytes;
   if (ns > replay::kMaxStages) ns = replay::kMaxStages;

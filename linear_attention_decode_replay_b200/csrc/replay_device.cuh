@@ -10,13 +10,13 @@
 
 namespace replay {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kConsumerWarps = 8;               // warps that compute units (split into groups)
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kMaxPos = 8;                       // query positions per verify call
+constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
 constexpr int kMaxStages = 8;
 constexpr int kFoldChunk = 8;                    // buffer entries folded per register pass
-constexpr int kRowsPerThread = 8;                // state rows one thread covers per row group
+constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 
 // status word bits (device-detected errors; the host reads them with replay_check_status)
@@ -76,21 +76,21 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
-// ---------------------------------------------------------------- consumer-only barriers
-// Named barrier 1 spans the consumer warps only (the producer warp never joins it).
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+// ---------------------------------------------------------------- consumer-group barriers
+// Named barrier `id` (1 + group) spans the `count` threads of one consumer group only.
+__device__ __forceinline__ void group_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-// Barrier with an AND-vote across the consumer threads.
-__device__ __forceinline__ bool consumer_all(bool v) {
+// Group barrier with an AND-vote across the group's threads.
+__device__ __forceinline__ bool group_all(bool v, int id, int count) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v), "n"(kConsumerThreads)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
       : "memory");
   return r != 0;
 }
@@ -105,6 +105,7 @@ struct IoT<float> {
     return *reinterpret_cast<const float4*>(p);
   }
   __device__ __forceinline__ static float load1(const void* p) { return *reinterpret_cast<const float*>(p); }
+  __device__ __forceinline__ static float2 load2(const void* p) { return *reinterpret_cast<const float2*>(p); }
 };
 template <>
 struct IoT<__nv_bfloat16> {
@@ -119,6 +120,9 @@ struct IoT<__nv_bfloat16> {
   }
   __device__ __forceinline__ static float load1(const void* p) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+  }
+  __device__ __forceinline__ static float2 load2(const void* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
   }
 };
 
@@ -155,6 +159,17 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
 }
 __device__ __forceinline__ float amax4(float4 a) {
   return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+}
+
+// ---------------------------------------------------------------- warp scans
+// Inclusive suffix product over the lanes of a warp: lane l gets x_l * x_{l+1} * ... * x_31.
+__device__ __forceinline__ float warp_suffix_prod(float x, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float t = __shfl_down_sync(0xffffffffu, x, off);
+    if (lane + off < 32) x *= t;
+  }
+  return x;
 }
 
 // ---------------------------------------------------------------- segment reductions
@@ -198,6 +213,15 @@ struct SegTranspose {
     }
   }
 };
+template <int R>
+struct SegLog2 {
+  static constexpr int value = (R <= 1) ? 0 : 1 + SegLog2<R / 2>::value;
+};
+template <>
+struct SegLog2<1> {
+  static constexpr int value = 0;
+};
+
 template <int R, int TPR>
 struct SegReduce {
   static constexpr int kHeld = (R >= TPR) ? R / TPR : 1;  // row sums each lane ends with

@@ -1,15 +1,19 @@
 // Persistent, warp-specialised kernel for the ReplaySSM decode path on sm_100a.
 //
 // One launch processes every (sequence b, head h) unit of a decode layer. Each CTA owns
-// the units blockIdx.x, blockIdx.x + gridDim.x, ... and runs them through a ring of
+// the units blockIdx.x, blockIdx.x + gridDim.x, ... and streams them through a ring of
 // shared-memory stages:
 //   * the producer warp reads the unit's buffer pointer word (prefetched one unit
-//     ahead), then issues 1-D bulk copies (TMA) of the unit's checkpoint tile S0[b,h]
-//     (P x N, FP32 master or FP8 read copy + per-row scales), of the live ring-buffer
-//     entries (k, v, Delta, a) and of this call's new inputs into a stage, completing
-//     on that stage's "full" mbarrier;
-//   * the eight consumer warps wait on "full", compute the unit, and release the stage
-//     through its "empty" mbarrier.
+//     ahead) and issues, one copy per lane in a single instruction, the 1-D bulk copies
+//     (TMA) of the unit's checkpoint tile S0[b,h] (P x N, FP32 master or FP8 read copy +
+//     per-row scales), of the live ring-buffer entries (k, v, Delta, a) and of this
+//     call's new tokens into a stage, completing on that stage's "full" mbarrier;
+//   * NG consumer groups (8/NG warps each) take alternate units end to end: decay
+//     scans and k_j . q_s products spread over the group's warps, then the state rows
+//     (output-only dot products, or the fused fold and its write-back), then the ring
+//     append; each group releases the stage through its "empty" mbarrier. Two groups
+//     keep two units in flight, so one unit's short dependent chains overlap the
+//     other's.
 // The state is streamed exactly once per call; every other byte is small.
 //
 // What a unit computes (blog "ReplaySSM: Cachear Inputs, No Estado": routes "estado y
@@ -24,9 +28,9 @@
 //   EAGER (baseline): S <- a S + Delta v k^T, y = S q, the state read and written every
 //     call (FP32, or a shared FP8 state re-quantised every call).
 //
-// Thread layout inside a unit: a state row of N floats is covered by TPR = N/4 lanes,
-// four columns each; 256 consumer threads cover RPP = 256/TPR rows per pass and each
-// thread takes kRowsPerThread rows of a row group.
+// Row layout inside a group: a state row of N floats is covered by TPR = N/4 lanes, four
+// columns each; the group covers 32/TPR rows per warp per pass, and each thread takes
+// kRowsPerThread rows of a row group.
 #pragma once
 
 #include "replay_device.cuh"
@@ -37,6 +41,20 @@ namespace replay {
 __device__ __forceinline__ void report_error(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }
+
+template <int NG>
+struct Groups {
+  static constexpr int kWarps = kConsumerWarps / NG;  // warps per consumer group
+  static constexpr int kThreads = kWarps * 32;
+};
+
+// barriers at the start of shared memory
+struct Bars {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "the barrier header must fit the 256 bytes the host layout reserves");
 
 struct Plan {
   int b, h, g, start, c;
@@ -58,7 +76,7 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
     pl.corrupt = false;
     pl.active = true;
     pl.fp32_tile = (CKPT == kCkptF32);
-    uint32_t tile = pl.fp32_tile ? P * N * 4u : P * N + P * 4u;
+    const uint32_t tile = pl.fp32_tile ? P * N * 4u : P * N + P * 4u;
     pl.bytes = tile + 2u * N * S_IO + P * S_IO;
     return pl;
   }
@@ -85,54 +103,116 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
   return pl;
 }
 
+// Entry j of the unit's buffer view: j < c are ring entries (slot start + j modulo cap),
+// j >= c are this call's new tokens. Eager units have only the new token (j = 0).
+template <int MODE>
+struct EntryScalars {
+  const float *dtr, *ar, *dtn, *an;
+  int start, cap, c;
+  __device__ __forceinline__ int slot(int j) const {
+    int s = start + j;
+    return s - ((s >= cap) ? cap : 0);
+  }
+  __device__ __forceinline__ float dt(int j) const {
+    if (MODE == kModeEager) return dtn[j];
+    return j < c ? dtr[slot(j)] : dtn[j - c];
+  }
+  __device__ __forceinline__ float a(int j) const {
+    if (MODE == kModeEager) return an[j];
+    return j < c ? ar[slot(j)] : an[j - c];
+  }
+};
+
 // ---------------------------------------------------------------------------- producer
+// Each lane issues at most one of the unit's copies: lane 0 the state tile, lane 1 the
+// FP8 row scales, lanes 2-5 the ring k and v pieces, lanes 6-7 the Delta and a rings,
+// lanes 8 + 3s .. 10 + 3s the new q, k, v of position s.
 template <int MODE, int CKPT, int S_IO>
-__device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& pl, uint8_t* st,
-                                                  uint64_t* bar) {
+__device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& pl, uint8_t* st, uint64_t* bar,
+                                                  int lane) {
   const size_t P = p.P, N = p.N;
   const size_t bh = (size_t)pl.b * p.H + pl.h;
-  uint8_t* tile = st;
-  if (pl.fp32_tile) {
-    bulk_g2s(tile, p.S + bh * P * N, (uint32_t)(P * N * 4), bar);
-  } else {
-    bulk_g2s(tile, p.S8 + bh * P * N, (uint32_t)(P * N), bar);
-    bulk_g2s(tile + P * N, p.Sscale + bh * P, (uint32_t)(P * 4), bar);
-  }
   const int n_new = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int c = pl.c;
   uint8_t* kbuf = st + p.off_k;
   uint8_t* vbuf = st + p.off_v;
-  if (c > 0) {
-    // live ring entries [start, start + c) modulo cap, in one or two pieces
-    const int first = min(c, p.cap - pl.start);
-    const int second = c - first;
-    const uint8_t* rk = static_cast<const uint8_t*>(p.ring_k) + ((size_t)pl.b * p.G + pl.g) * p.cap * N * S_IO;
-    const uint8_t* rv = static_cast<const uint8_t*>(p.ring_v) + bh * p.cap * P * S_IO;
-    bulk_g2s(kbuf, rk + (size_t)pl.start * N * S_IO, (uint32_t)(first * N * S_IO), bar);
-    bulk_g2s(vbuf, rv + (size_t)pl.start * P * S_IO, (uint32_t)(first * P * S_IO), bar);
-    if (second > 0) {
-      bulk_g2s(kbuf + (size_t)first * N * S_IO, rk, (uint32_t)(second * N * S_IO), bar);
-      bulk_g2s(vbuf + (size_t)first * P * S_IO, rv, (uint32_t)(second * P * S_IO), bar);
+  void* dst = nullptr;
+  const void* src = nullptr;
+  uint32_t bytes = 0;
+  if (lane == 0) {
+    dst = st;
+    if (pl.fp32_tile) {
+      src = p.S + bh * P * N;
+      bytes = (uint32_t)(P * N * 4);
+    } else {
+      src = p.S8 + bh * P * N;
+      bytes = (uint32_t)(P * N);
     }
-    bulk_g2s(st + p.off_dtr, p.ring_dt + bh * p.cap, (uint32_t)(p.cap * 4), bar);
-    bulk_g2s(st + p.off_ar, p.ring_a + bh * p.cap, (uint32_t)(p.cap * 4), bar);
-  }
-  if (n_new > 0) {
-    const uint8_t* q = static_cast<const uint8_t*>(p.q);
-    const uint8_t* k = static_cast<const uint8_t*>(p.k);
-    const uint8_t* v = static_cast<const uint8_t*>(p.v);
-    for (int s = 0; s < n_new; ++s) {
+  } else if (lane == 1) {
+    if (!pl.fp32_tile) {
+      dst = st + P * N;
+      src = p.Sscale + bh * P;
+      bytes = (uint32_t)(P * 4);
+    }
+  } else if (lane < 8) {
+    if (c > 0) {
+      // live ring entries [start, start + c) modulo cap, in one or two pieces
+      const int first = min(c, p.cap - pl.start);
+      const int second = c - first;
+      const uint8_t* rk = static_cast<const uint8_t*>(p.ring_k) + ((size_t)pl.b * p.G + pl.g) * p.cap * N * S_IO;
+      const uint8_t* rv = static_cast<const uint8_t*>(p.ring_v) + bh * p.cap * P * S_IO;
+      if (lane == 2) {
+        dst = kbuf;
+        src = rk + (size_t)pl.start * N * S_IO;
+        bytes = (uint32_t)(first * N * S_IO);
+      } else if (lane == 3 && second > 0) {
+        dst = kbuf + (size_t)first * N * S_IO;
+        src = rk;
+        bytes = (uint32_t)(second * N * S_IO);
+      } else if (lane == 4) {
+        dst = vbuf;
+        src = rv + (size_t)pl.start * P * S_IO;
+        bytes = (uint32_t)(first * P * S_IO);
+      } else if (lane == 5 && second > 0) {
+        dst = vbuf + (size_t)first * P * S_IO;
+        src = rv;
+        bytes = (uint32_t)(second * P * S_IO);
+      } else if (lane == 6) {
+        dst = st + p.off_dtr;
+        src = p.ring_dt + bh * p.cap;
+        bytes = (uint32_t)(p.cap * 4);
+      } else if (lane == 7) {
+        dst = st + p.off_ar;
+        src = p.ring_a + bh * p.cap;
+        bytes = (uint32_t)(p.cap * 4);
+      }
+    }
+  } else {
+    const int t = lane - 8;
+    const int s = t / 3;
+    if (s < n_new) {
       const size_t tok = (size_t)pl.b * n_new + s;
-      bulk_g2s(st + p.off_q + (size_t)s * N * S_IO, q + (tok * p.G + pl.g) * N * S_IO, (uint32_t)(N * S_IO), bar);
-      bulk_g2s(kbuf + (size_t)(c + s) * N * S_IO, k + (tok * p.G + pl.g) * N * S_IO, (uint32_t)(N * S_IO), bar);
-      bulk_g2s(vbuf + (size_t)(c + s) * P * S_IO, v + (tok * p.H + pl.h) * P * S_IO, (uint32_t)(P * S_IO), bar);
+      const int which = t - 3 * s;
+      if (which == 0) {
+        dst = st + p.off_q + (size_t)s * N * S_IO;
+        src = static_cast<const uint8_t*>(p.q) + (tok * p.G + pl.g) * N * S_IO;
+        bytes = (uint32_t)(N * S_IO);
+      } else if (which == 1) {
+        dst = kbuf + (size_t)(c + s) * N * S_IO;
+        src = static_cast<const uint8_t*>(p.k) + (tok * p.G + pl.g) * N * S_IO;
+        bytes = (uint32_t)(N * S_IO);
+      } else {
+        dst = vbuf + (size_t)(c + s) * P * S_IO;
+        src = static_cast<const uint8_t*>(p.v) + (tok * p.H + pl.h) * P * S_IO;
+        bytes = (uint32_t)(P * S_IO);
+      }
     }
   }
+  if (bytes) bulk_g2s(dst, src, bytes, bar);
 }
 
 template <int MODE, int CKPT, int S_IO>
-__device__ void producer_loop(const KParams& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
-                              volatile int* abort_flag) {
+__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   const int lane = threadIdx.x & 31;
   const int NS = p.num_stages;
   const int n_new = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
@@ -156,19 +236,18 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, uint64_t* full,
     const int s = i % NS;
     const int k = i / NS;
     if (k > 0) {
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait_bounded(&empty[s], (k - 1) & 1);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // every lane waits (each lane then writes into the stage), the warp agrees
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1));
       if (!ok) {
         if (lane == 0) {
           report_error(p.status, kErrWaitTimeout);
-          *abort_flag = 1;
+          bars->abort_flag = 1;
         }
         break;
       }
     }
-    int ab = (lane == 0) ? *abort_flag : 0;  // one lane reads, the warp decides together
-    if (__shfl_sync(0xffffffffu, ab, 0)) break;
+    int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
+    if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
     const int32_t word = __shfl_sync(0xffffffffu, w_next, 0);
     const int msk = __shfl_sync(0xffffffffu, m_next, 0);
     const float dtv = dt_next, av = a_next;
@@ -186,9 +265,10 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, uint64_t* full,
     __syncwarp();
     if (lane == 0) {
       if (pl.corrupt) report_error(p.status, kErrPointer);
-      mbar_arrive_expect_tx(&full[s], pl.bytes);
-      if (pl.bytes) issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &full[s]);
+      mbar_arrive_expect_tx(&bars->full[s], pl.bytes);
     }
+    __syncwarp();
+    if (pl.bytes) issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane);
     __syncwarp();
   }
   // Never leave with copies in flight into this CTA's shared memory: wait (bounded) for
@@ -196,147 +276,179 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, uint64_t* full,
   if (lane == 0) {
     const int first = i > NS ? i - NS : 0;
     for (int j = first; j < i; ++j) {
-      if (!mbar_wait_bounded(&full[j % NS], (j / NS) & 1)) report_error(p.status, kErrWaitTimeout);
+      if (!mbar_wait_bounded(&bars->full[j % NS], (j / NS) & 1)) report_error(p.status, kErrWaitTimeout);
     }
   }
 }
 
-// ---------------------------------------------------------------------------- consumer
-template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, uint8_t* st, uint8_t* ws,
-                                             int ctid) {
+// ---------------------------------------------------------------------------- consumers
+// kq[s][jj] = k_{o0+jj} . q_s for every query s < n and entry jj < width (<= 32).
+template <int N, typename IO, int GW>
+__device__ __forceinline__ void entry_dots(const uint8_t* kbuf, const uint8_t* qbuf, int o0, int width, int n,
+                                           float* kq, int gw, int lane) {
+  constexpr int S_IO = IoT<IO>::bytes;
+  if constexpr (N == 128) {
+    // a warp per (query, 8 entries): the lanes split N, a transposing reduction sums them
+    const int chunks = (width + 7) / 8;
+    for (int t = gw; t < n * chunks; t += GW) {
+      const int s = t / chunks;
+      const int ch = t - s * chunks;
+      const float4 qv = IoT<IO>::load4(qbuf + ((size_t)s * N + lane * 4) * S_IO);
+      float part[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int jj = ch * 8 + r;
+        part[r] = (jj < width) ? dot4(IoT<IO>::load4(kbuf + ((size_t)(o0 + jj) * N + lane * 4) * S_IO), qv) : 0.f;
+      }
+      int base;
+      const bool wr = SegReduce<8, 32>::run(part, lane, base);
+      const int jj = ch * 8 + base;
+      if (wr && jj < width) kq[s * kMaxWindow + jj] = part[0];
+    }
+  } else {
+    // short rows: a lane per (query, entry)
+    for (int t = gw * 32 + lane; t < n * width; t += GW * 32) {
+      const int s = t / width;
+      const int jj = t - s * width;
+      const uint8_t* kr = kbuf + (size_t)(o0 + jj) * N * S_IO;
+      const uint8_t* qr = qbuf + (size_t)s * N * S_IO;
+      float d = 0.f;
+#pragma unroll
+      for (int c4 = 0; c4 < N; c4 += 4) d += dot4(IoT<IO>::load4(kr + (size_t)c4 * S_IO), IoT<IO>::load4(qr + (size_t)c4 * S_IO));
+      kq[s * kMaxWindow + jj] = d;
+    }
+  }
+}
+
+template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
+__device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, uint8_t* st, uint8_t* ws, int gtid,
+                                             int bar_id) {
+  using Gr = Groups<NG>;
+  constexpr int GT = Gr::kThreads;
+  constexpr int GW = Gr::kWarps;
   constexpr int TPR = N / 4;
-  constexpr int RPP = kConsumerThreads / TPR;
+  constexpr int RPW = 32 / TPR;  // rows per warp pass
+  constexpr int RPG = GW * RPW;  // rows per group pass
   constexpr int RT = kRowsPerThread;
-  constexpr int RG = RPP * RT;
+  constexpr int RGR = RPG * RT;  // rows per row group
   constexpr int S_IO = IoT<IO>::bytes;
   using Red = SegReduce<RT, TPR>;
-  const int lane = ctid & 31;
-  const int row0 = ctid / TPR;
-  const int col = (ctid % TPR) * 4;
+  const int lane = gtid & 31;
+  const int gw = gtid >> 5;
+  const int row0 = gw * RPW + lane / TPR;
+  const int col = (lane % TPR) * 4;
   const int P = p.P;
   const int c = pl.c;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
-  const int o0 = pl.fold ? c : 0;  // first entry the outputs read from the buffer (replay)
-  const int J = c + n;
-  const int jw = p.jw;
+  const int o0 = pl.fold ? c : 0;                                // first entry the outputs read
+  const int width = c + n - o0;                                  // entries the outputs read
   const int fp = p.fp;
-
   const uint8_t* tile = st;
   const uint8_t* kbuf = st + p.off_k;
   const uint8_t* vbuf = st + p.off_v;
   const uint8_t* qbuf = st + p.off_q;
-  const float* dtr = reinterpret_cast<const float*>(st + p.off_dtr);
-  const float* ar = reinterpret_cast<const float*>(st + p.off_ar);
-  const float* dtn = reinterpret_cast<const float*>(st + p.off_dtn);
-  const float* an = reinterpret_cast<const float*>(st + p.off_an);
-  float* wout = reinterpret_cast<float*>(ws + p.ws_w);    // [kMaxPos][jw] output weights
-  float* kq = reinterpret_cast<float*>(ws + p.ws_kq);     // [kMaxPos][jw] k_j . q_s
+  const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
+  float* wout = reinterpret_cast<float*>(ws + p.ws_w);     // [kMaxPos][kMaxWindow] decay weight of entry o0+jj
+  float* kq = reinterpret_cast<float*>(ws + p.ws_kq);      // [kMaxPos][kMaxWindow] k_{o0+jj} . q_s
   float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);
-  float* sig = reinterpret_cast<float*>(ws + p.ws_sig);   // [jw] fold weights, [jw] = abar
-  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);     // [P][fp] fold weight * v_j[p]
-  float* bt = reinterpret_cast<float*>(ws + p.ws_bt);     // [kMaxPos][P] buffer term of y
-  const int start = pl.start;
-  const int cap = p.cap;
-  auto dt_of = [&](int j) -> float {
-    if (MODE == kModeEager) return dtn[j];
-    int slot = start + j;
-    slot -= (slot >= cap) ? cap : 0;
-    return j < c ? dtr[slot] : dtn[j - c];
-  };
-  auto a_of = [&](int j) -> float {
-    if (MODE == kModeEager) return an[j];
-    int slot = start + j;
-    slot -= (slot >= cap) ? cap : 0;
-    return j < c ? ar[slot] : an[j - c];
-  };
+  float* sig = reinterpret_cast<float*>(ws + p.ws_sig);    // fold weights; [kMaxWindow] = abar
+  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);      // [P][fp] fold weight times v_j[p]
+  const EntryScalars<MODE> es{reinterpret_cast<const float*>(st + p.off_dtr), reinterpret_cast<const float*>(st + p.off_ar),
+                              reinterpret_cast<const float*>(st + p.off_dtn), reinterpret_cast<const float*>(st + p.off_an),
+                              pl.start, p.cap, c};
+  const size_t bh = (size_t)pl.b * p.H + pl.h;
+  const int ngroups = (P + RGR - 1) / RGR;
 
-  // ---- phase 1: decay weights (one thread per query, one for the fold) and k_j . q_s
-  if (MODE == kModeReplay) {
-    if (ctid < n) {
-      const int s = ctid;
-      float run = 1.f;
-      for (int j = c + s; j >= o0; --j) {
-        wout[s * jw + j] = dt_of(j) * run;
-        run *= a_of(j);
-      }
-      alpha[s] = run;
-    }
-  } else if (MODE == kModeEager) {
-    if (ctid == 0) alpha[0] = 1.f;
-  }
-  if (cf > 0 && ctid == 32) {
-    float run = 1.f;
-    for (int j = cf - 1; j >= 0; --j) {
-      sig[j] = dt_of(j) * run;
-      run *= a_of(j);
-    }
-    sig[jw] = run;
-  }
-  if (MODE == kModeReplay) {
-    const int width = J - o0;
-    const int npairs = n * width;
-    const int iters = (npairs + RPP - 1) / RPP;
-    for (int it = 0; it < iters; ++it) {
-      const int pi = it * RPP + row0;
-      const bool valid = pi < npairs;
-      float d = 0.f;
-      int s = 0, j = 0;
-      if (valid) {
-        s = pi / width;
-        j = o0 + (pi - s * width);
-        const float4 kk = IoT<IO>::load4(kbuf + ((size_t)j * N + col) * S_IO);
-        const float4 qq = IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO);
-        d = dot4(kk, qq);
-      }
-      d = seg_allsum<TPR>(d);
-      if (valid && (ctid % TPR) == 0) kq[s * jw + j] = d;
-    }
-  }
-  consumer_sync();
-
-  // ---- phase 2: buffer term of every output, and fold weights times v
-  if (MODE == kModeReplay) {
-    for (int idx = ctid; idx < n * P; idx += kConsumerThreads) {
-      const int s = idx / P;
-      const int pp = idx - s * P;
-      float acc = 0.f;
-      for (int j = o0; j <= c + s; ++j)
-        acc = fmaf(wout[s * jw + j] * kq[s * jw + j], IoT<IO>::load1(vbuf + ((size_t)j * P + pp) * S_IO), acc);
-      bt[s * P + pp] = acc;
-    }
-  }
-  const int cf_pad = (cf + kFoldChunk - 1) / kFoldChunk * kFoldChunk;
-  if (cf > 0) {
-    for (int idx = ctid; idx < P * cf_pad; idx += kConsumerThreads) {
-      const int pp = idx / cf_pad;
-      const int j = idx - pp * cf_pad;
-      wt[pp * fp + j] = j < cf ? sig[j] * IoT<IO>::load1(vbuf + ((size_t)j * P + pp) * S_IO) : 0.f;
-    }
-  }
-  consumer_sync();
-
-  // ---- phase 3: stream the state rows
   float4 qr[NQ > 0 ? NQ : 1];
 #pragma unroll
   for (int s = 0; s < NQ; ++s)
     qr[s] = (s < n) ? IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
-  const size_t bh = (size_t)pl.b * p.H + pl.h;
-  const int ngroups = (P + RG - 1) / RG;
-  const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
 
+  // state rows of a row group; the first group is loaded before the scans so that its
+  // shared-memory latency overlaps them
+  auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const int pr = gi * RGR + row0 + RPG * r;
+      x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pr < P) {
+        if (pl.fp32_tile) {
+          x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
+        } else {
+          const float4 e = e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
+          if (dequant) {  // eager on a shared FP8 state: dequantise
+            const float sc = scale_tile[pr];
+            x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
+          } else {
+            x[r] = e;  // read copy: the row scale is applied to the dot product
+          }
+        }
+      }
+    }
+  };
+  float4 x[RT];
+  load_rows(x, 0, MODE == kModeEager);
+
+  // ---- phase A: decay scans (a warp per task) and k_j . q_s products
+  {
+    const int tasks = ((MODE == kModeReplay) ? n : 0) + (cf > 0 ? 1 : 0);
+    for (int t = gw; t < tasks; t += GW) {
+      const bool fold_task = !(MODE == kModeReplay && t < n);
+      float xa = 1.f, xd = 0.f;
+      int last;  // last lane of the scanned window
+      if (fold_task) {
+        last = cf - 1;
+        if (lane <= last) {
+          xa = es.a(lane);
+          xd = es.dt(lane);
+        }
+      } else {
+        last = c + t - o0;
+        if (lane <= last) {
+          xa = es.a(o0 + lane);
+          xd = es.dt(o0 + lane);
+        }
+      }
+      const float incl = warp_suffix_prod(xa, lane);  // prod_{lane <= i <= last} a_i
+      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+      if (lane == 31) excl = 1.f;
+      if (fold_task) {
+        if (lane <= last) sig[lane] = xd * excl;
+        if (lane == 0) sig[kMaxWindow] = incl;
+      } else {
+        if (lane <= last) wout[t * kMaxWindow + lane] = xd * excl;
+        if (lane == 0) alpha[t] = incl;
+      }
+    }
+    if (MODE == kModeReplay) entry_dots<N, IO, GW>(kbuf, qbuf, o0, width, n, kq, gw, lane);
+  }
+  group_sync(bar_id, GT);
+
+  // y = alpha_s d + sum_{jj} w_{s,jj} kq_{s,jj} v_{o0+jj}[p], by the lanes that hold row p's d
   auto write_outputs = [&](float (&part)[RT], int s, int gi, bool from_tile_fp8) {
     int base;
     const bool wr = Red::run(part, lane, base);
 #pragma unroll
     for (int i = 0; i < Red::kHeld; ++i) {
-      const int pr = gi * RG + row0 + RPP * (base + i);
+      const int pr = gi * RGR + row0 + RPG * (base + i);
       if (wr && pr < P) {
         float d = part[i];
         if (from_tile_fp8) d *= scale_tile[pr];
         if (MODE == kModeReplay) {
-          p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, bt[s * P + pr]);
+          const int last = c + s - o0;
+          float b0 = 0.f, b1 = 0.f;
+          int jj = 0;
+          for (; jj + 1 <= last; jj += 2) {
+            b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj],
+                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj) * P + pr) * S_IO), b0);
+            b1 = fmaf(wout[s * kMaxWindow + jj + 1] * kq[s * kMaxWindow + jj + 1],
+                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj + 1) * P + pr) * S_IO), b1);
+          }
+          if (jj <= last)
+            b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj],
+                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj) * P + pr) * S_IO), b0);
+          p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
         } else {
           p.y[bh * P + pr] = d;
         }
@@ -345,22 +457,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   };
 
   if (!pl.fold) {
-    // output-only route from the stored checkpoint (FP32 master or FP8 read copy)
+    // ---- phase B: output-only route from the stored checkpoint
     for (int gi = 0; gi < ngroups; ++gi) {
-      float4 x[RT];
-#pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const int pr = gi * RG + row0 + RPP * r;
-        if (pr < P) {
-          if (pl.fp32_tile) {
-            x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
-          } else {
-            x[r] = e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
-          }
-        } else {
-          x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
+      if (gi > 0) load_rows(x, gi, false);
 #pragma unroll
       for (int s = 0; s < NQ; ++s) {
         if (s < n) {
@@ -372,25 +471,19 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       }
     }
   } else {
-    // fold (state route), write the state back, then outputs from the fresh state
-    const float abar = sig[jw];
+    // ---- phase B: fold (state route), write the state back, outputs from the fresh rows
+    const int cf_pad = (cf + kFoldChunk - 1) / kFoldChunk * kFoldChunk;
+    for (int idx = gtid; idx < P * cf_pad; idx += GT) {
+      const int pp = idx / cf_pad;
+      const int j = idx - pp * cf_pad;
+      wt[pp * fp + j] = j < cf ? sig[j] * IoT<IO>::load1(vbuf + ((size_t)j * P + pp) * S_IO) : 0.f;
+    }
+    group_sync(bar_id, GT);
+    const float abar = sig[kMaxWindow];
     for (int gi = 0; gi < ngroups; ++gi) {
-      float4 acc[RT];
+      if (gi > 0) load_rows(x, gi, MODE == kModeEager);
 #pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const int pr = gi * RG + row0 + RPP * r;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (pr < P) {
-          if (pl.fp32_tile) {
-            x = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
-          } else {  // eager on a shared FP8 state: dequantise
-            const float sc = scale_tile[pr];
-            const float4 e = e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
-            x = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
-          }
-        }
-        acc[r] = make_float4(abar * x.x, abar * x.y, abar * x.z, abar * x.w);
-      }
+      for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
       for (int ch = 0; ch < cf_pad; ch += kFoldChunk) {
         float4 kr[kFoldChunk];
 #pragma unroll
@@ -400,7 +493,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         }
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-          const int pr = gi * RG + row0 + RPP * r;
+          const int pr = gi * RGR + row0 + RPG * r;
           if (pr < P) {
             const float* wrow = wt + (size_t)pr * fp + ch;
 #pragma unroll
@@ -409,10 +502,10 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
               const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
               for (int t = 0; t < 4; ++t) {
-                acc[r].x = fmaf(wv[t], kr[jj + t].x, acc[r].x);
-                acc[r].y = fmaf(wv[t], kr[jj + t].y, acc[r].y);
-                acc[r].z = fmaf(wv[t], kr[jj + t].z, acc[r].z);
-                acc[r].w = fmaf(wv[t], kr[jj + t].w, acc[r].w);
+                x[r].x = fmaf(wv[t], kr[jj + t].x, x[r].x);
+                x[r].y = fmaf(wv[t], kr[jj + t].y, x[r].y);
+                x[r].z = fmaf(wv[t], kr[jj + t].z, x[r].z);
+                x[r].w = fmaf(wv[t], kr[jj + t].w, x[r].w);
               }
             }
           }
@@ -423,15 +516,15 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       const bool store_fp8 = (CKPT == kCkptFp8);
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const int pr = gi * RG + row0 + RPP * r;
-        if (store_f32 && pr < P) *reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col) = acc[r];
+        const int pr = gi * RGR + row0 + RPG * r;
+        if (store_f32 && pr < P) *reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col) = x[r];
         if (store_fp8) {
-          const float am = seg_allmax<TPR>(amax4(acc[r]));
+          const float am = seg_allmax<TPR>(amax4(x[r]));
           float sc, inv;
           e4m3_row_scale(am, sc, inv);
           if (pr < P) {
-            *reinterpret_cast<uint32_t*>(p.S8 + (bh * P + pr) * N + col) = quant4_e4m3(acc[r], inv);
-            if ((ctid % TPR) == 0) p.Sscale[bh * P + pr] = sc;
+            *reinterpret_cast<uint32_t*>(p.S8 + (bh * P + pr) * N + col) = quant4_e4m3(x[r], inv);
+            if ((lane % TPR) == 0) p.Sscale[bh * P + pr] = sc;
           }
         }
       }
@@ -441,7 +534,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
           if (s < n) {
             float part[RT];
 #pragma unroll
-            for (int r = 0; r < RT; ++r) part[r] = dot4(acc[r], qr[s]);
+            for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
             write_outputs(part, s, gi, false);
           }
         }
@@ -449,7 +542,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     }
   }
 
-  // ---- phase 4: append this call's entries to the ring, publish the pointer word
+  // ---- phase C: append this call's entries to the ring, publish the pointer word
+  const int start = pl.start;
+  const int cap = p.cap;
   if (MODE == kModeReplay) {
     const int kchunks = N * S_IO / 16;
     const int vchunks = P * S_IO / 16;
@@ -457,28 +552,28 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     uint8_t* rv = static_cast<uint8_t*>(p.ring_v) + bh * cap * P * S_IO;
     const bool write_k = (pl.h % p.hpg) == 0;
     const int total = n * (kchunks + vchunks);
-    for (int idx = ctid; idx < total; idx += kConsumerThreads) {
+    for (int idx = gtid; idx < total; idx += GT) {
       const int s = idx / (kchunks + vchunks);
       const int ch = idx - s * (kchunks + vchunks);
-      int slot = start + c + s;
-      slot -= (slot >= cap) ? cap : 0;
+      int slot_i = start + c + s;
+      slot_i -= (slot_i >= cap) ? cap : 0;
       if (ch < kchunks) {
         if (write_k)
-          *reinterpret_cast<uint4*>(rk + (size_t)slot * N * S_IO + ch * 16) =
+          *reinterpret_cast<uint4*>(rk + (size_t)slot_i * N * S_IO + ch * 16) =
               *reinterpret_cast<const uint4*>(kbuf + (size_t)(c + s) * N * S_IO + ch * 16);
       } else {
         const int cv = ch - kchunks;
-        *reinterpret_cast<uint4*>(rv + (size_t)slot * P * S_IO + cv * 16) =
+        *reinterpret_cast<uint4*>(rv + (size_t)slot_i * P * S_IO + cv * 16) =
             *reinterpret_cast<const uint4*>(vbuf + (size_t)(c + s) * P * S_IO + cv * 16);
       }
     }
-    if (ctid < n) {
-      int slot = start + c + ctid;
-      slot -= (slot >= cap) ? cap : 0;
-      p.ring_dt[bh * cap + slot] = dtn[ctid];
-      p.ring_a[bh * cap + slot] = an[ctid];
+    if (gtid < n) {
+      int slot_i = start + c + gtid;
+      slot_i -= (slot_i >= cap) ? cap : 0;
+      p.ring_dt[bh * cap + slot_i] = reinterpret_cast<const float*>(st + p.off_dtn)[gtid];
+      p.ring_a[bh * cap + slot_i] = reinterpret_cast<const float*>(st + p.off_an)[gtid];
     }
-    if (pl.h == 0 && ctid == 0) {
+    if (pl.h == 0 && gtid == 0) {
       int start2 = pl.fold ? start + c : start;
       start2 -= (start2 >= cap) ? cap : 0;
       const int base = pl.fold ? 0 : c;
@@ -487,7 +582,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       if (p.flushed) p.flushed[pl.b] = pl.fold ? 1 : 0;
     }
   } else if (MODE == kModeFlush) {
-    if (pl.h == 0 && ctid == 0) {
+    if (pl.h == 0 && gtid == 0) {
       int start2 = start + c;
       start2 -= (start2 >= cap) ? cap : 0;
       p.counts_out[pl.b] = start2 << 16;
@@ -496,41 +591,42 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   }
 }
 
-template <int N, typename IO, int CKPT, int MODE, int NQ>
+template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
 __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_constant__ KParams p) {
+  using Gr = Groups<NG>;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + kMaxStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kMaxStages);
+  Bars* bars = reinterpret_cast<Bars*>(smem);
   uint8_t* stages = smem + p.stages_off;
-  uint8_t* ws = smem + p.ws_off;
   constexpr int S_IO = IoT<IO>::bytes;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.num_stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], Gr::kThreads);
     }
-    *abort_flag = 0;
+    bars->abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
   const int warp = threadIdx.x / 32;
   if (warp == kConsumerWarps) {
-    producer_loop<MODE, CKPT, S_IO>(p, stages, full, empty, abort_flag);
+    producer_loop<MODE, CKPT, S_IO>(p, stages, bars);
     return;
   }
-  const int ctid = threadIdx.x;
-  int i = 0;
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++i) {
-    const int s = i % p.num_stages;
-    const int k = i / p.num_stages;
-    const bool ok = consumer_all(mbar_wait_bounded(&full[s], k & 1));
+  const int g = warp / Gr::kWarps;  // consumer group
+  const int gtid = threadIdx.x - g * Gr::kThreads;
+  const int bar_id = 1 + g;
+  uint8_t* ws = smem + p.ws_off + (size_t)g * p.ws_group_bytes;
+  const int NS = p.num_stages;
+  int i = g;
+  for (int u = blockIdx.x + g * gridDim.x; u < p.num_units; u += NG * gridDim.x, i += NG) {
+    const int s = i % NS;
+    const bool ok = group_all(mbar_wait_bounded(&bars->full[s], (i / NS) & 1), bar_id, Gr::kThreads);
     if (!ok) {
-      if (ctid == 0) {
+      if (gtid == 0) {
         report_error(p.status, kErrWaitTimeout);
-        *abort_flag = 1;
+        bars->abort_flag = 1;
       }
       break;
     }
@@ -539,15 +635,13 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u, word, msk);
     if (pl.active) {
-      consume_unit<N, IO, CKPT, MODE, NQ>(p, pl, st, ws, ctid);
-    } else if (MODE == kModeFlush && !pl.corrupt && pl.h == 0 && ctid == 0) {
+      consume_unit<N, IO, CKPT, MODE, NQ, NG>(p, pl, st, ws, gtid, bar_id);
+    } else if (pl.h == 0 && gtid == 0) {
       p.counts_out[pl.b] = word;  // nothing to fold: the pointer word carries over
-      if (p.flushed) p.flushed[pl.b] = 0;
-    } else if (pl.corrupt && pl.h == 0 && ctid == 0) {
-      p.counts_out[pl.b] = word;
+      if (MODE == kModeFlush && p.flushed && !pl.corrupt) p.flushed[pl.b] = 0;
     }
-    consumer_sync();
-    if (ctid == 0) mbar_arrive(&empty[s]);
+    group_sync(bar_id, Gr::kThreads);
+    mbar_arrive(&bars->empty[s]);
   }
 }
 

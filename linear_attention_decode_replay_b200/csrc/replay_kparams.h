@@ -33,10 +33,11 @@ struct KParams {
   int32_t* counts_out;
   int32_t* status;
   // shared-memory layout, bytes
-  int32_t num_stages, stage_bytes, stages_off, ws_off;
+  int32_t num_stages, stage_bytes, stages_off;
   int32_t off_k, off_v, off_q, off_dtr, off_ar, off_dtn, off_an, off_meta;  // within a stage
-  int32_t ws_w, ws_kq, ws_alpha, ws_sig, ws_wt, ws_bt;                      // within the workspace
-  int32_t jw, fp;  // workspace row strides (entries per query row, fold entries per state row)
+  int32_t ws_off, ws_group_bytes;          // one workspace per consumer group
+  int32_t ws_w, ws_kq, ws_alpha, ws_sig, ws_wt;  // within a group's workspace
+  int32_t fp;                               // fold entries per state row in ws_wt, padded
   int32_t smem_bytes;
 };
 

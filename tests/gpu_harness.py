@@ -46,6 +46,20 @@ class Report:
     counts_equal: bool = True
     ckpt_err: float = 0.0
     per_step: list = field(default_factory=list)
+    fro_err: float = 0.0          # max over steps of ||Y - Y_ref||_F / ||Y_ref||_F (sampled batch)
+    shared_fro_err: float = 0.0   # same for the shared-FP8 eager kernel
+    per_vector: list = field(default_factory=list)  # every per-(sequence, head) error
+
+
+def frobenius_error(y, y_ref) -> float:
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    return float(np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-30))
+
+
+def vector_errors(y, y_ref) -> np.ndarray:
+    num = np.linalg.norm(np.asarray(y, np.float64) - y_ref, axis=-1)
+    return (num / np.maximum(np.linalg.norm(y_ref, axis=-1), 1e-30)).ravel()
 
 
 def setup(shape: gen.Shape, device="cuda"):
@@ -78,12 +92,17 @@ def run_decode(shape: gen.Shape, steps: int, rows, flush_at_end=True, fp8_emulat
         e = ro.relative_error(y_gpu, y_ref)
         rep.per_step.append(e)
         rep.max_err = max(rep.max_err, e)
+        rep.fro_err = max(rep.fro_err, frobenius_error(y_gpu, y_ref))
+        if shared_fp8:
+            rep.per_vector.append(vector_errors(y_gpu, y_ref))
         if emu is not None:
             y_emu, _ = emu.step(xs["q"], xs["k"], xs["v"], xs["dt"], xs["a"])
             rep.max_err_fp8_emul = max(rep.max_err_fp8_emul, ro.relative_error(y_gpu, y_emu))
         if shared_fp8:
             y_sh = lar.eager_step_fp8(cfg, codes_d, scale_d, x["q"], x["k"], x["v"], x["dt"], x["a"])
-            rep.max_err_shared_fp8 = max(rep.max_err_shared_fp8, ro.relative_error(_np(y_sh, rows), y_ref))
+            y_sh_np = _np(y_sh, rows)
+            rep.max_err_shared_fp8 = max(rep.max_err_shared_fp8, ro.relative_error(y_sh_np, y_ref))
+            rep.shared_fro_err = max(rep.shared_fro_err, frobenius_error(y_sh_np, y_ref))
         f_gpu = fl.cpu().numpy()
         all_flags.append(f_gpu.copy())
         if not np.array_equal(f_gpu[rows], f_ref):

@@ -28,7 +28,8 @@
  *    with replay_check_status. No kernel traps.
  *  - Layouts are dense, row-major, batch-major. Shapes use B = batch, H = heads,
  *    G = k/q groups (H % G == 0; head h uses group h / (H/G)), P = v-dim, N = k-dim,
- *    L = window, cap = replay_ring_capacity(cfg). "io" is the replay_config.io dtype.
+ *    L = window, cap = replay_ring_capacity(cfg), R = replay_ring_record_bytes(cfg).
+ *    "io" is the replay_config.io dtype.
  *  - A replay_ctx is not thread-safe; calls on one context must be serialised.
  */
 #ifndef REPLAY_H
@@ -81,15 +82,18 @@ typedef struct {
 } replay_config;
 
 /* Caller-owned device buffers of one decode layer. All 16-byte aligned except counts and
- * status (4-byte). P*N*4 bytes per head must not exceed 65536. */
+ * status (4-byte). P*N*4 bytes per head must not exceed 65536.
+ *
+ * The buffer of recent inputs is a ring of `cap` records per (sequence, head); record j
+ * holds one buffered input as R bytes: k (N io values), v (P io values), Delta (FP32),
+ * a (FP32), zero padding to a multiple of 16 bytes. Keeping an entry's pieces together
+ * lets a unit's whole buffer arrive in one or two bulk copies. */
 typedef struct {
   float* S0;         /* [B][H][P][N] FP32 checkpoint (master); row p of N floats contiguous */
   uint8_t* S0_fp8;   /* [B][H][P][N] e4m3 read copy (ckpt = REPLAY_CKPT_F32_FP8READ, else NULL) */
   float* S0_scale;   /* [B][H][P] FP32 per-row scale of the copy (same condition) */
-  void* ring_k;      /* [B][G][cap][N] io: buffered k entries */
-  void* ring_v;      /* [B][H][cap][P] io: buffered v entries */
-  float* ring_dt;    /* [B][H][cap] buffered Delta */
-  float* ring_a;     /* [B][H][cap] buffered decay a */
+  void* ring;        /* [B][H][cap] records of R bytes (see above) */
+  void* qpack;       /* [B][G][max_pos][N] io scratch for verify queries (max_pos > 1, else NULL) */
   int32_t* counts;   /* [2][B] buffer pointer words, double-buffered (the library alternates
                         halves each call so that no launch reads what it writes) */
   int32_t* status;   /* [1] device error word (REPLAY_DEV_* bits) */
@@ -97,11 +101,13 @@ typedef struct {
 
 typedef struct replay_ctx replay_ctx;
 
-/* Entries the ring arrays must hold per (sequence, head): L + max_pos rounded up to a
- * multiple of 4. A flush and the appends of the same call touch disjoint slots, so heads
- * that share a k/q group can run in any order. Returns a negative replay_status on a
- * bad config. */
+/* Records the ring holds per (sequence, head): L + max_pos. A flush and the appends of
+ * the same call touch disjoint records. Returns a negative replay_status on a bad config. */
 int32_t replay_ring_capacity(const replay_config* cfg);
+
+/* Bytes of one ring record: N*s + P*s + 8 rounded up to a multiple of 16, s = 2 (BF16) or
+ * 4 (FP32). Returns a negative replay_status on a bad config. */
+int32_t replay_ring_record_bytes(const replay_config* cfg);
 
 /* Validates cfg and bufs, zeroes both halves of counts (every buffer empty) and the
  * status word, and for REPLAY_CKPT_F32_FP8READ fills S0_fp8 / S0_scale from S0 (per-row

@@ -33,7 +33,7 @@ from ._abi import (  # noqa: F401
     strerror,
 )
 
-__all__ = ["Config", "Replay", "alloc_buffers", "ring_capacity", "eager_step", "eager_step_fp8",
+__all__ = ["Config", "Replay", "alloc_buffers", "ring_capacity", "ring_record_bytes", "eager_step", "eager_step_fp8",
            "quantize_rows_e4m3", "ReplayError", "load", "strerror"]
 
 
@@ -68,19 +68,26 @@ def ring_capacity(cfg: Config) -> int:
     return cap
 
 
+def ring_record_bytes(cfg: Config) -> int:
+    r = load().replay_ring_record_bytes(ctypes.byref(cfg.c()))
+    if r < 0:
+        raise ReplayError(r, "replay_ring_record_bytes")
+    return r
+
+
 def alloc_buffers(cfg: Config, device="cuda") -> dict:
     """Allocates the caller-owned device buffers of one layer (S0 left uninitialised)."""
     cap = ring_capacity(cfg)
+    rec = ring_record_bytes(cfg)
     B, H, G, P, N = cfg.batch, cfg.heads, cfg.groups, cfg.P, cfg.N
     bufs = {
         "S0": torch.empty(B, H, P, N, device=device, dtype=torch.float32),
-        "ring_k": torch.empty(B, G, cap, N, device=device, dtype=cfg.io_dtype),
-        "ring_v": torch.empty(B, H, cap, P, device=device, dtype=cfg.io_dtype),
-        "ring_dt": torch.empty(B, H, cap, device=device, dtype=torch.float32),
-        "ring_a": torch.empty(B, H, cap, device=device, dtype=torch.float32),
+        "ring": torch.zeros(B, H, cap, rec, device=device, dtype=torch.uint8),
         "counts": torch.zeros(2, B, device=device, dtype=torch.int32),
         "status": torch.zeros(1, device=device, dtype=torch.int32),
     }
+    if cfg.max_pos > 1:
+        bufs["qpack"] = torch.empty(B, G, cfg.max_pos, N, device=device, dtype=cfg.io_dtype)
     if cfg.ckpt == "f32_fp8read":
         bufs["S0_fp8"] = torch.empty(B, H, P, N, device=device, dtype=torch.uint8)
         bufs["S0_scale"] = torch.empty(B, H, P, device=device, dtype=torch.float32)
@@ -119,14 +126,13 @@ class Replay:
         B, H, G, P, N = cfg.batch, cfg.heads, cfg.groups, cfg.P, cfg.N
         cap = ring_capacity(cfg)
         fp8 = cfg.ckpt == "f32_fp8read"
+        rec = ring_record_bytes(cfg)
         cb = _abi.CBuffers(
             _ptr(buffers["S0"], (B, H, P, N), torch.float32, "S0"),
             _ptr(buffers.get("S0_fp8"), (B, H, P, N), torch.uint8, "S0_fp8") if fp8 else None,
             _ptr(buffers.get("S0_scale"), (B, H, P), torch.float32, "S0_scale") if fp8 else None,
-            _ptr(buffers["ring_k"], (B, G, cap, N), cfg.io_dtype, "ring_k"),
-            _ptr(buffers["ring_v"], (B, H, cap, P), cfg.io_dtype, "ring_v"),
-            _ptr(buffers["ring_dt"], (B, H, cap), torch.float32, "ring_dt"),
-            _ptr(buffers["ring_a"], (B, H, cap), torch.float32, "ring_a"),
+            _ptr(buffers["ring"], (B, H, cap, rec), torch.uint8, "ring"),
+            _ptr(buffers.get("qpack"), (B, G, cfg.max_pos, N), cfg.io_dtype, "qpack") if cfg.max_pos > 1 else None,
             _ptr(buffers["counts"], (2, B), torch.int32, "counts"),
             _ptr(buffers["status"], (1,), torch.int32, "status"),
         )

@@ -44,8 +44,8 @@ class CConfig(ctypes.Structure):
 
 class CBuffers(ctypes.Structure):
     _fields_ = [("S0", ctypes.c_void_p), ("S0_fp8", ctypes.c_void_p), ("S0_scale", ctypes.c_void_p),
-                ("ring_k", ctypes.c_void_p), ("ring_v", ctypes.c_void_p), ("ring_dt", ctypes.c_void_p),
-                ("ring_a", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("ring", ctypes.c_void_p), ("qpack", ctypes.c_void_p), ("counts", ctypes.c_void_p),
+                ("status", ctypes.c_void_p)]
 
 
 _lib = None
@@ -64,6 +64,7 @@ def load() -> ctypes.CDLL:
     cfgp = ctypes.POINTER(CConfig)
     sig = {
         "replay_ring_capacity": (i32, [cfgp]),
+        "replay_ring_record_bytes": (i32, [cfgp]),
         "replay_init": (ctypes.c_int, [cfgp, ctypes.POINTER(CBuffers), vp, ctypes.POINTER(vp)]),
         "replay_step": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_verify": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),

@@ -49,7 +49,11 @@ int validate_config(const replay_config* c, bool needs_window) {
   return REPLAY_OK;
 }
 
-int ring_capacity(const replay_config& c) { return round_up(c.L + c.max_pos, 4); }
+int ring_capacity(const replay_config& c) { return c.L + c.max_pos; }
+int record_bytes(const replay_config& c) {
+  const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
+  return round_up((c.N + c.P) * s_io + 8, 16);
+}
 
 struct DeviceInfo {
   int device, num_sms, smem_optin;
@@ -70,32 +74,25 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   std::memset(p, 0, sizeof(*p));
   const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
   const int P = c.P, N = c.N;
-  int jmax, nq_alloc, lfold, ring;
+  int jmax, nq_alloc, lfold;  // records a stage holds, query slots, most entries one unit folds
   if (mode == replay::kModeReplay) {
     jmax = c.L + c.max_pos;
     nq_alloc = c.max_pos;
     lfold = c.L;
-    ring = cap;
   } else if (mode == replay::kModeFlush) {
     jmax = c.L;
     nq_alloc = 0;
     lfold = c.L;
-    ring = cap;
   } else {
     jmax = 1;
     nq_alloc = 1;
     lfold = 1;
-    ring = 0;
   }
+  p->rec_bytes = record_bytes(c);
   const int tile = fp8_eager ? round_up(P * N + P * 4, 16) : P * N * 4;
-  p->off_k = round_up(tile, 16);
-  p->off_v = p->off_k + round_up(jmax * N * s_io, 16);
-  p->off_q = p->off_v + round_up(jmax * P * s_io, 16);
-  p->off_dtr = p->off_q + round_up(nq_alloc * N * s_io, 16);
-  p->off_ar = p->off_dtr + round_up(ring * 4, 16);
-  p->off_dtn = p->off_ar + round_up(ring * 4, 16);
-  p->off_an = p->off_dtn + replay::kMaxPos * 4;
-  p->off_meta = p->off_an + replay::kMaxPos * 4;
+  p->off_rec = round_up(tile, 16);
+  p->off_q = p->off_rec + jmax * p->rec_bytes;
+  p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
   p->stage_bytes = round_up(p->off_meta + 16, 128);
 
   // one workspace per consumer group: decay weights and k.q of the outputs
@@ -145,10 +142,9 @@ void set_state(KParams* p, const replay_ctx* ctx) {
   p->S = ctx->bufs.S0;
   p->S8 = ctx->bufs.S0_fp8;
   p->Sscale = ctx->bufs.S0_scale;
-  p->ring_k = ctx->bufs.ring_k;
-  p->ring_v = ctx->bufs.ring_v;
-  p->ring_dt = ctx->bufs.ring_dt;
-  p->ring_a = ctx->bufs.ring_a;
+  p->ring = ctx->bufs.ring;
+  p->qpack = nullptr;
+  p->qpack_pos = ctx->cfg.max_pos;
   p->counts_in = ctx->bufs.counts + (size_t)ctx->parity * ctx->cfg.batch;
   p->counts_out = ctx->bufs.counts + (size_t)(1 - ctx->parity) * ctx->cfg.batch;
   p->status = ctx->bufs.status;
@@ -174,6 +170,33 @@ int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const voi
   p.a = a;
   p.y = y;
   p.flushed = flushed;
+  // pre-pass: this call's entries into their ring records (and verify queries into qpack)
+  replay::PackParams pp;
+  pp.B = p.B;
+  pp.H = p.H;
+  pp.G = p.G;
+  pp.P = p.P;
+  pp.N = p.N;
+  pp.L = p.L;
+  pp.cap = p.cap;
+  pp.n_pos = n_pos;
+  pp.hpg = p.hpg;
+  pp.rec_bytes = p.rec_bytes;
+  pp.io_bytes = ctx->cfg.io == REPLAY_BF16 ? 2 : 4;
+  pp.qpack_pos = ctx->cfg.max_pos;
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.dt = dt;
+  pp.a = a;
+  pp.ring = ctx->bufs.ring;
+  pp.qpack = n_pos > 1 ? ctx->bufs.qpack : nullptr;
+  pp.counts_in = p.counts_in;
+  p.qpack = pp.qpack;
+  const long long tasks = (long long)p.B * p.H;
+  const long long blocks = (tasks + 7) / 8;
+  const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
+  if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
   const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
   if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos > 1 ? replay::kMaxPos : 1, ctx->num_sms, s) !=
       cudaSuccess)
@@ -230,21 +253,25 @@ int32_t replay_ring_capacity(const replay_config* cfg) {
   return ring_capacity(*cfg);
 }
 
+int32_t replay_ring_record_bytes(const replay_config* cfg) {
+  const int rc = validate_config(cfg, true);
+  if (rc) return rc;
+  return record_bytes(*cfg);
+}
+
 int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_stream_t stream, replay_ctx** out) {
   if (!out) return REPLAY_EINVAL;
   *out = nullptr;
   int rc = validate_config(cfg, true);
   if (rc) return rc;
-  if (!bufs || !bufs->S0 || !bufs->ring_k || !bufs->ring_v || !bufs->ring_dt || !bufs->ring_a || !bufs->counts ||
-      !bufs->status)
-    return REPLAY_EINVAL;
+  if (!bufs || !bufs->S0 || !bufs->ring || !bufs->counts || !bufs->status) return REPLAY_EINVAL;
   const bool fp8 = cfg->ckpt == REPLAY_CKPT_F32_FP8READ;
   if (fp8 && (!bufs->S0_fp8 || !bufs->S0_scale)) return REPLAY_EINVAL;
-  if (!aligned(bufs->S0, 16) || !aligned(bufs->ring_k, 16) || !aligned(bufs->ring_v, 16) ||
-      !aligned(bufs->ring_dt, 16) || !aligned(bufs->ring_a, 16) || !aligned(bufs->counts, 4) ||
-      !aligned(bufs->status, 4))
+  if (cfg->max_pos > 1 && !bufs->qpack) return REPLAY_EINVAL;
+  if (!aligned(bufs->S0, 16) || !aligned(bufs->ring, 16) || !aligned(bufs->counts, 4) || !aligned(bufs->status, 4))
     return REPLAY_EALIGN;
   if (fp8 && (!aligned(bufs->S0_fp8, 16) || !aligned(bufs->S0_scale, 16))) return REPLAY_EALIGN;
+  if (cfg->max_pos > 1 && !aligned(bufs->qpack, 16)) return REPLAY_EALIGN;
 
   DeviceInfo d;
   if ((rc = device_info(&d))) return rc;

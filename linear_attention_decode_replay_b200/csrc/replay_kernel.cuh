@@ -3,17 +3,18 @@
 // One launch processes every (sequence b, head h) unit of a decode layer. Each CTA owns
 // the units blockIdx.x, blockIdx.x + gridDim.x, ... and streams them through a ring of
 // shared-memory stages:
-//   * the producer warp reads the unit's buffer pointer word (prefetched one unit
-//     ahead) and issues, one copy per lane in a single instruction, the 1-D bulk copies
-//     (TMA) of the unit's checkpoint tile S0[b,h] (P x N, FP32 master or FP8 read copy +
-//     per-row scales), of the live ring-buffer entries (k, v, Delta, a) and of this
-//     call's new tokens into a stage, completing on that stage's "full" mbarrier;
-//   * NG consumer groups (8/NG warps each) take alternate units end to end: decay
-//     scans and k_j . q_s products spread over the group's warps, then the state rows
-//     (output-only dot products, or the fused fold and its write-back), then the ring
-//     append; each group releases the stage through its "empty" mbarrier. Two groups
-//     keep two units in flight, so one unit's short dependent chains overlap the
-//     other's.
+//   * the producer warp reads the unit's buffer pointer word (prefetched 32 units at a
+//     time) and fills a stage with 1-D bulk copies (TMA), one copy per lane: the unit's
+//     checkpoint tile S0[b,h] (P x N, FP32 master or FP8 read copy + per-row scales),
+//     the unit's live ring records (k, v, Delta, a of every buffered input and of this
+//     call's new tokens, which a pre-pass has already written into the ring) in one or
+//     two pieces, and the queries; all complete on the stage's "full" mbarrier;
+//   * NG consumer groups (8/NG warps each) take alternate units end to end: the state
+//     row dot products together with the decay scans and k_j . q_s products, spread
+//     over the group's warps, then the outputs (or the fused fold, its write-back and
+//     the outputs from the fresh rows); each group releases the stage through its
+//     "empty" mbarrier. Two groups keep two units in flight, so one unit's short
+//     dependent chains overlap the other's.
 // The state is streamed exactly once per call; every other byte is small.
 //
 // What a unit computes (blog "ReplaySSM: Cachear Inputs, No Estado": routes "estado y
@@ -22,8 +23,7 @@
 //     entries, fold it first, S0 <- abar S0 + sum_j s_j v_j k_j^T, writing the master
 //     (and the FP8 copy) once; then for each position s
 //       y_s = alpha_s (S q_s) + sum_{j <= c+s} w_{s,j} (k_j . q_s) v_j
-//     where S is the fresh fold (in registers) or the stored checkpoint, and append the
-//     new entries to the ring.
+//     where S is the fresh fold (in registers) or the stored checkpoint.
 //   FLUSH: fold the buffer of the selected sequences, no output.
 //   EAGER (baseline): S <- a S + Delta v k^T, y = S q, the state read and written every
 //     call (FP32, or a shared FP8 state re-quantised every call).
@@ -53,6 +53,7 @@ struct Bars {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   int abort_flag;
+  int last_fill[kMaxStages];  // CTA-local index of the latest unit copied into each stage
 };
 static_assert(sizeof(Bars) <= 256, "the barrier header must fit the 256 bytes the host layout reserves");
 
@@ -76,8 +77,7 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
     pl.corrupt = false;
     pl.active = true;
     pl.fp32_tile = (CKPT == kCkptF32);
-    const uint32_t tile = pl.fp32_tile ? P * N * 4u : P * N + P * 4u;
-    pl.bytes = tile + 2u * N * S_IO + P * S_IO;
+    pl.bytes = pl.fp32_tile ? P * N * 4u : P * N + P * 4u;  // bulk-copied (TMA) bytes
     return pl;
   }
   pl.start = word >> 16;
@@ -96,145 +96,139 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
     pl.bytes = 0;
     return pl;
   }
-  uint32_t bytes = pl.fp32_tile ? P * N * 4u : P * N + P * 4u;
-  if (pl.c > 0) bytes += pl.c * (N + P) * S_IO + 2u * p.cap * 4u;
-  if (MODE == kModeReplay) bytes += p.n_pos * (2u * N + P) * S_IO;
-  pl.bytes = bytes;
+  const uint32_t records = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
+  pl.bytes = (pl.fp32_tile ? P * N * 4u : P * N + P * 4u) + records * (uint32_t)p.rec_bytes +
+             ((MODE == kModeReplay) ? p.n_pos * N * S_IO : 0u);
   return pl;
 }
 
-// Entry j of the unit's buffer view: j < c are ring entries (slot start + j modulo cap),
-// j >= c are this call's new tokens. Eager units have only the new token (j = 0).
-template <int MODE>
-struct EntryScalars {
-  const float *dtr, *ar, *dtn, *an;
-  int start, cap, c;
-  __device__ __forceinline__ int slot(int j) const {
-    int s = start + j;
-    return s - ((s >= cap) ? cap : 0);
-  }
+// Entry j of a unit lives in record j of the stage: k (N io values), v (P io values),
+// Delta, a. Records 0..c-1 are the buffered inputs, c.. this call's new tokens.
+template <int N, int S_IO>
+struct Records {
+  const uint8_t* base;
+  int P, R;
+  __device__ __forceinline__ const uint8_t* k(int j) const { return base + (size_t)j * R; }
+  __device__ __forceinline__ const uint8_t* v(int j) const { return base + (size_t)j * R + N * S_IO; }
   __device__ __forceinline__ float dt(int j) const {
-    if (MODE == kModeEager) return dtn[j];
-    return j < c ? dtr[slot(j)] : dtn[j - c];
+    return *reinterpret_cast<const float*>(base + (size_t)j * R + (N + P) * S_IO);
   }
   __device__ __forceinline__ float a(int j) const {
-    if (MODE == kModeEager) return an[j];
-    return j < c ? ar[slot(j)] : an[j - c];
+    return *reinterpret_cast<const float*>(base + (size_t)j * R + (N + P) * S_IO + 4);
   }
 };
 
 // ---------------------------------------------------------------------------- producer
-// Each lane issues at most one of the unit's copies: lane 0 the state tile, lane 1 the
-// FP8 row scales, lanes 2-5 the ring k and v pieces, lanes 6-7 the Delta and a rings,
-// lanes 8 + 3s .. 10 + 3s the new q, k, v of position s.
+// One unit's copies into stage `st`, one bulk copy (TMA) per lane, counted in bytes on
+// `bar`: lane 0 the state tile, lane 1 the FP8 row scales, lanes 2-3 the live ring
+// records [start, start + count) modulo cap, lane 4 the queries. The eager baseline has
+// no ring: its new token's k, v, Delta, a (and q) are gathered with per-lane cp.async.
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& pl, uint8_t* st, uint64_t* bar,
-                                                  int lane) {
+                                                  int lane, uint64_t stream_policy) {
   const size_t P = p.P, N = p.N;
   const size_t bh = (size_t)pl.b * p.H + pl.h;
-  const int n_new = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
-  const int c = pl.c;
-  uint8_t* kbuf = st + p.off_k;
-  uint8_t* vbuf = st + p.off_v;
-  void* dst = nullptr;
+  if (!pl.active) return;
+  uint8_t* recbuf = st + p.off_rec;
+  if (MODE == kModeEager) {
+    if (lane == 0)
+      bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + bh * P * N) : (const void*)(p.S8 + bh * P * N),
+                    pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N), bar, stream_policy);
+    if (lane == 1 && !pl.fp32_tile) bulk_g2s(st + P * N, p.Sscale + bh * P, (uint32_t)(P * 4), bar);
+    const int kpe = (int)(N * S_IO / 16);
+    const int vpe = (int)(P * S_IO / 16);
+    const size_t bg = (size_t)pl.b * p.G + pl.g;
+    for (int idx = lane; idx < 2 * kpe + vpe; idx += 32) {
+      if (idx < kpe) {
+        cp_async16(st + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
+      } else if (idx < 2 * kpe) {
+        const int ch = idx - kpe;
+        cp_async16(recbuf + ch * 16, static_cast<const uint8_t*>(p.k) + bg * N * S_IO + ch * 16);
+      } else {
+        const int ch = idx - 2 * kpe;
+        cp_async16(recbuf + N * S_IO + ch * 16, static_cast<const uint8_t*>(p.v) + bh * P * S_IO + ch * 16);
+      }
+    }
+    if (lane == 0) cp_async4(recbuf + (N + P) * S_IO, p.dt + bh);
+    if (lane == 1) cp_async4(recbuf + (N + P) * S_IO + 4, p.a + bh);
+    return;
+  }
   const void* src = nullptr;
+  void* dst = nullptr;
   uint32_t bytes = 0;
+  const int R = p.rec_bytes;
+  const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
+  const int first = min(cnt, p.cap - pl.start);
+  const uint8_t* ring = static_cast<const uint8_t*>(p.ring) + bh * p.cap * R;
   if (lane == 0) {
     dst = st;
-    if (pl.fp32_tile) {
-      src = p.S + bh * P * N;
-      bytes = (uint32_t)(P * N * 4);
-    } else {
-      src = p.S8 + bh * P * N;
-      bytes = (uint32_t)(P * N);
-    }
+    src = pl.fp32_tile ? (const void*)(p.S + bh * P * N) : (const void*)(p.S8 + bh * P * N);
+    bytes = pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N);
   } else if (lane == 1) {
     if (!pl.fp32_tile) {
       dst = st + P * N;
       src = p.Sscale + bh * P;
       bytes = (uint32_t)(P * 4);
     }
-  } else if (lane < 8) {
-    if (c > 0) {
-      // live ring entries [start, start + c) modulo cap, in one or two pieces
-      const int first = min(c, p.cap - pl.start);
-      const int second = c - first;
-      const uint8_t* rk = static_cast<const uint8_t*>(p.ring_k) + ((size_t)pl.b * p.G + pl.g) * p.cap * N * S_IO;
-      const uint8_t* rv = static_cast<const uint8_t*>(p.ring_v) + bh * p.cap * P * S_IO;
-      if (lane == 2) {
-        dst = kbuf;
-        src = rk + (size_t)pl.start * N * S_IO;
-        bytes = (uint32_t)(first * N * S_IO);
-      } else if (lane == 3 && second > 0) {
-        dst = kbuf + (size_t)first * N * S_IO;
-        src = rk;
-        bytes = (uint32_t)(second * N * S_IO);
-      } else if (lane == 4) {
-        dst = vbuf;
-        src = rv + (size_t)pl.start * P * S_IO;
-        bytes = (uint32_t)(first * P * S_IO);
-      } else if (lane == 5 && second > 0) {
-        dst = vbuf + (size_t)first * P * S_IO;
-        src = rv;
-        bytes = (uint32_t)(second * P * S_IO);
-      } else if (lane == 6) {
-        dst = st + p.off_dtr;
-        src = p.ring_dt + bh * p.cap;
-        bytes = (uint32_t)(p.cap * 4);
-      } else if (lane == 7) {
-        dst = st + p.off_ar;
-        src = p.ring_a + bh * p.cap;
-        bytes = (uint32_t)(p.cap * 4);
-      }
+  } else if (lane == 2) {
+    dst = recbuf;
+    src = ring + (size_t)pl.start * R;
+    bytes = (uint32_t)(first * R);
+  } else if (lane == 3) {
+    if (cnt > first) {
+      dst = recbuf + (size_t)first * R;
+      src = ring;
+      bytes = (uint32_t)((cnt - first) * R);
     }
-  } else {
-    const int t = lane - 8;
-    const int s = t / 3;
-    if (s < n_new) {
-      const size_t tok = (size_t)pl.b * n_new + s;
-      const int which = t - 3 * s;
-      if (which == 0) {
-        dst = st + p.off_q + (size_t)s * N * S_IO;
-        src = static_cast<const uint8_t*>(p.q) + (tok * p.G + pl.g) * N * S_IO;
-        bytes = (uint32_t)(N * S_IO);
-      } else if (which == 1) {
-        dst = kbuf + (size_t)(c + s) * N * S_IO;
-        src = static_cast<const uint8_t*>(p.k) + (tok * p.G + pl.g) * N * S_IO;
-        bytes = (uint32_t)(N * S_IO);
-      } else {
-        dst = vbuf + (size_t)(c + s) * P * S_IO;
-        src = static_cast<const uint8_t*>(p.v) + (tok * p.H + pl.h) * P * S_IO;
-        bytes = (uint32_t)(P * S_IO);
-      }
+  } else if (lane == 4 && MODE == kModeReplay) {
+    dst = st + p.off_q;
+    const size_t bg = (size_t)pl.b * p.G + pl.g;
+    src = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
+                  : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
+    bytes = (uint32_t)(p.n_pos * N * S_IO);
+  }
+  if (bytes) {
+    if (lane == 0) {
+      bulk_g2s_hint(dst, src, bytes, bar, stream_policy);
+    } else {
+      bulk_g2s(dst, src, bytes, bar);
     }
   }
-  if (bytes) bulk_g2s(dst, src, bytes, bar);
 }
 
 template <int MODE, int CKPT, int S_IO>
-__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
+__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars, int pw) {
   const int lane = threadIdx.x & 31;
   const int NS = p.num_stages;
-  const int n_new = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
-  int32_t w_next = 0;
-  int m_next = 1;
-  float dt_next = 0.f, a_next = 0.f;
-  auto prefetch = [&](int uu) {
-    const int b = uu / p.H;
-    const int h = uu - b * p.H;
-    if (MODE != kModeEager && lane == 0) w_next = __ldg(p.counts_in + b);
-    if (MODE == kModeFlush && lane == 0) m_next = p.mask ? __ldg(p.mask + b) : 1;
-    if (lane < n_new) {
-      dt_next = __ldg(p.dt + ((size_t)b * n_new + lane) * p.H + h);
-      a_next = __ldg(p.a + ((size_t)b * n_new + lane) * p.H + h);
+  const uint64_t stream_policy = l2_evict_first_policy();
+  // Producer warp pw fills the CTA's units i = pw, pw + kProducerWarps, ... Their pointer
+  // words (and flush masks) are prefetched 32 units at a time, one chunk ahead: lane j
+  // of a chunk holds the word of the chunk's j-th unit.
+  auto unit_of = [&](int m) { return blockIdx.x + (pw + kProducerWarps * m) * gridDim.x; };
+  auto load_words = [&](int m0, int32_t& w, int& msk) {
+    w = 0;
+    msk = 1;
+    const int uu = unit_of(m0 + lane);
+    if (MODE != kModeEager && uu < p.num_units) {
+      const int b = uu / p.H;
+      w = __ldg(p.counts_in + b);
+      if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
     }
   };
-  int i = 0;
-  int u = blockIdx.x;
-  if (u < p.num_units) prefetch(u);
-  for (; u < p.num_units; u += gridDim.x, ++i) {
+  int32_t w_cur, w_nxt;
+  int m_cur, m_nxt;
+  load_words(0, w_cur, m_cur);
+  load_words(32, w_nxt, m_nxt);
+  int m = 0;
+  for (int u = unit_of(0); u < p.num_units; ++m, u = unit_of(m)) {
+    const int i = pw + kProducerWarps * m;  // the CTA-local unit index
     const int s = i % NS;
     const int k = i / NS;
+    if ((m & 31) == 0 && m > 0) {
+      w_cur = w_nxt;
+      m_cur = m_nxt;
+      load_words(m + 32, w_nxt, m_nxt);
+    }
     if (k > 0) {
       // every lane waits (each lane then writes into the stage), the warp agrees
       const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1));
@@ -248,35 +242,29 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     }
     int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
     if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
-    const int32_t word = __shfl_sync(0xffffffffu, w_next, 0);
-    const int msk = __shfl_sync(0xffffffffu, m_next, 0);
-    const float dtv = dt_next, av = a_next;
-    if (u + (int)gridDim.x < p.num_units) prefetch(u + gridDim.x);
+    const int32_t word = __shfl_sync(0xffffffffu, w_cur, m & 31);
+    const int msk = __shfl_sync(0xffffffffu, m_cur, m & 31);
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u, word, msk);
     uint8_t* st = stages + (size_t)s * p.stage_bytes;
-    if (lane < n_new) {
-      reinterpret_cast<float*>(st + p.off_dtn)[lane] = dtv;
-      reinterpret_cast<float*>(st + p.off_an)[lane] = av;
-    }
     if (lane == 0) {
       reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
       reinterpret_cast<int32_t*>(st + p.off_meta)[1] = msk;
-    }
-    __syncwarp();
-    if (lane == 0) {
       if (pl.corrupt) report_error(p.status, kErrPointer);
       mbar_arrive_expect_tx(&bars->full[s], pl.bytes);
     }
     __syncwarp();
-    if (pl.bytes) issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane);
-    __syncwarp();
+    issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane, stream_policy);
+    cp_async_arrive(&bars->full[s]);
+    if (lane == 0) bars->last_fill[s] = i;
   }
-  // Never leave with copies in flight into this CTA's shared memory: wait (bounded) for
-  // the last fill of every stage; fills the consumers already saw return at once.
-  if (lane == 0) {
-    const int first = i > NS ? i - NS : 0;
-    for (int j = first; j < i; ++j) {
-      if (!mbar_wait_bounded(&bars->full[j % NS], (j / NS) & 1)) report_error(p.status, kErrWaitTimeout);
+  // Never leave with copies in flight into this CTA's shared memory. A fill that was
+  // followed by a later fill of the same stage has been consumed; so once both producer
+  // warps are done, each waits (bounded) for the latest fill of every stage that it made.
+  asm volatile("bar.sync %0, %1;" ::"r"(kProducerBarrier), "r"(kProducerWarps * 32) : "memory");
+  for (int st_i = 0; st_i < NS; ++st_i) {
+    const int i = bars->last_fill[st_i];
+    if (i >= 0 && i % kProducerWarps == pw) {
+      if (!mbar_wait_bounded(&bars->full[st_i], (i / NS) & 1) && lane == 0) report_error(p.status, kErrWaitTimeout);
     }
   }
 }
@@ -284,8 +272,8 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
 // ---------------------------------------------------------------------------- consumers
 // kq[s][jj] = k_{o0+jj} . q_s for every query s < n and entry jj < width (<= 32).
 template <int N, typename IO, int GW>
-__device__ __forceinline__ void entry_dots(const uint8_t* kbuf, const uint8_t* qbuf, int o0, int width, int n,
-                                           float* kq, int gw, int lane) {
+__device__ __forceinline__ void entry_dots(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int o0,
+                                           int width, int n, float* kq, int gw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
   if constexpr (N == 128) {
     // a warp per (query, 8 entries): the lanes split N, a transposing reduction sums them
@@ -298,7 +286,7 @@ __device__ __forceinline__ void entry_dots(const uint8_t* kbuf, const uint8_t* q
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int jj = ch * 8 + r;
-        part[r] = (jj < width) ? dot4(IoT<IO>::load4(kbuf + ((size_t)(o0 + jj) * N + lane * 4) * S_IO), qv) : 0.f;
+        part[r] = (jj < width) ? dot4(IoT<IO>::load4(rec.k(o0 + jj) + lane * 4 * S_IO), qv) : 0.f;
       }
       int base;
       const bool wr = SegReduce<8, 32>::run(part, lane, base);
@@ -310,7 +298,7 @@ __device__ __forceinline__ void entry_dots(const uint8_t* kbuf, const uint8_t* q
     for (int t = gw * 32 + lane; t < n * width; t += GW * 32) {
       const int s = t / width;
       const int jj = t - s * width;
-      const uint8_t* kr = kbuf + (size_t)(o0 + jj) * N * S_IO;
+      const uint8_t* kr = rec.k(o0 + jj);
       const uint8_t* qr = qbuf + (size_t)s * N * S_IO;
       float d = 0.f;
 #pragma unroll
@@ -332,6 +320,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   constexpr int RT = kRowsPerThread;
   constexpr int RGR = RPG * RT;  // rows per row group
   constexpr int S_IO = IoT<IO>::bytes;
+  constexpr int NQR = NQ > 0 ? NQ : 1;
   using Red = SegReduce<RT, TPR>;
   const int lane = gtid & 31;
   const int gw = gtid >> 5;
@@ -345,28 +334,23 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const int width = c + n - o0;                                  // entries the outputs read
   const int fp = p.fp;
   const uint8_t* tile = st;
-  const uint8_t* kbuf = st + p.off_k;
-  const uint8_t* vbuf = st + p.off_v;
   const uint8_t* qbuf = st + p.off_q;
+  const Records<N, S_IO> rec{st + p.off_rec, P, p.rec_bytes};
   const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
   float* wout = reinterpret_cast<float*>(ws + p.ws_w);     // [kMaxPos][kMaxWindow] decay weight of entry o0+jj
   float* kq = reinterpret_cast<float*>(ws + p.ws_kq);      // [kMaxPos][kMaxWindow] k_{o0+jj} . q_s
   float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);
   float* sig = reinterpret_cast<float*>(ws + p.ws_sig);    // fold weights; [kMaxWindow] = abar
   float* wt = reinterpret_cast<float*>(ws + p.ws_wt);      // [P][fp] fold weight times v_j[p]
-  const EntryScalars<MODE> es{reinterpret_cast<const float*>(st + p.off_dtr), reinterpret_cast<const float*>(st + p.off_ar),
-                              reinterpret_cast<const float*>(st + p.off_dtn), reinterpret_cast<const float*>(st + p.off_an),
-                              pl.start, p.cap, c};
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   const int ngroups = (P + RGR - 1) / RGR;
 
-  float4 qr[NQ > 0 ? NQ : 1];
+  float4 qr[NQR];
 #pragma unroll
   for (int s = 0; s < NQ; ++s)
     qr[s] = (s < n) ? IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
 
-  // state rows of a row group; the first group is loaded before the scans so that its
-  // shared-memory latency overlaps them
+  // state rows of one row group (the read copy keeps its row scale for the dot product)
   auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
@@ -381,7 +365,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
             const float sc = scale_tile[pr];
             x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
           } else {
-            x[r] = e;  // read copy: the row scale is applied to the dot product
+            x[r] = e;
           }
         }
       }
@@ -390,25 +374,37 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   float4 x[RT];
   load_rows(x, 0, MODE == kModeEager);
 
-  // ---- phase A: decay scans (a warp per task) and k_j . q_s products
+  // output-only units with a single row group: the row dot products and their reduction
+  // need nothing from the scans, so they run first; the sums wait in registers
+  const bool early = !pl.fold && ngroups == 1;
+  float dv[NQR][Red::kHeld];
+  int dbase = 0;
+  bool dwr = false;
+  if (early) {
+#pragma unroll
+    for (int s = 0; s < NQ; ++s) {
+      if (s < n) {
+        float part[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
+        dwr = Red::run(part, lane, dbase);
+#pragma unroll
+        for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
+      }
+    }
+  }
+
+  // ---- phase A: decay scans (a warp per task, on the group's last warps) and k_j . q_s
   {
     const int tasks = ((MODE == kModeReplay) ? n : 0) + (cf > 0 ? 1 : 0);
-    for (int t = gw; t < tasks; t += GW) {
+    for (int t = GW - 1 - gw; t < tasks; t += GW) {
       const bool fold_task = !(MODE == kModeReplay && t < n);
+      const int last = fold_task ? cf - 1 : c + t - o0;  // last lane of the scanned window
+      const int e0 = fold_task ? 0 : o0;
       float xa = 1.f, xd = 0.f;
-      int last;  // last lane of the scanned window
-      if (fold_task) {
-        last = cf - 1;
-        if (lane <= last) {
-          xa = es.a(lane);
-          xd = es.dt(lane);
-        }
-      } else {
-        last = c + t - o0;
-        if (lane <= last) {
-          xa = es.a(o0 + lane);
-          xd = es.dt(o0 + lane);
-        }
+      if (lane <= last) {
+        xa = rec.a(e0 + lane);
+        xd = rec.dt(e0 + lane);
       }
       const float incl = warp_suffix_prod(xa, lane);  // prod_{lane <= i <= last} a_i
       float excl = __shfl_down_sync(0xffffffffu, incl, 1);
@@ -421,43 +417,52 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         if (lane == 0) alpha[t] = incl;
       }
     }
-    if (MODE == kModeReplay) entry_dots<N, IO, GW>(kbuf, qbuf, o0, width, n, kq, gw, lane);
+    if (MODE == kModeReplay) entry_dots<N, IO, GW>(rec, qbuf, o0, width, n, kq, gw, lane);
   }
   group_sync(bar_id, GT);
 
   // y = alpha_s d + sum_{jj} w_{s,jj} kq_{s,jj} v_{o0+jj}[p], by the lanes that hold row p's d
+  auto emit = [&](float d, int s, int pr) {
+    if (MODE == kModeReplay) {
+      const int last = c + s - o0;
+      float b0 = 0.f, b1 = 0.f;
+      int jj = 0;
+      for (; jj + 1 <= last; jj += 2) {
+        b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj], IoT<IO>::load1(rec.v(o0 + jj) + pr * S_IO), b0);
+        b1 = fmaf(wout[s * kMaxWindow + jj + 1] * kq[s * kMaxWindow + jj + 1],
+                  IoT<IO>::load1(rec.v(o0 + jj + 1) + pr * S_IO), b1);
+      }
+      if (jj <= last)
+        b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj], IoT<IO>::load1(rec.v(o0 + jj) + pr * S_IO), b0);
+      p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
+    } else {
+      p.y[bh * P + pr] = d;
+    }
+  };
   auto write_outputs = [&](float (&part)[RT], int s, int gi, bool from_tile_fp8) {
     int base;
     const bool wr = Red::run(part, lane, base);
 #pragma unroll
     for (int i = 0; i < Red::kHeld; ++i) {
       const int pr = gi * RGR + row0 + RPG * (base + i);
-      if (wr && pr < P) {
-        float d = part[i];
-        if (from_tile_fp8) d *= scale_tile[pr];
-        if (MODE == kModeReplay) {
-          const int last = c + s - o0;
-          float b0 = 0.f, b1 = 0.f;
-          int jj = 0;
-          for (; jj + 1 <= last; jj += 2) {
-            b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj],
-                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj) * P + pr) * S_IO), b0);
-            b1 = fmaf(wout[s * kMaxWindow + jj + 1] * kq[s * kMaxWindow + jj + 1],
-                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj + 1) * P + pr) * S_IO), b1);
-          }
-          if (jj <= last)
-            b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj],
-                      IoT<IO>::load1(vbuf + ((size_t)(o0 + jj) * P + pr) * S_IO), b0);
-          p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
-        } else {
-          p.y[bh * P + pr] = d;
-        }
-      }
+      if (wr && pr < P) emit(from_tile_fp8 ? part[i] * scale_tile[pr] : part[i], s, pr);
     }
   };
 
-  if (!pl.fold) {
-    // ---- phase B: output-only route from the stored checkpoint
+  if (early) {
+    // ---- phase B: combine the early row sums with the buffer term
+#pragma unroll
+    for (int s = 0; s < NQ; ++s) {
+      if (s < n) {
+#pragma unroll
+        for (int i = 0; i < Red::kHeld; ++i) {
+          const int pr = row0 + RPG * (dbase + i);
+          if (dwr && pr < P) emit(pl.fp32_tile ? dv[s][i] : dv[s][i] * scale_tile[pr], s, pr);
+        }
+      }
+    }
+  } else if (!pl.fold) {
+    // ---- phase B: output-only route, several row groups
     for (int gi = 0; gi < ngroups; ++gi) {
       if (gi > 0) load_rows(x, gi, false);
 #pragma unroll
@@ -476,7 +481,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     for (int idx = gtid; idx < P * cf_pad; idx += GT) {
       const int pp = idx / cf_pad;
       const int j = idx - pp * cf_pad;
-      wt[pp * fp + j] = j < cf ? sig[j] * IoT<IO>::load1(vbuf + ((size_t)j * P + pp) * S_IO) : 0.f;
+      wt[pp * fp + j] = j < cf ? sig[j] * IoT<IO>::load1(rec.v(j) + pp * S_IO) : 0.f;
     }
     group_sync(bar_id, GT);
     const float abar = sig[kMaxWindow];
@@ -489,7 +494,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 #pragma unroll
         for (int jj = 0; jj < kFoldChunk; ++jj) {
           const int j = ch + jj;
-          kr[jj] = (j < cf) ? IoT<IO>::load4(kbuf + ((size_t)j * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
+          kr[jj] = (j < cf) ? IoT<IO>::load4(rec.k(j) + col * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
@@ -517,13 +522,13 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
         const int pr = gi * RGR + row0 + RPG * r;
-        if (store_f32 && pr < P) *reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col) = x[r];
+        if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col), x[r]);
         if (store_fp8) {
           const float am = seg_allmax<TPR>(amax4(x[r]));
           float sc, inv;
           e4m3_row_scale(am, sc, inv);
           if (pr < P) {
-            *reinterpret_cast<uint32_t*>(p.S8 + (bh * P + pr) * N + col) = quant4_e4m3(x[r], inv);
+            __stcs(reinterpret_cast<unsigned int*>(p.S8 + (bh * P + pr) * N + col), quant4_e4m3(x[r], inv));
             if ((lane % TPR) == 0) p.Sscale[bh * P + pr] = sc;
           }
         }
@@ -542,37 +547,10 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     }
   }
 
-  // ---- phase C: append this call's entries to the ring, publish the pointer word
+  // ---- publish the pointer word (the pre-pass already wrote this call's entries)
   const int start = pl.start;
   const int cap = p.cap;
   if (MODE == kModeReplay) {
-    const int kchunks = N * S_IO / 16;
-    const int vchunks = P * S_IO / 16;
-    uint8_t* rk = static_cast<uint8_t*>(p.ring_k) + ((size_t)pl.b * p.G + pl.g) * cap * N * S_IO;
-    uint8_t* rv = static_cast<uint8_t*>(p.ring_v) + bh * cap * P * S_IO;
-    const bool write_k = (pl.h % p.hpg) == 0;
-    const int total = n * (kchunks + vchunks);
-    for (int idx = gtid; idx < total; idx += GT) {
-      const int s = idx / (kchunks + vchunks);
-      const int ch = idx - s * (kchunks + vchunks);
-      int slot_i = start + c + s;
-      slot_i -= (slot_i >= cap) ? cap : 0;
-      if (ch < kchunks) {
-        if (write_k)
-          *reinterpret_cast<uint4*>(rk + (size_t)slot_i * N * S_IO + ch * 16) =
-              *reinterpret_cast<const uint4*>(kbuf + (size_t)(c + s) * N * S_IO + ch * 16);
-      } else {
-        const int cv = ch - kchunks;
-        *reinterpret_cast<uint4*>(rv + (size_t)slot_i * P * S_IO + cv * 16) =
-            *reinterpret_cast<const uint4*>(vbuf + (size_t)(c + s) * P * S_IO + cv * 16);
-      }
-    }
-    if (gtid < n) {
-      int slot_i = start + c + gtid;
-      slot_i -= (slot_i >= cap) ? cap : 0;
-      p.ring_dt[bh * cap + slot_i] = reinterpret_cast<const float*>(st + p.off_dtn)[gtid];
-      p.ring_a[bh * cap + slot_i] = reinterpret_cast<const float*>(st + p.off_an)[gtid];
-    }
     if (pl.h == 0 && gtid == 0) {
       int start2 = pl.fold ? start + c : start;
       start2 -= (start2 >= cap) ? cap : 0;
@@ -593,6 +571,8 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 
 template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
 __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_constant__ KParams p) {
+  static_assert(NG == 1 || NG == 2, "the stage protocol relies on a stage's uses two apart being one group's");
+  static_assert(kProducerWarps == 1, "stages must be filled in unit order");
   using Gr = Groups<NG>;
   extern __shared__ __align__(128) uint8_t smem[];
   Bars* bars = reinterpret_cast<Bars*>(smem);
@@ -601,17 +581,18 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.num_stages; ++s) {
-      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->full[s], 1 + 32);  // the filling warp: lane 0's expect_tx + 32 lanes' cp.async
       mbar_init(&bars->empty[s], Gr::kThreads);
     }
     bars->abort_flag = 0;
+    for (int s = 0; s < kMaxStages; ++s) bars->last_fill[s] = -1;
     fence_mbar_init();
   }
   __syncthreads();
 
   const int warp = threadIdx.x / 32;
-  if (warp == kConsumerWarps) {
-    producer_loop<MODE, CKPT, S_IO>(p, stages, bars);
+  if (warp >= kConsumerWarps) {
+    producer_loop<MODE, CKPT, S_IO>(p, stages, bars, warp - kConsumerWarps);
     return;
   }
   const int g = warp / Gr::kWarps;  // consumer group
@@ -622,7 +603,16 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   int i = g;
   for (int u = blockIdx.x + g * gridDim.x; u < p.num_units; u += NG * gridDim.x, i += NG) {
     const int s = i % NS;
-    const bool ok = group_all(mbar_wait_bounded(&bars->full[s], (i / NS) & 1), bar_id, Gr::kThreads);
+    const int k = i / NS;  // this is the k-th use of stage s
+    // Parity waits only tell apart a phase and the one just before it, so before waiting
+    // for its own fill (phase k of "full"), a group waits for the stage's previous use to
+    // be released (phase k-1 of "empty"). That release may come from the other group;
+    // the use before it (k-2) was this group's own, already released, so both waits are
+    // exact even when the two groups drift apart.
+    bool ready = true;
+    if (k > 0) ready = mbar_wait_bounded(&bars->empty[s], (k - 1) & 1);
+    if (ready) ready = mbar_wait_bounded(&bars->full[s], k & 1);
+    const bool ok = group_all(ready, bar_id, Gr::kThreads);
     if (!ok) {
       if (gtid == 0) {
         report_error(p.status, kErrWaitTimeout);

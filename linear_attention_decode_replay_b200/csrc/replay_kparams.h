@@ -1,4 +1,4 @@
-// Launch parameters shared by the host launcher and the replay kernel.
+// Launch parameters shared by the host launcher and the replay kernels.
 #pragma once
 
 #include <stdint.h>
@@ -25,20 +25,32 @@ struct KParams {
   float* S;
   uint8_t* S8;
   float* Sscale;
-  void* ring_k;
-  void* ring_v;
-  float* ring_dt;
-  float* ring_a;
+  void* ring;          // [B][H][cap] records of rec_bytes: k (N io), v (P io), Delta, a
+  const void* qpack;   // [B][G][qpack_pos][N] io verify queries packed per group, or null
   const int32_t* counts_in;
   int32_t* counts_out;
   int32_t* status;
   // shared-memory layout, bytes
   int32_t num_stages, stage_bytes, stages_off;
-  int32_t off_k, off_v, off_q, off_dtr, off_ar, off_dtn, off_an, off_meta;  // within a stage
+  int32_t rec_bytes, qpack_pos;                // ring record size; positions per qpack group
+  int32_t off_rec, off_q, off_meta;            // within a stage
   int32_t ws_off, ws_group_bytes;          // one workspace per consumer group
   int32_t ws_w, ws_kq, ws_alpha, ws_sig, ws_wt;  // within a group's workspace
   int32_t fp;                               // fold entries per state row in ws_wt, padded
   int32_t smem_bytes;
+};
+
+// The pre-pass that writes this call's new entries into their ring records.
+struct PackParams {
+  int32_t B, H, G, P, N, L, cap, n_pos, hpg, rec_bytes, io_bytes, qpack_pos;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* dt;
+  const float* a;
+  void* ring;
+  void* qpack;  // null: no packing of the queries
+  const int32_t* counts_in;
 };
 
 }  // namespace replay

@@ -14,6 +14,7 @@ cudaError_t launch_replay_n32(const KParams& p, int io, int ckpt, int mode, int 
 cudaError_t launch_replay_n64(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
 cudaError_t launch_replay_n128(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
 
+cudaError_t launch_pack_entries(const PackParams& pp, int grid, cudaStream_t s);
 cudaError_t launch_quantize_rows(const float* x, long long rows, int n, unsigned char* codes, float* scale,
                                  int grid, cudaStream_t s);
 cudaError_t launch_rollback(const int* counts_in, int* counts_out, const int* n_keep, int B, int n_pos,

@@ -1,4 +1,5 @@
-// Launchers of the small kernels: per-row e4m3 quantisation and rollback.
+// Small kernels and their launchers: the entry pre-pass, per-row e4m3 quantisation and
+// rollback.
 #include "replay_kernel.cuh"
 #include "replay_launch.h"
 
@@ -20,6 +21,60 @@ __global__ void rollback_kernel(const int32_t* __restrict__ counts_in, int32_t* 
   }
 }
 
+
+// Writes this call's new entries into their ring records before the main kernel runs:
+// record (start + c + s) mod cap of (b, h) gets k, v, Delta, a of position s, where
+// (start, c) is the sequence's current pointer word. A flush in the main kernel reads
+// records [start, start + c) and the appends land in [start + c, start + c + n_pos), so
+// the two never overlap (cap = L + max_pos). Verify queries are also gathered per group
+// into qpack so that a unit's queries are one contiguous piece. One warp per (b, h).
+__global__ void pack_entries_kernel(const PackParams pp) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x / 32;
+  const int S = pp.io_bytes;
+  const int kpe = pp.N * S / 16;  // 16-byte chunks of a k (or q) row
+  const int vpe = pp.P * S / 16;
+  const long long total = (long long)pp.B * pp.H;
+  for (long long task = (long long)blockIdx.x * wpb + threadIdx.x / 32; task < total; task += (long long)gridDim.x * wpb) {
+    const int b = (int)(task / pp.H);
+    const int h = (int)(task - (long long)b * pp.H);
+    const int g = h / pp.hpg;
+    const int32_t word = pp.counts_in[b];
+    const int start = word >> 16;
+    const int c = word & 0xFFFF;
+    if (word < 0 || c > pp.L || start >= pp.cap) continue;  // the main kernel reports it
+    for (int s = 0; s < pp.n_pos; ++s) {
+      int slot = start + c + s;
+      slot -= (slot >= pp.cap) ? pp.cap : 0;
+      uint8_t* rec = static_cast<uint8_t*>(pp.ring) + (((size_t)b * pp.H + h) * pp.cap + slot) * pp.rec_bytes;
+      const size_t tok = (size_t)b * pp.n_pos + s;
+      const uint8_t* kin = static_cast<const uint8_t*>(pp.k) + (tok * pp.G + g) * pp.N * S;
+      const uint8_t* vin = static_cast<const uint8_t*>(pp.v) + (tok * pp.H + h) * pp.P * S;
+      for (int idx = lane; idx < kpe + vpe; idx += 32) {
+        if (idx < kpe) {
+          reinterpret_cast<uint4*>(rec)[idx] = reinterpret_cast<const uint4*>(kin)[idx];
+        } else {
+          reinterpret_cast<uint4*>(rec + pp.N * S)[idx - kpe] = reinterpret_cast<const uint4*>(vin)[idx - kpe];
+        }
+      }
+      if (lane == 0) {
+        float* sc = reinterpret_cast<float*>(rec + (pp.N + pp.P) * S);
+        sc[0] = pp.dt[tok * pp.H + h];
+        sc[1] = pp.a[tok * pp.H + h];
+      }
+      if (pp.qpack && (h % pp.hpg) == 0) {
+        const uint8_t* qin = static_cast<const uint8_t*>(pp.q) + (tok * pp.G + g) * pp.N * S;
+        uint8_t* qout = static_cast<uint8_t*>(pp.qpack) + (((size_t)b * pp.G + g) * pp.qpack_pos + s) * pp.N * S;
+        for (int idx = lane; idx < kpe; idx += 32) reinterpret_cast<uint4*>(qout)[idx] = reinterpret_cast<const uint4*>(qin)[idx];
+      }
+    }
+  }
+}
+
+cudaError_t launch_pack_entries(const PackParams& pp, int grid, cudaStream_t s) {
+  pack_entries_kernel<<<grid, 256, 0, s>>>(pp);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_rows(const float* x, long long rows, int n, unsigned char* codes, float* scale,
                                  int grid, cudaStream_t s) {

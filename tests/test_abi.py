@@ -25,7 +25,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("replay_init", "replay_step", "replay_verify", "replay_rollback", "replay_flush",
                  "replay_read_counts", "replay_check_status", "replay_destroy", "eager_step",
-                 "eager_step_fp8", "replay_quantize_rows_e4m3", "replay_ring_capacity", "replay_strerror"):
+                 "eager_step_fp8", "replay_quantize_rows_e4m3", "replay_ring_capacity", "replay_ring_record_bytes",
+                 "replay_strerror"):
         assert want in names
 
 
@@ -44,29 +45,36 @@ def _cfg(**kw):
 
 def test_ring_capacity_and_config_checks():
     lib = _abi.load()
-    assert lib.replay_ring_capacity(ctypes.byref(_cfg())) == 8  # 4 + 2 rounded up to 4
-    assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=1))) == 20
-    assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=5))) == 24
+    assert lib.replay_ring_capacity(ctypes.byref(_cfg())) == 6  # L + max_pos
+    assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=1))) == 17
+    assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=5))) == 21
+    # record: k (N io) + v (P io) + Delta + a, padded to 16 bytes
+    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg())) == 144  # (16 + 16) * 4 + 8 -> 144
+    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 400
     for bad in (dict(groups=3), dict(P=12), dict(P=0), dict(N=48), dict(N=256), dict(L=0),
                 dict(max_pos=9), dict(max_pos=5, L=4), dict(io=7), dict(ckpt=3), dict(batch=0),
                 dict(P=256, N=128)):
         assert lib.replay_ring_capacity(ctypes.byref(_cfg(**bad))) == _abi.REPLAY_EINVAL, bad
+        assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(**bad))) == _abi.REPLAY_EINVAL, bad
 
 
 def test_init_rejects_bad_arguments_before_any_cuda_call():
     lib = _abi.load()
     ctx = ctypes.c_void_p()
     good = ctypes.c_void_p(0x10000)
-    bufs = _abi.CBuffers(good, None, None, good, good, good, good, good, good)
+    bufs = _abi.CBuffers(good, None, None, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg(groups=3)), ctypes.byref(bufs), None, ctypes.byref(ctx)) == \
         _abi.REPLAY_EINVAL
-    nulls = _abi.CBuffers(None, None, None, good, good, good, good, good, good)
+    nulls = _abi.CBuffers(None, None, None, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(nulls), None, ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
-    odd = _abi.CBuffers(ctypes.c_void_p(0x10008), None, None, good, good, good, good, good, good)
+    odd = _abi.CBuffers(ctypes.c_void_p(0x10008), None, None, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(odd), None, ctypes.byref(ctx)) == _abi.REPLAY_EALIGN
-    fp8_missing = _abi.CBuffers(good, None, None, good, good, good, good, good, good)
+    fp8_missing = _abi.CBuffers(good, None, None, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg(ckpt=_abi.REPLAY_CKPT_F32_FP8READ)), ctypes.byref(fp8_missing), None,
                            ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
+    no_qpack = _abi.CBuffers(good, None, None, good, None, good, good)
+    assert lib.replay_init(ctypes.byref(_cfg(max_pos=2)), ctypes.byref(no_qpack), None, ctypes.byref(ctx)) == \
+        _abi.REPLAY_EINVAL
     assert not ctx.value
 
 

@@ -98,6 +98,13 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// L2 policy for everything else the kernel reads (ring records, queries): normal priority.
+__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // ---------------------------------------------------------------- cp.async (LDGSTS)
 // Small global -> shared copies issued per thread; their completion is tracked by an
 // mbarrier through cp_async_arrive (each issuing thread arrives once per phase).

@@ -125,7 +125,7 @@ struct Records {
 // no ring: its new token's k, v, Delta, a (and q) are gathered with per-lane cp.async.
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& pl, uint8_t* st, uint64_t* bar,
-                                                  int lane, uint64_t stream_policy) {
+                                                  int lane, uint64_t stream_policy, uint64_t keep_policy) {
   const size_t P = p.P, N = p.N;
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   if (!pl.active) return;
@@ -153,47 +153,34 @@ __device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& 
     if (lane == 1) cp_async4(recbuf + (N + P) * S_IO + 4, p.a + bh);
     return;
   }
-  const void* src = nullptr;
-  void* dst = nullptr;
-  uint32_t bytes = 0;
+  // every lane works out its copy without branching, then one predicated instruction
+  // issues all of them
   const int R = p.rec_bytes;
   const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
   const int first = min(cnt, p.cap - pl.start);
   const uint8_t* ring = static_cast<const uint8_t*>(p.ring) + bh * p.cap * R;
-  if (lane == 0) {
-    dst = st;
-    src = pl.fp32_tile ? (const void*)(p.S + bh * P * N) : (const void*)(p.S8 + bh * P * N);
-    bytes = pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N);
-  } else if (lane == 1) {
-    if (!pl.fp32_tile) {
-      dst = st + P * N;
-      src = p.Sscale + bh * P;
-      bytes = (uint32_t)(P * 4);
-    }
-  } else if (lane == 2) {
-    dst = recbuf;
-    src = ring + (size_t)pl.start * R;
-    bytes = (uint32_t)(first * R);
-  } else if (lane == 3) {
-    if (cnt > first) {
-      dst = recbuf + (size_t)first * R;
-      src = ring;
-      bytes = (uint32_t)((cnt - first) * R);
-    }
-  } else if (lane == 4 && MODE == kModeReplay) {
-    dst = st + p.off_q;
-    const size_t bg = (size_t)pl.b * p.G + pl.g;
-    src = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
-                  : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
-    bytes = (uint32_t)(p.n_pos * N * S_IO);
-  }
-  if (bytes) {
-    if (lane == 0) {
-      bulk_g2s_hint(dst, src, bytes, bar, stream_policy);
-    } else {
-      bulk_g2s(dst, src, bytes, bar);
-    }
-  }
+  const size_t bg = (size_t)pl.b * p.G + pl.g;
+  const uint8_t* qsrc = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
+                                : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
+  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + bh * P * N) : p.S8 + bh * P * N;
+  const uint8_t* src = (lane == 0)   ? tsrc
+                       : (lane == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + bh * P)
+                       : (lane == 2) ? ring + (size_t)pl.start * R
+                       : (lane == 3) ? ring
+                                     : qsrc;
+  uint8_t* dst = (lane == 0)   ? st
+                 : (lane == 1) ? st + P * N
+                 : (lane == 2) ? recbuf
+                 : (lane == 3) ? recbuf + (size_t)first * R
+                               : st + p.off_q;
+  uint32_t bytes = 0;
+  bytes = (lane == 0) ? (pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N)) : bytes;
+  bytes = (lane == 1 && !pl.fp32_tile) ? (uint32_t)(P * 4) : bytes;
+  bytes = (lane == 2) ? (uint32_t)(first * R) : bytes;
+  bytes = (lane == 3) ? (uint32_t)((cnt - first) * R) : bytes;
+  bytes = (lane == 4 && MODE == kModeReplay) ? (uint32_t)(p.n_pos * N * S_IO) : bytes;
+  __syncwarp();
+  if (bytes) bulk_g2s_hint(dst, src, bytes, bar, lane == 0 ? stream_policy : keep_policy);
 }
 
 template <int MODE, int CKPT, int S_IO>
@@ -201,6 +188,7 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars, int
   const int lane = threadIdx.x & 31;
   const int NS = p.num_stages;
   const uint64_t stream_policy = l2_evict_first_policy();
+  const uint64_t keep_policy = l2_evict_normal_policy();
   // Producer warp pw fills the CTA's units i = pw, pw + kProducerWarps, ... Their pointer
   // words (and flush masks) are prefetched 32 units at a time, one chunk ahead: lane j
   // of a chunk holds the word of the chunk's j-th unit.
@@ -253,7 +241,7 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars, int
       mbar_arrive_expect_tx(&bars->full[s], pl.bytes);
     }
     __syncwarp();
-    issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane, stream_policy);
+    issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane, stream_policy, keep_policy);
     cp_async_arrive(&bars->full[s]);
     if (lane == 0) bars->last_fill[s] = i;
   }

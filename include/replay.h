@@ -52,7 +52,9 @@ typedef enum {
   REPLAY_EPENDING = -4,    /* a verify is pending: call replay_rollback first */
   REPLAY_ENOPENDING = -5,  /* replay_rollback without a pending verify */
   REPLAY_EDEVICE = -6,     /* the device status word is non-zero (see replay_check_status) */
-  REPLAY_ENOMEM = -7       /* host allocation of the context failed */
+  REPLAY_ENOMEM = -7,      /* host allocation of the context failed */
+  REPLAY_ESCRATCH = -8     /* replay_verify_static_scratch: the call's queries exceed
+                              REPLAY_STATIC_SCRATCH_BYTES */
 } replay_status;
 
 typedef enum { REPLAY_F32 = 0, REPLAY_BF16 = 1 } replay_dtype;
@@ -189,6 +191,43 @@ int eager_step_fp8(const replay_config* cfg, uint8_t* S8, float* scale, const vo
  *   n: 16, 32, 64 or 128. */
 int replay_quantize_rows_e4m3(const float* x, int64_t rows, int32_t n, uint8_t* codes,
                               float* scale, replay_stream_t stream);
+
+/* ---- Verify without a query buffer from the caller (library extension) ----
+ * The paper has no counterpart to this call. It serves callers that cannot allocate
+ * device memory: a layer hosted by a program that owns all of the GPU's memory (a serving
+ * engine that gives the free HBM to its own cache pool at start-up and hands each layer
+ * only its state and per-call tensors), or a plug-in interface that passes inputs and
+ * outputs but offers no way to ask for extra buffers. Such a caller cannot cudaMalloc the
+ * qpack buffer that replay_verify needs when max_pos > 1.
+ *
+ * Size of the fixed device array that holds the packed queries: 32 MiB, enough for
+ * B * G * n_pos * N io values up to B = 256, G = 64, n_pos = 8, N = 128 in BF16. */
+#define REPLAY_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* replay_verify with the queries packed into the library's own fixed device array instead
+ * of bufs.qpack, which this call never touches (it may be NULL: a context made with
+ * max_pos = 1 needs none). Arguments, outputs and the pending-verify protocol are those of
+ * replay_verify, with these differences:
+ *  - Limit: B * G * n_pos * N * s bytes (s = 2 for BF16, 4 for FP32) must not exceed
+ *    REPLAY_STATIC_SCRATCH_BYTES, else REPLAY_ESCRATCH is returned and nothing is queued.
+ *  - 1 <= n_pos <= min(L, 8), even above the context's max_pos. When n_pos > max_pos the
+ *    ring (L + max_pos records) has room for n_pos new entries only beside an empty
+ *    buffer, so the call first folds every sequence's buffer into its checkpoint, as
+ *    replay_flush(ctx, NULL, stream) does: one more state read and write, not reported
+ *    in `flushed`.
+ *  - Allocation: none, on the device or the host. The array is part of the library's
+ *    device code, so every GPU that loads libreplay.so holds its 32 MiB until the process
+ *    exits.
+ *  - Set-up: the first call with n_pos > 1 on a device looks up that device's copy of the
+ *    array (cudaGetSymbolAddress); it must run with the context's device current (else
+ *    REPLAY_EINVAL), and it should come before any stream capture.
+ *  - Sharing: every call on a device, from any context, stream or thread, uses the same
+ *    array. Calls whose work overlaps on the GPU race and corrupt each other's queries;
+ *    order them (one stream, or events). The array keeps the last call's contents, but
+ *    nothing in it needs to start at zero: a call writes each query before reading it. */
+int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k,
+                                 const void* v, const float* dt, const float* a, float* y,
+                                 uint8_t* flushed, replay_stream_t stream);
 
 /* Static text for a replay_status code. */
 const char* replay_strerror(int code);

@@ -173,6 +173,24 @@ class Replay:
               "replay_verify")
         return y
 
+    def verify_static_scratch(self, q, k, v, dt, a, y=None, flushed=None, stream=None):
+        """verify() for callers that cannot allocate device memory: the queries are packed
+        into the library's fixed 32 MiB device array instead of the qpack buffer, so the
+        layer needs no qpack (max_pos = 1 works; n_pos above max_pos first folds every
+        buffer). Calls that overlap on the GPU share that array and race. Pass `y` to
+        keep this binding from allocating the output itself."""
+        n_pos = q.shape[1]
+        qs, vs, ds = self._token_shapes(n_pos)
+        t = self.cfg.io_dtype
+        if y is None:
+            y = torch.empty(vs, device=q.device, dtype=torch.float32)
+        check(self._lib.replay_verify_static_scratch(
+            self._ctx, n_pos, _ptr(q, qs, t, "q"), _ptr(k, qs, t, "k"), _ptr(v, vs, t, "v"),
+            _ptr(dt, ds, torch.float32, "dt"), _ptr(a, ds, torch.float32, "a"), _ptr(y, vs, torch.float32, "y"),
+            _ptr(flushed, (self.cfg.batch,), torch.uint8, "flushed"), _stream(stream)),
+            "replay_verify_static_scratch")
+        return y
+
     def rollback(self, n_keep, stream=None):
         """Keep n_keep[b] (int32 [B] on the device) of the pending verify's positions."""
         check(self._lib.replay_rollback(self._ctx, _ptr(n_keep, (self.cfg.batch,), torch.int32, "n_keep"),

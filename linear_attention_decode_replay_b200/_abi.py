@@ -19,6 +19,10 @@ REPLAY_EPENDING = -4
 REPLAY_ENOPENDING = -5
 REPLAY_EDEVICE = -6
 REPLAY_ENOMEM = -7
+REPLAY_ESCRATCH = -8
+
+# size of the library's fixed query scratch (replay_verify_static_scratch)
+STATIC_SCRATCH_BYTES = 32 << 20
 
 REPLAY_F32 = 0
 REPLAY_BF16 = 1
@@ -68,6 +72,7 @@ def load() -> ctypes.CDLL:
         "replay_init": (ctypes.c_int, [cfgp, ctypes.POINTER(CBuffers), vp, ctypes.POINTER(vp)]),
         "replay_step": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_verify": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "replay_verify_static_scratch": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_rollback": (ctypes.c_int, [vp, vp, vp]),
         "replay_flush": (ctypes.c_int, [vp, vp, vp]),
         "replay_read_counts": (ctypes.c_int, [vp, vp, vp]),

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/replay.h"
@@ -439,8 +440,117 @@ const char* replay_strerror(int code) {
     case REPLAY_ENOPENDING: return "no verify is pending";
     case REPLAY_EDEVICE: return "device reported an error (see the status bits)";
     case REPLAY_ENOMEM: return "host allocation failed";
+    case REPLAY_ESCRATCH: return "the call needs more query scratch than REPLAY_STATIC_SCRATCH_BYTES";
     default: return "unknown status";
   }
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Verify with the query scratch in a fixed device array (replay_verify_static_scratch).
+// A library extension without a counterpart in the method: for callers that cannot
+// allocate device memory, so cannot give replay_init a qpack buffer.
+// ---------------------------------------------------------------------------------------
+
+// The scratch itself. Every GPU that loads this library holds it until the process exits.
+// In host code this name is only a handle for the runtime, not a device address.
+static __device__ __align__(256) unsigned char replay_static_qpack[REPLAY_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kScratchDevices];  // per device: its copy of replay_static_qpack
+
+// Set-up, once per device, with that device current: its address of the scratch array.
+int static_scratch_address(int device, void** out) {
+  if (device < 0 || device >= kScratchDevices) return REPLAY_EINVAL;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[device]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress((void**)&ptr, replay_static_qpack) != cudaSuccess || !ptr) return REPLAY_ECUDA;
+    g_scratch_addr[device] = ptr;
+  }
+  *out = g_scratch_addr[device];
+  return REPLAY_OK;
+}
+
+}  // namespace
+
+extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k,
+                                            const void* v, const float* dt, const float* a, float* y,
+                                            uint8_t* flushed, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  const replay_config& cfg = ctx->cfg;
+  if (n_pos < 1 || n_pos > replay::kMaxPos || n_pos > cfg.L) return REPLAY_EINVAL;
+  const int64_t s_io = cfg.io == REPLAY_BF16 ? 2 : 4;
+  const int64_t need = n_pos > 1 ? (int64_t)cfg.batch * cfg.groups * n_pos * cfg.N * s_io : 0;
+  if (need > (int64_t)REPLAY_STATIC_SCRATCH_BYTES) return REPLAY_ESCRATCH;
+  int rc = check_inputs(q, k, v, dt, a, y);
+  if (rc) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n_pos == 1) {
+    // a single position packs no queries: the plain tentative step, no scratch
+    rc = replay_call(ctx, 1, 0, q, k, v, dt, a, y, flushed, s);
+    if (rc == REPLAY_OK) ctx->pending = 1;
+    return rc;
+  }
+  DeviceInfo d;
+  if ((rc = device_info(&d))) return rc;
+  if (d.device != ctx->device) return REPLAY_EINVAL;
+  void* scratch = nullptr;
+  if ((rc = static_scratch_address(d.device, &scratch))) return rc;
+  replay_config c = cfg;
+  c.max_pos = n_pos;
+  KParams p;
+  if ((rc = build_layout(&p, c, replay::kModeReplay, 0, ctx->cap, d.smem_optin))) return rc;
+  if (cfg.max_pos < n_pos) {
+    // a ring of L + max_pos records holds n_pos new entries only beside an empty buffer
+    if ((rc = replay_flush(ctx, nullptr, stream))) return rc;
+  }
+  set_state(&p, ctx);
+  p.qpack = scratch;
+  p.qpack_pos = n_pos;
+  p.n_pos = n_pos;
+  p.commit = 0;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.dt = dt;
+  p.a = a;
+  p.y = y;
+  p.flushed = flushed;
+  replay::PackParams pp;
+  pp.B = p.B;
+  pp.H = p.H;
+  pp.G = p.G;
+  pp.P = p.P;
+  pp.N = p.N;
+  pp.L = p.L;
+  pp.cap = p.cap;
+  pp.n_pos = n_pos;
+  pp.hpg = p.hpg;
+  pp.rec_bytes = p.rec_bytes;
+  pp.io_bytes = (int)s_io;
+  pp.qpack_pos = n_pos;
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.dt = dt;
+  pp.a = a;
+  pp.ring = ctx->bufs.ring;
+  pp.qpack = scratch;
+  pp.counts_in = p.counts_in;
+  const long long tasks = (long long)p.B * p.H;
+  const long long blocks = (tasks + 7) / 8;
+  const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
+  if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
+  const int ckpt = cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
+  if (launch_main(p, cfg, ckpt, replay::kModeReplay, replay::kMaxPos, ctx->num_sms, s) != cudaSuccess)
+    return REPLAY_ECUDA;
+  ctx->parity ^= 1;
+  ctx->pending = n_pos;
+  return REPLAY_OK;
+}

@@ -29,7 +29,7 @@ struct replay_ctx {
 namespace {
 
 constexpr int kHeaderBytes = 256;  // the kernel's mbarriers and abort flag
-constexpr int kGroups = 2;         // consumer groups per CTA (must match the launcher)
+constexpr int kGroups = replay::kGroups;  // consumer groups per CTA
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -96,15 +96,14 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
   p->stage_bytes = round_up(p->off_meta + 16, 128);
 
-  // one workspace per consumer group: decay weights and k.q of the outputs
-  // [kMaxPos][kMaxWindow] each, alpha[kMaxPos], fold weights [kMaxWindow] + abar, and the
-  // fold weights times v, [P][fp]
+  // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
+  // abar, the buffer terms of the outputs u[nq_alloc][P], and the fold weights times v,
+  // [P][fp]
   p->fp = round_up(lfold, replay::kFoldChunk);
-  p->ws_w = 0;
-  p->ws_kq = p->ws_w + replay::kMaxPos * replay::kMaxWindow * 4;
-  p->ws_alpha = p->ws_kq + replay::kMaxPos * replay::kMaxWindow * 4;
+  p->ws_alpha = 0;
   p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
-  p->ws_wt = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
+  p->ws_u = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
+  p->ws_wt = round_up(p->ws_u + nq_alloc * P * 4, 16);
   p->ws_group_bytes = round_up(p->ws_wt + P * p->fp * 4, 128);
   p->ws_off = kHeaderBytes;
   p->stages_off = round_up(p->ws_off + kGroups * p->ws_group_bytes, 128);

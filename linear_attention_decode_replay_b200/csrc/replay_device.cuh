@@ -10,13 +10,16 @@
 
 namespace replay {
 
-constexpr int kConsumerWarps = 8;               // warps that compute units (split into groups)
-constexpr int kProducerWarps = 1;               // warps that fill stages, in unit order
-constexpr int kProducerBarrier = 15;            // named barrier joining the producer warps
+constexpr int kGroupGemvWarps = 4;              // per consumer group: warps that stream the state rows
+constexpr int kGroupWarps = kGroupGemvWarps + 1; // ... plus one warp for the buffer coefficients
+constexpr int kGroups = 2;                       // consumer groups per CTA
+constexpr int kConsumerWarps = kGroups * kGroupWarps;
+constexpr int kProducerWarps = 1;                // the warp that fills stages, in unit order
 constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
 constexpr int kMaxPos = 8;                       // query positions per verify call
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
 constexpr int kMaxStages = 8;
+constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
 constexpr int kFoldChunk = 8;                    // buffer entries folded per register pass
 constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock

@@ -17,7 +17,7 @@ constexpr int kMaxDevices = 64;
 
 template <typename IO, int CKPT, int MODE, int NQ>
 cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
-  constexpr int NG = 2;  // consumer groups (the host layout reserves one workspace per group)
+  constexpr int NG = kGroups;  // consumer groups (the host layout reserves one workspace per group)
   auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ, NG>;
   // the dynamic shared-memory opt-in is per function and device; remember the largest set
   static int configured[kMaxDevices] = {0};

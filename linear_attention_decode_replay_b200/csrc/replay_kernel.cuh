@@ -119,25 +119,166 @@ struct Records {
 };
 
 // ---------------------------------------------------------------------------- producer
-// One unit's copies into stage `st`, one bulk copy (TMA) per lane, counted in bytes on
-// `bar`: lane 0 the state tile, lane 1 the FP8 row scales, lanes 2-3 the live ring
-// records [start, start + count) modulo cap, lane 4 the queries. The eager baseline has
-// no ring: its new token's k, v, Delta, a (and q) are gathered with per-lane cp.async.
+// Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile, 1 the FP8 row
+// scales, 2-3 the live ring records [start, start + count) modulo cap, 4 the queries.
+// Returns the bytes of copy `kind` (0 if none) and its addresses.
+constexpr int kCopyKinds = 5;
 template <int MODE, int CKPT, int S_IO>
-__device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& pl, uint8_t* st, uint64_t* bar,
-                                                  int lane, uint64_t stream_policy, uint64_t keep_policy) {
+__device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, uint8_t* st, int kind,
+                                              const uint8_t*& src, uint8_t*& dst) {
   const size_t P = p.P, N = p.N;
   const size_t bh = (size_t)pl.b * p.H + pl.h;
-  if (!pl.active) return;
-  uint8_t* recbuf = st + p.off_rec;
-  if (MODE == kModeEager) {
+  const int R = p.rec_bytes;
+  const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
+  const int first = min(cnt, p.cap - pl.start);
+  const uint8_t* ring = static_cast<const uint8_t*>(p.ring) + bh * p.cap * R;
+  const size_t bg = (size_t)pl.b * p.G + pl.g;
+  const uint8_t* qsrc = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
+                                : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
+  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + bh * P * N) : p.S8 + bh * P * N;
+  src = (kind == 0)   ? tsrc
+        : (kind == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + bh * P)
+        : (kind == 2) ? ring + (size_t)pl.start * R
+        : (kind == 3) ? ring
+                      : qsrc;
+  dst = (kind == 0)   ? st
+        : (kind == 1) ? st + P * N
+        : (kind == 2) ? st + p.off_rec
+        : (kind == 3) ? st + p.off_rec + (size_t)first * R
+                      : st + p.off_q;
+  uint32_t bytes = 0;
+  bytes = (kind == 0) ? (pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N)) : bytes;
+  bytes = (kind == 1 && !pl.fp32_tile) ? (uint32_t)(P * 4) : bytes;
+  bytes = (kind == 2) ? (uint32_t)(first * R) : bytes;
+  bytes = (kind == 3) ? (uint32_t)((cnt - first) * R) : bytes;
+  bytes = (kind == 4 && MODE == kModeReplay) ? (uint32_t)(p.n_pos * N * S_IO) : bytes;
+  return pl.active ? bytes : 0u;
+}
+
+// The producer warp fills the CTA's units in order, kUnitsPerIssue at a time: it waits
+// until their stages are free, arms each stage's "full" barrier with the unit's byte
+// count, and then one predicated bulk-copy instruction issues every copy of the batch
+// (lane = unit in batch * kCopyKinds + kind). Issuing costs the warp about as much for
+// one copy as for a whole batch, so batching is what keeps the stream fed.
+template <int MODE, int CKPT, int S_IO>
+__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
+  constexpr int U = kUnitsPerIssue;
+  static_assert(U * kCopyKinds <= 32 && (32 % U) == 0, "a batch's copies must fit one warp and tile 32 units");
+  const int lane = threadIdx.x & 31;
+  const int NS = p.num_stages;
+  const uint64_t stream_policy = l2_evict_first_policy();
+  const uint64_t keep_policy = l2_evict_normal_policy();
+  const int total = (p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  auto unit_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
+  // pointer words (and flush masks) 32 units at a time, one chunk ahead: lane j of a
+  // chunk holds the word of the chunk's j-th unit
+  auto load_words = [&](int i0, int32_t& w, int& msk) {
+    w = 0;
+    msk = 1;
+    const int uu = unit_of(i0 + lane);
+    if (uu < p.num_units) {
+      const int b = uu / p.H;
+      w = __ldg(p.counts_in + b);
+      if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
+    }
+  };
+  int32_t w_cur, w_nxt;
+  int m_cur, m_nxt;
+  load_words(0, w_cur, m_cur);
+  load_words(32, w_nxt, m_nxt);
+  const int j = lane / kCopyKinds;     // this lane's unit within the batch
+  const int kind = lane % kCopyKinds;  // and its copy
+  for (int i0 = 0; i0 < total; i0 += U) {
+    if ((i0 & 31) == 0 && i0 > 0) {
+      w_cur = w_nxt;
+      m_cur = m_nxt;
+      load_words(i0 + 32, w_nxt, m_nxt);
+    }
+    // every lane waits for the batch's stages (each lane then writes into one), the
+    // warp agrees
+    bool ready = true;
+#pragma unroll
+    for (int jj = 0; jj < U; ++jj) {
+      const int i = i0 + jj;
+      if (i < total && i >= NS) ready = ready && mbar_wait_bounded(&bars->empty[i % NS], ((i / NS) - 1) & 1);
+    }
+    if (!__all_sync(0xffffffffu, ready)) {
+      if (lane == 0) {
+        report_error(p.status, kErrWaitTimeout);
+        bars->abort_flag = 1;
+      }
+      break;
+    }
+    const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
+    if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
+    const int i = i0 + j;
+    const bool valid = j < U && i < total;
+    const int32_t word = __shfl_sync(0xffffffffu, w_cur, i & 31);
+    const int msk = __shfl_sync(0xffffffffu, m_cur, i & 31);
+    const int s = i % NS;
+    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint64_t* bar = &bars->full[s];
+    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), word, msk);
+    if (valid && kind == 0) {
+      reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
+      reinterpret_cast<int32_t*>(st + p.off_meta)[1] = msk;
+      if (pl.corrupt) report_error(p.status, kErrPointer);
+      mbar_arrive_expect_tx(bar, pl.bytes);
+    }
+    __syncwarp();
+    const uint8_t* src;
+    uint8_t* dst;
+    uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, st, kind, src, dst);
+    if (!valid) bytes = 0;
+    __syncwarp();
+    if (bytes) bulk_g2s_hint(dst, src, bytes, bar, kind == 0 ? stream_policy : keep_policy);
+    if (valid && kind == 0) bars->last_fill[s] = i;
+  }
+  // Never leave with copies in flight into this CTA's shared memory: wait (bounded) for
+  // the latest fill of every stage.
+  __syncwarp();
+  for (int st_i = 0; st_i < NS; ++st_i) {
+    const int i = bars->last_fill[st_i];
+    if (i >= 0 && !mbar_wait_bounded(&bars->full[st_i], (i / NS) & 1) && lane == 0)
+      report_error(p.status, kErrWaitTimeout);
+  }
+}
+
+// The eager baseline's producer: one unit at a time; the tile (and FP8 scales) by bulk
+// copy, the new token's k, v, Delta, a and q gathered with per-lane cp.async.
+template <int CKPT, int S_IO>
+__device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bars) {
+  const int lane = threadIdx.x & 31;
+  const int NS = p.num_stages;
+  const uint64_t stream_policy = l2_evict_first_policy();
+  const size_t P = p.P, N = p.N;
+  int i = 0;
+  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++i) {
+    const int s = i % NS;
+    const int k = i / NS;
+    if (k > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1))) {
+      if (lane == 0) {
+        report_error(p.status, kErrWaitTimeout);
+        bars->abort_flag = 1;
+      }
+      break;
+    }
+    const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
+    if (__shfl_sync(0xffffffffu, ab, 0)) break;
+    const Plan pl = make_plan<kModeEager, CKPT, S_IO>(p, u, 0, 1);
+    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint64_t* bar = &bars->full[s];
+    const size_t bh = (size_t)pl.b * p.H + pl.h;
+    const size_t bg = (size_t)pl.b * p.G + pl.g;
+    uint8_t* recbuf = st + p.off_rec;
+    if (lane == 0) mbar_arrive_expect_tx(bar, pl.bytes);
+    __syncwarp();
     if (lane == 0)
       bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + bh * P * N) : (const void*)(p.S8 + bh * P * N),
                     pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N), bar, stream_policy);
     if (lane == 1 && !pl.fp32_tile) bulk_g2s(st + P * N, p.Sscale + bh * P, (uint32_t)(P * 4), bar);
     const int kpe = (int)(N * S_IO / 16);
     const int vpe = (int)(P * S_IO / 16);
-    const size_t bg = (size_t)pl.b * p.G + pl.g;
     for (int idx = lane; idx < 2 * kpe + vpe; idx += 32) {
       if (idx < kpe) {
         cp_async16(st + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
@@ -151,157 +292,122 @@ __device__ __forceinline__ void issue_unit_copies(const KParams& p, const Plan& 
     }
     if (lane == 0) cp_async4(recbuf + (N + P) * S_IO, p.dt + bh);
     if (lane == 1) cp_async4(recbuf + (N + P) * S_IO + 4, p.a + bh);
-    return;
-  }
-  // every lane works out its copy without branching, then one predicated instruction
-  // issues all of them
-  const int R = p.rec_bytes;
-  const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
-  const int first = min(cnt, p.cap - pl.start);
-  const uint8_t* ring = static_cast<const uint8_t*>(p.ring) + bh * p.cap * R;
-  const size_t bg = (size_t)pl.b * p.G + pl.g;
-  const uint8_t* qsrc = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
-                                : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
-  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + bh * P * N) : p.S8 + bh * P * N;
-  const uint8_t* src = (lane == 0)   ? tsrc
-                       : (lane == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + bh * P)
-                       : (lane == 2) ? ring + (size_t)pl.start * R
-                       : (lane == 3) ? ring
-                                     : qsrc;
-  uint8_t* dst = (lane == 0)   ? st
-                 : (lane == 1) ? st + P * N
-                 : (lane == 2) ? recbuf
-                 : (lane == 3) ? recbuf + (size_t)first * R
-                               : st + p.off_q;
-  uint32_t bytes = 0;
-  bytes = (lane == 0) ? (pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N)) : bytes;
-  bytes = (lane == 1 && !pl.fp32_tile) ? (uint32_t)(P * 4) : bytes;
-  bytes = (lane == 2) ? (uint32_t)(first * R) : bytes;
-  bytes = (lane == 3) ? (uint32_t)((cnt - first) * R) : bytes;
-  bytes = (lane == 4 && MODE == kModeReplay) ? (uint32_t)(p.n_pos * N * S_IO) : bytes;
-  __syncwarp();
-  if (bytes) bulk_g2s_hint(dst, src, bytes, bar, lane == 0 ? stream_policy : keep_policy);
-}
-
-template <int MODE, int CKPT, int S_IO>
-__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars, int pw) {
-  const int lane = threadIdx.x & 31;
-  const int NS = p.num_stages;
-  const uint64_t stream_policy = l2_evict_first_policy();
-  const uint64_t keep_policy = l2_evict_normal_policy();
-  // Producer warp pw fills the CTA's units i = pw, pw + kProducerWarps, ... Their pointer
-  // words (and flush masks) are prefetched 32 units at a time, one chunk ahead: lane j
-  // of a chunk holds the word of the chunk's j-th unit.
-  auto unit_of = [&](int m) { return blockIdx.x + (pw + kProducerWarps * m) * gridDim.x; };
-  auto load_words = [&](int m0, int32_t& w, int& msk) {
-    w = 0;
-    msk = 1;
-    const int uu = unit_of(m0 + lane);
-    if (MODE != kModeEager && uu < p.num_units) {
-      const int b = uu / p.H;
-      w = __ldg(p.counts_in + b);
-      if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
-    }
-  };
-  int32_t w_cur, w_nxt;
-  int m_cur, m_nxt;
-  load_words(0, w_cur, m_cur);
-  load_words(32, w_nxt, m_nxt);
-  int m = 0;
-  for (int u = unit_of(0); u < p.num_units; ++m, u = unit_of(m)) {
-    const int i = pw + kProducerWarps * m;  // the CTA-local unit index
-    const int s = i % NS;
-    const int k = i / NS;
-    if ((m & 31) == 0 && m > 0) {
-      w_cur = w_nxt;
-      m_cur = m_nxt;
-      load_words(m + 32, w_nxt, m_nxt);
-    }
-    if (k > 0) {
-      // every lane waits (each lane then writes into the stage), the warp agrees
-      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1));
-      if (!ok) {
-        if (lane == 0) {
-          report_error(p.status, kErrWaitTimeout);
-          bars->abort_flag = 1;
-        }
-        break;
-      }
-    }
-    int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
-    if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
-    const int32_t word = __shfl_sync(0xffffffffu, w_cur, m & 31);
-    const int msk = __shfl_sync(0xffffffffu, m_cur, m & 31);
-    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u, word, msk);
-    uint8_t* st = stages + (size_t)s * p.stage_bytes;
-    if (lane == 0) {
-      reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
-      reinterpret_cast<int32_t*>(st + p.off_meta)[1] = msk;
-      if (pl.corrupt) report_error(p.status, kErrPointer);
-      mbar_arrive_expect_tx(&bars->full[s], pl.bytes);
-    }
-    __syncwarp();
-    issue_unit_copies<MODE, CKPT, S_IO>(p, pl, st, &bars->full[s], lane, stream_policy, keep_policy);
-    cp_async_arrive(&bars->full[s]);
+    cp_async_arrive(bar);
     if (lane == 0) bars->last_fill[s] = i;
   }
-  // Never leave with copies in flight into this CTA's shared memory. A fill that was
-  // followed by a later fill of the same stage has been consumed; so once both producer
-  // warps are done, each waits (bounded) for the latest fill of every stage that it made.
-  asm volatile("bar.sync %0, %1;" ::"r"(kProducerBarrier), "r"(kProducerWarps * 32) : "memory");
+  __syncwarp();
   for (int st_i = 0; st_i < NS; ++st_i) {
-    const int i = bars->last_fill[st_i];
-    if (i >= 0 && i % kProducerWarps == pw) {
-      if (!mbar_wait_bounded(&bars->full[st_i], (i / NS) & 1) && lane == 0) report_error(p.status, kErrWaitTimeout);
-    }
+    const int i2 = bars->last_fill[st_i];
+    if (i2 >= 0 && !mbar_wait_bounded(&bars->full[st_i], (i2 / NS) & 1) && lane == 0)
+      report_error(p.status, kErrWaitTimeout);
   }
 }
 
 // ---------------------------------------------------------------------------- consumers
-// kq[s][jj] = k_{o0+jj} . q_s for every query s < n and entry jj < width (<= 32).
-template <int N, typename IO, int GW>
-__device__ __forceinline__ void entry_dots(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int o0,
-                                           int width, int n, float* kq, int gw, int lane) {
-  constexpr int S_IO = IoT<IO>::bytes;
-  if constexpr (N == 128) {
-    // a warp per (query, 8 entries): the lanes split N, a transposing reduction sums them
-    const int chunks = (width + 7) / 8;
-    for (int t = gw; t < n * chunks; t += GW) {
-      const int s = t / chunks;
-      const int ch = t - s * chunks;
-      const float4 qv = IoT<IO>::load4(qbuf + ((size_t)s * N + lane * 4) * S_IO);
-      float part[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int jj = ch * 8 + r;
-        part[r] = (jj < width) ? dot4(IoT<IO>::load4(rec.k(o0 + jj) + lane * 4 * S_IO), qv) : 0.f;
-      }
-      int base;
-      const bool wr = SegReduce<8, 32>::run(part, lane, base);
-      const int jj = ch * 8 + base;
-      if (wr && jj < width) kq[s * kMaxWindow + jj] = part[0];
+// The coefficient warp's share of a unit (all 32 lanes; ws is its group's workspace):
+//  * fold weights of the c buffered entries when the unit folds (blog "Ruta 'estado y
+//    salida'"): sig_j = Delta_j prod_{j<i<c} a_i and abar = prod_{i<c} a_i (the eager
+//    baseline: its single entry, sig_0 = Delta, abar = a);
+//  * for every position s the outputs replay the entries o0 .. c+s, o0 = c after a fold
+//    and 0 otherwise (blog "Ruta 'solo salida'"):
+//        alpha_s = prod_{o0<=i<=c+s} a_i,   w_{s,j} = Delta_j prod_{j<i<=c+s} a_i,
+//        u_s[p]  = sum_{o0<=j<=c+s} w_{s,j} (k_j . q_s) v_j[p],
+//    so that y_s = alpha_s (S q_s) + u_s. The products of decay factors are suffix
+//    products over the window, one lane per entry.
+template <int N, typename IO, int MODE>
+__device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& rec, int c, float* sig, int lane) {
+  if (MODE == kModeEager) {
+    if (lane == 0) {
+      sig[0] = rec.dt(0);
+      sig[kMaxWindow] = rec.a(0);
     }
-  } else {
-    // short rows: a lane per (query, entry)
-    for (int t = gw * 32 + lane; t < n * width; t += GW * 32) {
-      const int s = t / width;
-      const int jj = t - s * width;
-      const uint8_t* kr = rec.k(o0 + jj);
-      const uint8_t* qr = qbuf + (size_t)s * N * S_IO;
-      float d = 0.f;
+    return;
+  }
+  float xa = 1.f, xd = 0.f;
+  if (lane < c) {
+    xa = rec.a(lane);
+    xd = rec.dt(lane);
+  }
+  const float incl = warp_suffix_prod(xa, lane);  // prod_{lane <= i < c} a_i
+  float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+  if (lane == 31) excl = 1.f;
+  if (lane < c) sig[lane] = xd * excl;
+  if (lane == 0) sig[kMaxWindow] = incl;
+}
+
+// The coefficient warp keeps its dependent chains short: lane l holds entry o0 + l, so
+// k_l . q_s is a private dot product (no cross-lane reduction), and u takes one
+// broadcast of each entry's coefficient.
+template <int N, typename IO>
+__device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
+                                             int n, int o0, int P, float* alpha, float* u, int lane) {
+  constexpr int S_IO = IoT<IO>::bytes;
+  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
+  const int width = c + n - o0;   // window entries (at most L): lane l holds entry o0 + l
+  const bool mine = lane < width;
+  float xa = 1.f, xd = 0.f;
+  if (mine) {
+    xa = rec.a(o0 + lane);
+    xd = rec.dt(o0 + lane);
+  }
+  const uint8_t* kr = rec.k(o0 + (mine ? lane : 0));
+  for (int s = 0; s < n; ++s) {
+    const int last = c + s - o0;  // position s replays window entries 0 .. last
+    const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
+    float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+    if (lane == 31) excl = 1.f;
+    if (lane == 0) alpha[s] = incl;
+    // k_l . q_s
+    const uint8_t* qs = qbuf + (size_t)s * N * S_IO;
+    float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-      for (int c4 = 0; c4 < N; c4 += 4) d += dot4(IoT<IO>::load4(kr + (size_t)c4 * S_IO), IoT<IO>::load4(qr + (size_t)c4 * S_IO));
-      kq[s * kMaxWindow + jj] = d;
+    for (int e = 0; e < N; e += 2 * EPV) {
+      d0 += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qs + (size_t)e * S_IO));
+      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 4) * S_IO));
+      if (EPV == 8) {
+        d0 += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 8) * S_IO));
+        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 12) * S_IO));
+      }
+    }
+    const float coef = (lane <= last) ? xd * excl * (d0 + d1) : 0.f;  // w_{s,l} (k_l . q_s)
+    // u_s[p] = sum_l coef_l v_l[p], two adjacent p per lane; coef_l comes from lane l
+    // (every lane runs every pass: the shuffles need the whole warp)
+    for (int pb = 0; pb < P; pb += 64) {
+      const int p2 = pb + lane * 2;
+      const bool act = p2 < P;
+      float u0 = 0.f, u1 = 0.f;
+      for (int l0 = 0; l0 <= last; l0 += 8) {
+        float2 vv[8];
+        float cl[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          cl[r] = __shfl_sync(0xffffffffu, coef, (l0 + r) & 31);
+          vv[r] = (act && l0 + r <= last) ? IoT<IO>::load2(rec.v(o0 + l0 + r) + (size_t)p2 * S_IO)
+                                          : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float cr = (l0 + r <= last) ? cl[r] : 0.f;
+          u0 = fmaf(cr, vv[r].x, u0);
+          u1 = fmaf(cr, vv[r].y, u1);
+        }
+      }
+      if (act) *reinterpret_cast<float2*>(u + (size_t)s * P + p2) = make_float2(u0, u1);
     }
   }
 }
 
+// One unit, by one consumer group: kGroupGemvWarps warps stream the state rows (dot
+// products, or the fold and its write-back) while the group's coefficient warp works out
+// the decay weights and the buffer terms from the records; the two meet at the group
+// barrier before the outputs are written.
 template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
 __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, uint8_t* st, uint8_t* ws, int gtid,
-                                             int bar_id) {
+                                             int bar_id, int gemv_bar_id) {
   using Gr = Groups<NG>;
-  constexpr int GT = Gr::kThreads;
-  constexpr int GW = Gr::kWarps;
+  constexpr int GT = Gr::kThreads;    // the whole group (barriers)
+  constexpr int GW = kGroupGemvWarps;  // warps on the state rows
+  constexpr int GTG = GW * 32;
   constexpr int TPR = N / 4;
   constexpr int RPW = 32 / TPR;  // rows per warp pass
   constexpr int RPG = GW * RPW;  // rows per group pass
@@ -312,225 +418,177 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   using Red = SegReduce<RT, TPR>;
   const int lane = gtid & 31;
   const int gw = gtid >> 5;
+  const bool coef_warp = gw == GW;
   const int row0 = gw * RPW + lane / TPR;
   const int col = (lane % TPR) * 4;
   const int P = p.P;
   const int c = pl.c;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
-  const int o0 = pl.fold ? c : 0;                                // first entry the outputs read
-  const int width = c + n - o0;                                  // entries the outputs read
+  const int o0 = pl.fold ? c : 0;                                // first entry the outputs replay
   const int fp = p.fp;
   const uint8_t* tile = st;
   const uint8_t* qbuf = st + p.off_q;
   const Records<N, S_IO> rec{st + p.off_rec, P, p.rec_bytes};
   const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
-  float* wout = reinterpret_cast<float*>(ws + p.ws_w);     // [kMaxPos][kMaxWindow] decay weight of entry o0+jj
-  float* kq = reinterpret_cast<float*>(ws + p.ws_kq);      // [kMaxPos][kMaxWindow] k_{o0+jj} . q_s
-  float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);
-  float* sig = reinterpret_cast<float*>(ws + p.ws_sig);    // fold weights; [kMaxWindow] = abar
-  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);      // [P][fp] fold weight times v_j[p]
+  float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);  // [kMaxPos]
+  float* sig = reinterpret_cast<float*>(ws + p.ws_sig);      // fold weights; [kMaxWindow] = abar
+  float* ublk = reinterpret_cast<float*>(ws + p.ws_u);       // [n][P] buffer terms of the outputs
+  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [P][fp] fold weight times v_j[p]
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   const int ngroups = (P + RGR - 1) / RGR;
+  const bool fold = pl.fold;
 
-  float4 qr[NQR];
+  if (coef_warp) {
+    // ---- the coefficient warp: fold weights first (the fold waits for them), then the
+    // outputs' buffer terms while the fold runs
+    if (fold) {
+      fold_weights<N, IO, MODE>(rec, c, sig, lane);
+      group_sync(bar_id, GT);
+    }
+    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, P, alpha, ublk, lane);
+    group_sync(bar_id, GT);
+  } else {
+    float4 qr[NQR];
 #pragma unroll
-  for (int s = 0; s < NQ; ++s)
-    qr[s] = (s < n) ? IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < NQ; ++s)
+      qr[s] = (s < n) ? IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
 
-  // state rows of one row group (the read copy keeps its row scale for the dot product)
-  auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
+    // state rows of one row group (the read copy keeps its row scale for the dot product)
+    auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      const int pr = gi * RGR + row0 + RPG * r;
-      x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (pr < P) {
-        if (pl.fp32_tile) {
-          x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
-        } else {
-          const float4 e = e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
-          if (dequant) {  // eager on a shared FP8 state: dequantise
-            const float sc = scale_tile[pr];
-            x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
+      for (int r = 0; r < RT; ++r) {
+        const int pr = gi * RGR + row0 + RPG * r;
+        x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (pr < P) {
+          if (pl.fp32_tile) {
+            x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
           } else {
-            x[r] = e;
+            const float4 e = e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
+            if (dequant) {  // eager on a shared FP8 state: dequantise
+              const float sc = scale_tile[pr];
+              x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
+            } else {
+              x[r] = e;
+            }
           }
         }
       }
-    }
-  };
-  float4 x[RT];
-  load_rows(x, 0, MODE == kModeEager);
-
-  // output-only units with a single row group: the row dot products and their reduction
-  // need nothing from the scans, so they run first; the sums wait in registers
-  const bool early = !pl.fold && ngroups == 1;
-  float dv[NQR][Red::kHeld];
-  int dbase = 0;
-  bool dwr = false;
-  if (early) {
-#pragma unroll
-    for (int s = 0; s < NQ; ++s) {
-      if (s < n) {
-        float part[RT];
-#pragma unroll
-        for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
-        dwr = Red::run(part, lane, dbase);
-#pragma unroll
-        for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
-      }
-    }
-  }
-
-  // ---- phase A: decay scans (a warp per task, on the group's last warps) and k_j . q_s
-  {
-    const int tasks = ((MODE == kModeReplay) ? n : 0) + (cf > 0 ? 1 : 0);
-    for (int t = GW - 1 - gw; t < tasks; t += GW) {
-      const bool fold_task = !(MODE == kModeReplay && t < n);
-      const int last = fold_task ? cf - 1 : c + t - o0;  // last lane of the scanned window
-      const int e0 = fold_task ? 0 : o0;
-      float xa = 1.f, xd = 0.f;
-      if (lane <= last) {
-        xa = rec.a(e0 + lane);
-        xd = rec.dt(e0 + lane);
-      }
-      const float incl = warp_suffix_prod(xa, lane);  // prod_{lane <= i <= last} a_i
-      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
-      if (lane == 31) excl = 1.f;
-      if (fold_task) {
-        if (lane <= last) sig[lane] = xd * excl;
-        if (lane == 0) sig[kMaxWindow] = incl;
-      } else {
-        if (lane <= last) wout[t * kMaxWindow + lane] = xd * excl;
-        if (lane == 0) alpha[t] = incl;
-      }
-    }
-    if (MODE == kModeReplay) entry_dots<N, IO, GW>(rec, qbuf, o0, width, n, kq, gw, lane);
-  }
-  group_sync(bar_id, GT);
-
-  // y = alpha_s d + sum_{jj} w_{s,jj} kq_{s,jj} v_{o0+jj}[p], by the lanes that hold row p's d
-  auto emit = [&](float d, int s, int pr) {
-    if (MODE == kModeReplay) {
-      const int last = c + s - o0;
-      float b0 = 0.f, b1 = 0.f;
-      int jj = 0;
-      for (; jj + 1 <= last; jj += 2) {
-        b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj], IoT<IO>::load1(rec.v(o0 + jj) + pr * S_IO), b0);
-        b1 = fmaf(wout[s * kMaxWindow + jj + 1] * kq[s * kMaxWindow + jj + 1],
-                  IoT<IO>::load1(rec.v(o0 + jj + 1) + pr * S_IO), b1);
-      }
-      if (jj <= last)
-        b0 = fmaf(wout[s * kMaxWindow + jj] * kq[s * kMaxWindow + jj], IoT<IO>::load1(rec.v(o0 + jj) + pr * S_IO), b0);
-      p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
-    } else {
-      p.y[bh * P + pr] = d;
-    }
-  };
-  auto write_outputs = [&](float (&part)[RT], int s, int gi, bool from_tile_fp8) {
-    int base;
-    const bool wr = Red::run(part, lane, base);
-#pragma unroll
-    for (int i = 0; i < Red::kHeld; ++i) {
-      const int pr = gi * RGR + row0 + RPG * (base + i);
-      if (wr && pr < P) emit(from_tile_fp8 ? part[i] * scale_tile[pr] : part[i], s, pr);
-    }
-  };
-
-  if (early) {
-    // ---- phase B: combine the early row sums with the buffer term
-#pragma unroll
-    for (int s = 0; s < NQ; ++s) {
-      if (s < n) {
-#pragma unroll
-        for (int i = 0; i < Red::kHeld; ++i) {
-          const int pr = row0 + RPG * (dbase + i);
-          if (dwr && pr < P) emit(pl.fp32_tile ? dv[s][i] : dv[s][i] * scale_tile[pr], s, pr);
-        }
-      }
-    }
-  } else if (!pl.fold) {
-    // ---- phase B: output-only route, several row groups
-    for (int gi = 0; gi < ngroups; ++gi) {
-      if (gi > 0) load_rows(x, gi, false);
+    };
+    // the row dot products of one row group, reduced: lane holds rows base .. base+kHeld
+    float dv[NQR][Red::kHeld];
+    int dbase = 0;
+    bool dwr = false;
+    auto row_dots = [&](const float4 (&x)[RT]) {
 #pragma unroll
       for (int s = 0; s < NQ; ++s) {
         if (s < n) {
           float part[RT];
 #pragma unroll
           for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
-          write_outputs(part, s, gi, !pl.fp32_tile);
+          dwr = Red::run(part, lane, dbase);
+#pragma unroll
+          for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
         }
       }
-    }
-  } else {
-    // ---- phase B: fold (state route), write the state back, outputs from the fresh rows
-    const int cf_pad = (cf + kFoldChunk - 1) / kFoldChunk * kFoldChunk;
-    for (int idx = gtid; idx < P * cf_pad; idx += GT) {
-      const int pp = idx / cf_pad;
-      const int j = idx - pp * cf_pad;
-      wt[pp * fp + j] = j < cf ? sig[j] * IoT<IO>::load1(rec.v(j) + pp * S_IO) : 0.f;
-    }
-    group_sync(bar_id, GT);
-    const float abar = sig[kMaxWindow];
-    for (int gi = 0; gi < ngroups; ++gi) {
-      if (gi > 0) load_rows(x, gi, MODE == kModeEager);
+    };
+    // y_s[p] = alpha_s d + u_s[p] (replay) or y[p] = d (eager)
+    auto emit = [&](int gi, bool from_tile_fp8) {
+      if (MODE == kModeFlush) return;
 #pragma unroll
-      for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
-      for (int ch = 0; ch < cf_pad; ch += kFoldChunk) {
-        float4 kr[kFoldChunk];
+      for (int s = 0; s < NQ; ++s) {
+        if (s < n) {
 #pragma unroll
-        for (int jj = 0; jj < kFoldChunk; ++jj) {
-          const int j = ch + jj;
-          kr[jj] = (j < cf) ? IoT<IO>::load4(rec.k(j) + col * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          const int pr = gi * RGR + row0 + RPG * r;
-          if (pr < P) {
-            const float* wrow = wt + (size_t)pr * fp + ch;
-#pragma unroll
-            for (int jj = 0; jj < kFoldChunk; jj += 4) {
-              const float4 w4 = *reinterpret_cast<const float4*>(wrow + jj);
-              const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                x[r].x = fmaf(wv[t], kr[jj + t].x, x[r].x);
-                x[r].y = fmaf(wv[t], kr[jj + t].y, x[r].y);
-                x[r].z = fmaf(wv[t], kr[jj + t].z, x[r].z);
-                x[r].w = fmaf(wv[t], kr[jj + t].w, x[r].w);
-              }
+          for (int i = 0; i < Red::kHeld; ++i) {
+            const int pr = gi * RGR + row0 + RPG * (dbase + i);
+            if (dwr && pr < P) {
+              const float d = from_tile_fp8 ? dv[s][i] * scale_tile[pr] : dv[s][i];
+              if (MODE == kModeReplay)
+                p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, ublk[(size_t)s * P + pr]);
+              else
+                p.y[bh * P + pr] = d;
             }
           }
         }
       }
-      // write the state: FP32 master, and/or the FP8 codes with per-row scales
-      const bool store_f32 = (MODE != kModeEager) || (CKPT == kCkptF32);
-      const bool store_fp8 = (CKPT == kCkptFp8);
-#pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const int pr = gi * RGR + row0 + RPG * r;
-        if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col), x[r]);
-        if (store_fp8) {
-          const float am = seg_allmax<TPR>(amax4(x[r]));
-          float sc, inv;
-          e4m3_row_scale(am, sc, inv);
-          if (pr < P) {
-            __stcs(reinterpret_cast<unsigned int*>(p.S8 + (bh * P + pr) * N + col), quant4_e4m3(x[r], inv));
-            if ((lane % TPR) == 0) p.Sscale[bh * P + pr] = sc;
-          }
-        }
+    };
+
+    float4 x[RT];
+    if (!fold) {
+      // ---- output-only route: row group 0's dot products, then wait for the buffer
+      // terms; further row groups (P > one row group) follow with the terms in hand
+      load_rows(x, 0, false);
+      row_dots(x);
+      group_sync(bar_id, GT);
+      emit(0, !pl.fp32_tile);
+      for (int gi = 1; gi < ngroups; ++gi) {
+        load_rows(x, gi, false);
+        row_dots(x);
+        emit(gi, !pl.fp32_tile);
       }
-      if (MODE != kModeFlush) {
+    } else {
+      // ---- fold (state route), write the state back, outputs from the fresh rows
+      load_rows(x, 0, MODE == kModeEager);
+      group_sync(bar_id, GT);  // the fold weights are in
+      const int cf_pad = (cf + kFoldChunk - 1) / kFoldChunk * kFoldChunk;
+      for (int idx = gtid; idx < P * cf_pad; idx += GTG) {
+        const int pp = idx / cf_pad;
+        const int jj = idx - pp * cf_pad;
+        wt[pp * fp + jj] = jj < cf ? sig[jj] * IoT<IO>::load1(rec.v(jj) + pp * S_IO) : 0.f;
+      }
+      group_sync(gemv_bar_id, GTG);
+      const float abar = sig[kMaxWindow];
+      for (int gi = 0; gi < ngroups; ++gi) {
+        if (gi > 0) load_rows(x, gi, MODE == kModeEager);
 #pragma unroll
-        for (int s = 0; s < NQ; ++s) {
-          if (s < n) {
-            float part[RT];
+        for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
+        for (int ch = 0; ch < cf_pad; ch += kFoldChunk) {
+          float4 kr[kFoldChunk];
 #pragma unroll
-            for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
-            write_outputs(part, s, gi, false);
+          for (int jj = 0; jj < kFoldChunk; ++jj) {
+            const int jx = ch + jj;
+            kr[jj] = (jx < cf) ? IoT<IO>::load4(rec.k(jx) + col * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const int pr = gi * RGR + row0 + RPG * r;
+            if (pr < P) {
+              const float* wrow = wt + (size_t)pr * fp + ch;
+#pragma unroll
+              for (int jj = 0; jj < kFoldChunk; jj += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wrow + jj);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  x[r].x = fmaf(wv[t], kr[jj + t].x, x[r].x);
+                  x[r].y = fmaf(wv[t], kr[jj + t].y, x[r].y);
+                  x[r].z = fmaf(wv[t], kr[jj + t].z, x[r].z);
+                  x[r].w = fmaf(wv[t], kr[jj + t].w, x[r].w);
+                }
+              }
+            }
           }
         }
+        // write the state: FP32 master, and/or the FP8 codes with per-row scales
+        const bool store_f32 = (MODE != kModeEager) || (CKPT == kCkptF32);
+        const bool store_fp8 = (CKPT == kCkptFp8);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const int pr = gi * RGR + row0 + RPG * r;
+          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col), x[r]);
+          if (store_fp8) {
+            const float am = seg_allmax<TPR>(amax4(x[r]));
+            float sc, inv;
+            e4m3_row_scale(am, sc, inv);
+            if (pr < P) {
+              __stcs(reinterpret_cast<unsigned int*>(p.S8 + (bh * P + pr) * N + col), quant4_e4m3(x[r], inv));
+              if ((lane % TPR) == 0) p.Sscale[bh * P + pr] = sc;
+            }
+          }
+        }
+        if (MODE != kModeFlush) row_dots(x);
+        if (gi == 0) group_sync(bar_id, GT);  // the outputs' buffer terms are in
+        emit(gi, false);
       }
     }
   }
@@ -540,12 +598,12 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const int cap = p.cap;
   if (MODE == kModeReplay) {
     if (pl.h == 0 && gtid == 0) {
-      int start2 = pl.fold ? start + c : start;
+      int start2 = fold ? start + c : start;
       start2 -= (start2 >= cap) ? cap : 0;
-      const int base = pl.fold ? 0 : c;
+      const int base = fold ? 0 : c;
       const int cnt2 = base + (p.commit ? n : 0);
       p.counts_out[pl.b] = (start2 << 16) | cnt2;
-      if (p.flushed) p.flushed[pl.b] = pl.fold ? 1 : 0;
+      if (p.flushed) p.flushed[pl.b] = fold ? 1 : 0;
     }
   } else if (MODE == kModeFlush) {
     if (pl.h == 0 && gtid == 0) {
@@ -569,7 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.num_stages; ++s) {
-      mbar_init(&bars->full[s], 1 + 32);  // the filling warp: lane 0's expect_tx + 32 lanes' cp.async
+      // the producer's expect_tx (the eager gather adds its 32 lanes' cp.async arrivals)
+      mbar_init(&bars->full[s], MODE == kModeEager ? 1 + 32 : 1);
       mbar_init(&bars->empty[s], Gr::kThreads);
     }
     bars->abort_flag = 0;
@@ -580,12 +639,16 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
 
   const int warp = threadIdx.x / 32;
   if (warp >= kConsumerWarps) {
-    producer_loop<MODE, CKPT, S_IO>(p, stages, bars, warp - kConsumerWarps);
+    if constexpr (MODE == kModeEager)
+      producer_loop_eager<CKPT, S_IO>(p, stages, bars);
+    else
+      producer_loop<MODE, CKPT, S_IO>(p, stages, bars);
     return;
   }
   const int g = warp / Gr::kWarps;  // consumer group
   const int gtid = threadIdx.x - g * Gr::kThreads;
-  const int bar_id = 1 + g;
+  const int bar_id = 1 + g;                 // the whole group
+  const int gemv_bar_id = 1 + NG + g;       // the group's row warps only
   uint8_t* ws = smem + p.ws_off + (size_t)g * p.ws_group_bytes;
   const int NS = p.num_stages;
   int i = g;
@@ -613,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u, word, msk);
     if (pl.active) {
-      consume_unit<N, IO, CKPT, MODE, NQ, NG>(p, pl, st, ws, gtid, bar_id);
+      consume_unit<N, IO, CKPT, MODE, NQ, NG>(p, pl, st, ws, gtid, bar_id, gemv_bar_id);
     } else if (pl.h == 0 && gtid == 0) {
       p.counts_out[pl.b] = word;  // nothing to fold: the pointer word carries over
       if (MODE == kModeFlush && p.flushed && !pl.corrupt) p.flushed[pl.b] = 0;

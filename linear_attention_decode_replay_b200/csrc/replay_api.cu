@@ -97,13 +97,13 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->stage_bytes = round_up(p->off_meta + 16, 128);
 
   // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
-  // abar, the buffer terms of the outputs u[nq_alloc][P], and the fold weights times v,
-  // [P][fp]
+  // abar, the outputs' entry coefficients [kMaxPos][kMaxWindow], and the fold weights
+  // times v, [P][fp]
   p->fp = round_up(lfold, replay::kFoldChunk);
   p->ws_alpha = 0;
   p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
-  p->ws_u = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
-  p->ws_wt = round_up(p->ws_u + nq_alloc * P * 4, 16);
+  p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
+  p->ws_wt = round_up(p->ws_cw + replay::kMaxPos * replay::kMaxWindow * 4, 16);
   p->ws_group_bytes = round_up(p->ws_wt + P * p->fp * 4, 128);
   p->ws_off = kHeaderBytes;
   p->stages_off = round_up(p->ws_off + kGroups * p->ws_group_bytes, 128);

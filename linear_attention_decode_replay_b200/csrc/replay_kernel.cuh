@@ -336,11 +336,12 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
 }
 
 // The coefficient warp keeps its dependent chains short: lane l holds entry o0 + l, so
-// k_l . q_s is a private dot product (no cross-lane reduction), and u takes one
-// broadcast of each entry's coefficient.
+// k_l . q_s is a private dot product (no cross-lane reduction). It leaves, per position
+// s, alpha_s and cw[s][l] = w_{s,l} (k_l . q_s); the row lanes then form
+// u_s[p] = sum_l cw[s][l] v_l[p] for the rows they hold.
 template <int N, typename IO>
 __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
-                                             int n, int o0, int P, float* alpha, float* u, int lane) {
+                                             int n, int o0, float* alpha, float* cw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
   constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
   const int width = c + n - o0;   // window entries (at most L): lane l holds entry o0 + l
@@ -369,31 +370,7 @@ __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& r
         d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 12) * S_IO));
       }
     }
-    const float coef = (lane <= last) ? xd * excl * (d0 + d1) : 0.f;  // w_{s,l} (k_l . q_s)
-    // u_s[p] = sum_l coef_l v_l[p], two adjacent p per lane; coef_l comes from lane l
-    // (every lane runs every pass: the shuffles need the whole warp)
-    for (int pb = 0; pb < P; pb += 64) {
-      const int p2 = pb + lane * 2;
-      const bool act = p2 < P;
-      float u0 = 0.f, u1 = 0.f;
-      for (int l0 = 0; l0 <= last; l0 += 8) {
-        float2 vv[8];
-        float cl[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          cl[r] = __shfl_sync(0xffffffffu, coef, (l0 + r) & 31);
-          vv[r] = (act && l0 + r <= last) ? IoT<IO>::load2(rec.v(o0 + l0 + r) + (size_t)p2 * S_IO)
-                                          : make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const float cr = (l0 + r <= last) ? cl[r] : 0.f;
-          u0 = fmaf(cr, vv[r].x, u0);
-          u1 = fmaf(cr, vv[r].y, u1);
-        }
-      }
-      if (act) *reinterpret_cast<float2*>(u + (size_t)s * P + p2) = make_float2(u0, u1);
-    }
+    if (lane <= last) cw[s * kMaxWindow + lane] = xd * excl * (d0 + d1);  // w_{s,l} (k_l . q_s)
   }
 }
 
@@ -433,7 +410,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
   float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);  // [kMaxPos]
   float* sig = reinterpret_cast<float*>(ws + p.ws_sig);      // fold weights; [kMaxWindow] = abar
-  float* ublk = reinterpret_cast<float*>(ws + p.ws_u);       // [n][P] buffer terms of the outputs
+  float* cw = reinterpret_cast<float*>(ws + p.ws_cw);        // [kMaxPos][kMaxWindow] entry coefficients
   float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [P][fp] fold weight times v_j[p]
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   const int ngroups = (P + RGR - 1) / RGR;
@@ -446,7 +423,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       fold_weights<N, IO, MODE>(rec, c, sig, lane);
       group_sync(bar_id, GT);
     }
-    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, P, alpha, ublk, lane);
+    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, alpha, cw, lane);
     group_sync(bar_id, GT);
   } else {
     float4 qr[NQR];
@@ -492,7 +469,8 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         }
       }
     };
-    // y_s[p] = alpha_s d + u_s[p] (replay) or y[p] = d (eager)
+    // y_s[p] = alpha_s d + sum_l cw[s][l] v_l[p] (replay) or y[p] = d (eager), by the
+    // lanes that hold row p's dot product; eight entries' v in flight at a time
     auto emit = [&](int gi, bool from_tile_fp8) {
       if (MODE == kModeFlush) return;
 #pragma unroll
@@ -503,10 +481,25 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
             const int pr = gi * RGR + row0 + RPG * (dbase + i);
             if (dwr && pr < P) {
               const float d = from_tile_fp8 ? dv[s][i] * scale_tile[pr] : dv[s][i];
-              if (MODE == kModeReplay)
-                p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, ublk[(size_t)s * P + pr]);
-              else
+              if (MODE == kModeReplay) {
+                const int last = c + s - o0;
+                const float* cws = cw + s * kMaxWindow;
+                float b0 = 0.f, b1 = 0.f;
+                for (int l0 = 0; l0 <= last; l0 += 8) {
+                  float vv[8];
+#pragma unroll
+                  for (int r = 0; r < 8; ++r)
+                    vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
+#pragma unroll
+                  for (int r = 0; r < 8; r += 2) {
+                    if (l0 + r <= last) b0 = fmaf(cws[l0 + r], vv[r], b0);
+                    if (l0 + r + 1 <= last) b1 = fmaf(cws[l0 + r + 1], vv[r + 1], b1);
+                  }
+                }
+                p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
+              } else {
                 p.y[bh * P + pr] = d;
+              }
             }
           }
         }

@@ -29,6 +29,7 @@ __global__ void rollback_kernel(const int32_t* __restrict__ counts_in, int32_t* 
 // the two never overlap (cap = L + max_pos). Verify queries are also gathered per group
 // into qpack so that a unit's queries are one contiguous piece. One warp per (b, h).
 __global__ void pack_entries_kernel(const PackParams pp) {
+  constexpr int kMaxChunks = 3;  // 16-byte chunks of one entry's k and v per lane: (N + P) * 4 / 16 / 32 <= 3
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x / 32;
   const int S = pp.io_bytes;
@@ -40,27 +41,37 @@ __global__ void pack_entries_kernel(const PackParams pp) {
     const int h = (int)(task - (long long)b * pp.H);
     const int g = h / pp.hpg;
     const int32_t word = pp.counts_in[b];
-    const int start = word >> 16;
-    const int c = word & 0xFFFF;
-    if (word < 0 || c > pp.L || start >= pp.cap) continue;  // the main kernel reports it
     for (int s = 0; s < pp.n_pos; ++s) {
-      int slot = start + c + s;
-      slot -= (slot >= pp.cap) ? pp.cap : 0;
-      uint8_t* rec = static_cast<uint8_t*>(pp.ring) + (((size_t)b * pp.H + h) * pp.cap + slot) * pp.rec_bytes;
+      // the entry's pieces are read before the pointer word is needed, so both reads
+      // are in flight together
       const size_t tok = (size_t)b * pp.n_pos + s;
       const uint8_t* kin = static_cast<const uint8_t*>(pp.k) + (tok * pp.G + g) * pp.N * S;
       const uint8_t* vin = static_cast<const uint8_t*>(pp.v) + (tok * pp.H + h) * pp.P * S;
-      for (int idx = lane; idx < kpe + vpe; idx += 32) {
-        if (idx < kpe) {
-          reinterpret_cast<uint4*>(rec)[idx] = reinterpret_cast<const uint4*>(kin)[idx];
-        } else {
-          reinterpret_cast<uint4*>(rec + pp.N * S)[idx - kpe] = reinterpret_cast<const uint4*>(vin)[idx - kpe];
-        }
+      uint4 chunk[kMaxChunks];
+#pragma unroll
+      for (int r = 0; r < kMaxChunks; ++r) {
+        const int idx = lane + 32 * r;
+        chunk[r] = idx < kpe         ? reinterpret_cast<const uint4*>(kin)[idx]
+                   : idx < kpe + vpe ? reinterpret_cast<const uint4*>(vin)[idx - kpe]
+                                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+      const float dts = (lane == 0) ? pp.dt[tok * pp.H + h] : 0.f;
+      const float as = (lane == 0) ? pp.a[tok * pp.H + h] : 0.f;
+      const int start = word >> 16;
+      const int c = word & 0xFFFF;
+      if (word < 0 || c > pp.L || start >= pp.cap) break;  // the main kernel reports it
+      int slot = start + c + s;
+      slot -= (slot >= pp.cap) ? pp.cap : 0;
+      uint8_t* rec = static_cast<uint8_t*>(pp.ring) + (((size_t)b * pp.H + h) * pp.cap + slot) * pp.rec_bytes;
+#pragma unroll
+      for (int r = 0; r < kMaxChunks; ++r) {
+        const int idx = lane + 32 * r;
+        if (idx < kpe + vpe) reinterpret_cast<uint4*>(rec)[idx] = chunk[r];  // k then v, back to back
       }
       if (lane == 0) {
         float* sc = reinterpret_cast<float*>(rec + (pp.N + pp.P) * S);
-        sc[0] = pp.dt[tok * pp.H + h];
-        sc[1] = pp.a[tok * pp.H + h];
+        sc[0] = dts;
+        sc[1] = as;
       }
       if (pp.qpack && (h % pp.hpg) == 0) {
         const uint8_t* qin = static_cast<const uint8_t*>(pp.q) + (tok * pp.G + g) * pp.N * S;

@@ -98,13 +98,13 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
 
   // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
   // abar, the outputs' entry coefficients [kMaxPos][kMaxWindow], and the fold weights
-  // times v, [P][fp]
-  p->fp = round_up(lfold, replay::kFoldChunk);
+  // times v, [lfold][wt_stride] (rows padded to a multiple of kRowsPerThread)
+  p->wt_stride = round_up(c.P, replay::kRowsPerThread);
   p->ws_alpha = 0;
   p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
   p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
   p->ws_wt = round_up(p->ws_cw + replay::kMaxPos * replay::kMaxWindow * 4, 16);
-  p->ws_group_bytes = round_up(p->ws_wt + P * p->fp * 4, 128);
+  p->ws_group_bytes = round_up(p->ws_wt + lfold * p->wt_stride * 4, 128);
   p->ws_off = kHeaderBytes;
   p->stages_off = round_up(p->ws_off + kGroups * p->ws_group_bytes, 128);
   const int avail = smem_optin - p->stages_off;

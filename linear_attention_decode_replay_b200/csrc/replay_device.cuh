@@ -20,7 +20,6 @@ constexpr int kMaxPos = 8;                       // query positions per verify c
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
 constexpr int kMaxStages = 8;
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
-constexpr int kFoldChunk = 8;                    // buffer entries folded per register pass
 constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 

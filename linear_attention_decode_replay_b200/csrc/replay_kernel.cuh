@@ -396,14 +396,16 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const int lane = gtid & 31;
   const int gw = gtid >> 5;
   const bool coef_warp = gw == GW;
-  const int row0 = gw * RPW + lane / TPR;
+  // this thread's rows of a row group: rbase .. rbase + RT - 1 (contiguous, so that a
+  // fold reads their weights as four 16-byte vectors)
+  const int rbase = (gw * RPW + lane / TPR) * RT;
   const int col = (lane % TPR) * 4;
   const int P = p.P;
   const int c = pl.c;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
   const int o0 = pl.fold ? c : 0;                                // first entry the outputs replay
-  const int fp = p.fp;
+  const int wts = p.wt_stride;  // row stride of the fold weight table, >= P, multiple of RT
   const uint8_t* tile = st;
   const uint8_t* qbuf = st + p.off_q;
   const Records<N, S_IO> rec{st + p.off_rec, P, p.rec_bytes};
@@ -411,7 +413,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);  // [kMaxPos]
   float* sig = reinterpret_cast<float*>(ws + p.ws_sig);      // fold weights; [kMaxWindow] = abar
   float* cw = reinterpret_cast<float*>(ws + p.ws_cw);        // [kMaxPos][kMaxWindow] entry coefficients
-  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [P][fp] fold weight times v_j[p]
+  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [c][wts] fold weight times v_j[p]
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   const int ngroups = (P + RGR - 1) / RGR;
   const bool fold = pl.fold;
@@ -435,7 +437,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        const int pr = gi * RGR + row0 + RPG * r;
+        const int pr = gi * RGR + rbase + r;
         x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (pr < P) {
           if (pl.fp32_tile) {
@@ -478,7 +480,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         if (s < n) {
 #pragma unroll
           for (int i = 0; i < Red::kHeld; ++i) {
-            const int pr = gi * RGR + row0 + RPG * (dbase + i);
+            const int pr = gi * RGR + rbase + dbase + i;
             if (dwr && pr < P) {
               const float d = from_tile_fp8 ? dv[s][i] * scale_tile[pr] : dv[s][i];
               if (MODE == kModeReplay) {
@@ -523,11 +525,16 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       // ---- fold (state route), write the state back, outputs from the fresh rows
       load_rows(x, 0, MODE == kModeEager);
       group_sync(bar_id, GT);  // the fold weights are in
-      const int cf_pad = (cf + kFoldChunk - 1) / kFoldChunk * kFoldChunk;
-      for (int idx = gtid; idx < P * cf_pad; idx += GTG) {
-        const int pp = idx / cf_pad;
-        const int jj = idx - pp * cf_pad;
-        wt[pp * fp + jj] = jj < cf ? sig[jj] * IoT<IO>::load1(rec.v(jj) + pp * S_IO) : 0.f;
+      // wt[j][p] = sig_j v_j[p] (zero for p >= P), a thread per (8 entries, row): every
+      // load independent, consecutive threads on consecutive rows
+      for (int job = gtid; job < wts * ((cf + 7) / 8); job += GTG) {
+        const int j8 = job / wts;
+        const int pp = job - j8 * wts;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int jj = j8 * 8 + r;
+          if (jj < cf) wt[(size_t)jj * wts + pp] = pp < P ? sig[jj] * IoT<IO>::load1(rec.v(jj) + pp * S_IO) : 0.f;
+        }
       }
       group_sync(gemv_bar_id, GTG);
       const float abar = sig[kMaxWindow];
@@ -535,30 +542,23 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         if (gi > 0) load_rows(x, gi, MODE == kModeEager);
 #pragma unroll
         for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
-        for (int ch = 0; ch < cf_pad; ch += kFoldChunk) {
-          float4 kr[kFoldChunk];
+        // rank-cf update: per entry, k_j's four columns of this lane and the weights of
+        // the thread's RT rows (four 16-byte broadcasts), then 4 * RT FMAs
+        const int wbase = (gi * RGR + rbase < P) ? gi * RGR + rbase : 0;  // all-invalid threads read row 0
+        for (int jj = 0; jj < cf; ++jj) {
+          const float4 kt = IoT<IO>::load4(rec.k(jj) + col * S_IO);
+          const float4* wv = reinterpret_cast<const float4*>(wt + (size_t)jj * wts + wbase);
 #pragma unroll
-          for (int jj = 0; jj < kFoldChunk; ++jj) {
-            const int jx = ch + jj;
-            kr[jj] = (jx < cf) ? IoT<IO>::load4(rec.k(jx) + col * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+          for (int r4 = 0; r4 < RT / 4; ++r4) {
+            const float4 w = wv[r4];
+            const float ws4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int r = 0; r < RT; ++r) {
-            const int pr = gi * RGR + row0 + RPG * r;
-            if (pr < P) {
-              const float* wrow = wt + (size_t)pr * fp + ch;
-#pragma unroll
-              for (int jj = 0; jj < kFoldChunk; jj += 4) {
-                const float4 w4 = *reinterpret_cast<const float4*>(wrow + jj);
-                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  x[r].x = fmaf(wv[t], kr[jj + t].x, x[r].x);
-                  x[r].y = fmaf(wv[t], kr[jj + t].y, x[r].y);
-                  x[r].z = fmaf(wv[t], kr[jj + t].z, x[r].z);
-                  x[r].w = fmaf(wv[t], kr[jj + t].w, x[r].w);
-                }
-              }
+            for (int t = 0; t < 4; ++t) {
+              float4& xr = x[r4 * 4 + t];
+              xr.x = fmaf(ws4[t], kt.x, xr.x);
+              xr.y = fmaf(ws4[t], kt.y, xr.y);
+              xr.z = fmaf(ws4[t], kt.z, xr.z);
+              xr.w = fmaf(ws4[t], kt.w, xr.w);
             }
           }
         }
@@ -567,7 +567,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         const bool store_fp8 = (CKPT == kCkptFp8);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-          const int pr = gi * RGR + row0 + RPG * r;
+          const int pr = gi * RGR + rbase + r;
           if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col), x[r]);
           if (store_fp8) {
             const float am = seg_allmax<TPR>(amax4(x[r]));

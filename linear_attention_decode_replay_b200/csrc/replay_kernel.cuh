@@ -530,10 +530,17 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       for (int job = gtid; job < wts * ((cf + 7) / 8); job += GTG) {
         const int j8 = job / wts;
         const int pp = job - j8 * wts;
+        const int pv = pp < P ? pp : 0;
+        float wv[8];  // all eight reads first: the table writes could alias them
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int jj = min(j8 * 8 + r, cf - 1);
+          wv[r] = sig[jj] * IoT<IO>::load1(rec.v(jj) + pv * S_IO);
+        }
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           const int jj = j8 * 8 + r;
-          if (jj < cf) wt[(size_t)jj * wts + pp] = pp < P ? sig[jj] * IoT<IO>::load1(rec.v(jj) + pp * S_IO) : 0.f;
+          if (jj < cf) wt[(size_t)jj * wts + pp] = pp < P ? wv[r] : 0.f;
         }
       }
       group_sync(gemv_bar_id, GTG);
@@ -545,13 +552,20 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         // rank-cf update: per entry, k_j's four columns of this lane and the weights of
         // the thread's RT rows (four 16-byte broadcasts), then 4 * RT FMAs
         const int wbase = (gi * RGR + rbase < P) ? gi * RGR + rbase : 0;  // all-invalid threads read row 0
+        // the next entry's k and weights are read while this entry's FMAs run
+        float4 kt = IoT<IO>::load4(rec.k(0) + col * S_IO);
+        float4 wcur[RT / 4];
+#pragma unroll
+        for (int r4 = 0; r4 < RT / 4; ++r4) wcur[r4] = reinterpret_cast<const float4*>(wt + wbase)[r4];
         for (int jj = 0; jj < cf; ++jj) {
-          const float4 kt = IoT<IO>::load4(rec.k(jj) + col * S_IO);
-          const float4* wv = reinterpret_cast<const float4*>(wt + (size_t)jj * wts + wbase);
+          const int jn = min(jj + 1, cf - 1);
+          const float4 kn = IoT<IO>::load4(rec.k(jn) + col * S_IO);
+          float4 wn[RT / 4];
+#pragma unroll
+          for (int r4 = 0; r4 < RT / 4; ++r4) wn[r4] = reinterpret_cast<const float4*>(wt + (size_t)jn * wts + wbase)[r4];
 #pragma unroll
           for (int r4 = 0; r4 < RT / 4; ++r4) {
-            const float4 w = wv[r4];
-            const float ws4[4] = {w.x, w.y, w.z, w.w};
+            const float ws4[4] = {wcur[r4].x, wcur[r4].y, wcur[r4].z, wcur[r4].w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
               float4& xr = x[r4 * 4 + t];
@@ -561,6 +575,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
               xr.w = fmaf(ws4[t], kt.w, xr.w);
             }
           }
+          kt = kn;
+#pragma unroll
+          for (int r4 = 0; r4 < RT / 4; ++r4) wcur[r4] = wn[r4];
         }
         // write the state: FP32 master, and/or the FP8 codes with per-row scales
         const bool store_f32 = (MODE != kModeEager) || (CKPT == kCkptF32);

@@ -34,13 +34,14 @@ from workloads import gen  # noqa: E402
 
 METRIC = "decode tokens/s per SSM layer at batch 256, L=16 (1 B200); achieved HBM GB/s vs peak"
 UNIT = "tokens/s"
+SPEC_METRIC = "speculative decode tokens/s per SSM layer at batch 256, L=16, draft 4 (1 B200); achieved HBM GB/s vs peak"
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
 # window) from an ncu capture, and the hash of the kernel sources it was taken on. When
 # the sources change the figure no longer applies and is reported as null.
-NCU_TRAFFIC = {"sources_sha256": "0924d48fa3d1c4dd151b29b5465544b5aa6eae047e3cf9d748a5f8f078d7646d",
-               "bytes_per_launch": 597.7e6}
+NCU_TRAFFIC = {"sources_sha256": "3dbe106e41a904adb78688b8dcbd6c002b8b4a7ccbeb582965619f1157ce6b4c",
+               "bytes_per_launch": 596.7e6}
 
 
 def kernel_sources_hash() -> str:
@@ -332,6 +333,131 @@ def run_ours(args, rank, world, local):
     return result
 
 
+# ------------------------------------------------------------------ our arm, speculative verify
+
+def verify_round_bytes(s: gen.Shape, counts: np.ndarray, n_pos: int) -> float:
+    """Algorithmic bytes of one verify round over the batch, given every sequence's
+    committed count before it: the state read (and written when the round folds), the
+    buffered and new entries read, the new entries written, the queries, the outputs."""
+    sio = s.io_bytes
+    E = s.G * s.N * sio + s.H * s.P * sio + 8 * s.H
+    state = s.H * s.P * s.N * 4
+    fold = counts + n_pos > s.L
+    per_seq = (state * (1 + fold) + (counts + n_pos) * E + n_pos * E + n_pos * s.G * s.N * sio
+               + n_pos * 4 * s.H * s.P)
+    return float(per_seq.sum())
+
+
+def run_spec_ours(args, rank, world, local):
+    """One bench step = R verify rounds of n_pos = max_pos positions over the batch, each
+    followed by the rollback that keeps 1 + accepted entries (accepted drawn per sequence
+    and round); tokens = sum of (1 + accepted)."""
+    import linear_attention_decode_replay_b200 as lar
+
+    shape = gen.SHAPES[args.workload]
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    n_pos = shape.max_pos
+    cfg = lar.Config(batch=shape.B, heads=shape.H, groups=shape.G, P=shape.P, N=shape.N, L=shape.L,
+                     max_pos=n_pos, io=shape.io, ckpt=shape.ckpt)
+    B, R = shape.B, shape.L
+    bufs = lar.alloc_buffers(cfg, device)
+    bufs["S0"].copy_(gen.initial_state(shape, device=device))
+    r = lar.Replay(cfg, bufs)
+    rounds = [gen.verify_inputs(shape, t, n_pos, device=device) for t in range(R)]
+    keeps = [(gen.accepted_lengths(shape, t, n_pos, device=device) + 1).to(torch.int32) for t in range(R)]
+    keeps_h = [k.cpu().numpy().astype(np.int64) for k in keeps]
+    y = torch.empty(B, n_pos, shape.H, shape.P, device=device)
+
+    def one_step():
+        for x, nk in zip(rounds, keeps):
+            r.verify(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+            r.rollback(nk)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    counts0 = np.array(r.read_counts(), dtype=np.int64)
+    barrier(world)
+
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start.record(stream)
+    for _ in range(K):
+        one_step()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), world, device)
+    status = r.check_status()
+    if status:
+        raise RuntimeError(f"device status bits {status} after the timed region")
+
+    # algorithmic bytes of the timed rounds, following the counts
+    counts = counts0.copy()
+    total_bytes = 0.0
+    for _ in range(K):
+        for nk in keeps_h:
+            total_bytes += verify_round_bytes(shape, counts, n_pos)
+            counts = np.where(counts + n_pos > shape.L, 0, counts) + nk
+    tokens_per_step = float(sum(k.sum() for k in keeps_h))
+    tokens = world * tokens_per_step * K
+    value = tokens / (elapsed_ms * 1e-3)
+    round_ms = elapsed_ms / (K * R)
+    achieved_gbs = total_bytes / (K * R) / (round_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+
+    # end to end: pinned host inputs of every round in, y back
+    host_rounds = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in rounds]
+    host_keeps = [k.cpu().pin_memory() for k in keeps]
+    dev_in = {k: torch.empty_like(v) for k, v in rounds[0].items()}
+    dev_keep = torch.empty_like(keeps[0])
+    host_y = torch.empty(B, n_pos, shape.H, shape.P).pin_memory()
+    h2d = (sum(v.numel() * v.element_size() for v in host_rounds[0].values()) + B * 4) * R
+    d2h = host_y.numel() * host_y.element_size() * R
+    Kx = max(3, min(K, 50))
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(Kx):
+        for hx, hk in zip(host_rounds, host_keeps):
+            for k in dev_in:
+                dev_in[k].copy_(hx[k], non_blocking=True)
+            dev_keep.copy_(hk, non_blocking=True)
+            r.verify(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dt"], dev_in["a"], y=y)
+            r.rollback(dev_keep)
+            host_y.copy_(y, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / Kx, world, device)
+    r.close()
+
+    return {
+        "metric": SPEC_METRIC,
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": shape.name, "batch": B, "heads": shape.H, "groups": shape.G, "P": shape.P,
+                   "N": shape.N, "L": shape.L, "n_pos": n_pos, "io": shape.io, "ckpt": shape.ckpt,
+                   "step": f"{R} verify rounds of {n_pos} positions x {B} sequences, each rolled back to 1 + accepted",
+                   "global_batch": B * world, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (checkpoint %d MiB per GPU)" % (B * shape.H * shape.P * shape.N * 4 >> 20)},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": achieved_gbs / peak, "traffic": None, "peak_source": peak_kind,
+                     "kernel": "verify round = pack_entries_kernel + replay_kernel + rollback_kernel (events bracket the rounds)",
+                     "round_us": round_ms * 1e3, "algorithmic_bytes_per_round": total_bytes / (K * R)},
+        "e2e": {"value": world * tokens_per_step / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K * R,
+        "clocks": clk,
+        "tokens_per_round": tokens_per_step / R,
+    }
+
+
 # ------------------------------------------------------------------ reference arm (the oracle)
 
 def run_reference(args, rank, world):
@@ -344,13 +470,28 @@ def run_reference(args, rank, world):
 
     one = shape.replace(B=1)
     S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))
-    xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()}
-          for t in range(shape.L)]
+    spec = shape.max_pos > 1
+    if spec:
+        # one step: L verify rounds of max_pos positions, each rolled back to 1 + accepted
+        xs = [{k: gen.to_numpy64(v) for k, v in gen.verify_inputs(one, t, shape.max_pos, device="cpu").items()}
+              for t in range(shape.L)]
+        keeps = [gen.accepted_lengths(one, t, shape.max_pos, device="cpu").numpy().astype(np.int64) + 1
+                 for t in range(shape.L)]
+        step_tokens = int(sum(k.sum() for k in keeps))
+    else:
+        xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()}
+              for t in range(shape.L)]
+        step_tokens = shape.L + 1
 
     def step():
         seq = ro.ReplayBatch(S0, shape.G, shape.L)
-        for x in xs + xs[:1]:  # one window plus the step that folds it
-            seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
+        if spec:
+            for x, nk in zip(xs, keeps):
+                seq.verify(x["q"], x["k"], x["v"], x["dt"], x["a"])
+                seq.rollback(nk)
+        else:
+            for x in xs + xs[:1]:  # one window plus the step that folds it
+                seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
 
     with threadpool_limits(1):
         for _ in range(args.warmup):
@@ -359,11 +500,15 @@ def run_reference(args, rank, world):
         for _ in range(args.steps):
             step()
         secs = time.perf_counter() - t0
-    tokens = (shape.L + 1) * args.steps
+    tokens = step_tokens * args.steps
     value = tokens / secs
-    sample = f"each step: 1 sequence x {shape.H} heads x {shape.L + 1} decode steps of {shape.name}"
+    if spec:
+        sample = (f"each step: 1 sequence x {shape.H} heads x {shape.L} verify rounds of {shape.max_pos} positions "
+                  f"({step_tokens} accepted tokens) of {shape.name}")
+    else:
+        sample = f"each step: 1 sequence x {shape.H} heads x {shape.L + 1} decode steps of {shape.name}"
     return {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "impl": "reference", "metric": SPEC_METRIC if spec else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": shape.name, "batch": shape.B, "heads": shape.H, "groups": shape.G, "P": shape.P,
@@ -389,6 +534,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             out = run_reference(args, rank, world)
+        elif gen.SHAPES[args.workload].max_pos > 1:
+            out = run_spec_ours(args, rank, world, local)
         else:
             out = run_ours(args, rank, world, local)
         if rank == 0 and out is not None:

@@ -339,11 +339,11 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
 // k_l . q_s is a private dot product (no cross-lane reduction). It leaves, per position
 // s, alpha_s and cw[s][l] = w_{s,l} (k_l . q_s); the row lanes then form
 // u_s[p] = sum_l cw[s][l] v_l[p] for the rows they hold.
-template <int N, typename IO>
+template <int N, typename IO, int NQ>
 __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
                                              int n, int o0, float* alpha, float* cw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
+  constexpr int NQR = NQ > 0 ? NQ : 1;
   const int width = c + n - o0;   // window entries (at most L): lane l holds entry o0 + l
   const bool mine = lane < width;
   float xa = 1.f, xd = 0.f;
@@ -351,26 +351,50 @@ __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& r
     xa = rec.a(o0 + lane);
     xd = rec.dt(o0 + lane);
   }
+  // k_l . q_s: for one position two independent chains over the row; for several, each
+  // k element is read once for all positions (their chains are independent)
+  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
   const uint8_t* kr = rec.k(o0 + (mine ? lane : 0));
-  for (int s = 0; s < n; ++s) {
-    const int last = c + s - o0;  // position s replays window entries 0 .. last
-    const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
-    float excl = __shfl_down_sync(0xffffffffu, incl, 1);
-    if (lane == 31) excl = 1.f;
-    if (lane == 0) alpha[s] = incl;
-    // k_l . q_s
-    const uint8_t* qs = qbuf + (size_t)s * N * S_IO;
-    float d0 = 0.f, d1 = 0.f;
+  float d[NQR];
+#pragma unroll
+  for (int s = 0; s < NQR; ++s) d[s] = 0.f;
+  if constexpr (NQR == 1) {
+    float d1 = 0.f;
 #pragma unroll
     for (int e = 0; e < N; e += 2 * EPV) {
-      d0 += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qs + (size_t)e * S_IO));
-      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 4) * S_IO));
+      d[0] += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qbuf + (size_t)e * S_IO));
+      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 4) * S_IO));
       if (EPV == 8) {
-        d0 += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 8) * S_IO));
-        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 12) * S_IO));
+        d[0] += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 8) * S_IO));
+        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 12) * S_IO));
       }
     }
-    if (lane <= last) cw[s * kMaxWindow + lane] = xd * excl * (d0 + d1);  // w_{s,l} (k_l . q_s)
+    d[0] += d1;
+  } else {
+#pragma unroll 2
+    for (int e = 0; e < N; e += 8) {
+      const float4 k0 = IoT<IO>::load4(kr + (size_t)e * S_IO);
+      const float4 k1 = IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO);
+#pragma unroll
+      for (int s = 0; s < NQR; ++s) {
+        if (s < n) {
+          const uint8_t* qs = qbuf + ((size_t)s * N + e) * S_IO;
+          d[s] += dot4(k0, IoT<IO>::load4(qs)) + dot4(k1, IoT<IO>::load4(qs + 4 * S_IO));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < NQR; ++s) {
+    if (s < n) {
+      const int last = c + s - o0;  // position s replays window entries 0 .. last
+      const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
+      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+      if (lane == 31) excl = 1.f;
+      if (lane == 0) alpha[s] = incl;
+      // w_{s,l} (k_l . q_s); zero past `last`, so that the row lanes may read whole vectors
+      cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * d[s] : 0.f;
+    }
   }
 }
 
@@ -425,7 +449,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       fold_weights<N, IO, MODE>(rec, c, sig, lane);
       group_sync(bar_id, GT);
     }
-    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, alpha, cw, lane);
+    if (MODE == kModeReplay) output_coefs<N, IO, NQ>(rec, qbuf, c, n, o0, alpha, cw, lane);
     group_sync(bar_id, GT);
   } else {
     float4 qr[NQR];
@@ -472,37 +496,56 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       }
     };
     // y_s[p] = alpha_s d + sum_l cw[s][l] v_l[p] (replay) or y[p] = d (eager), by the
-    // lanes that hold row p's dot product; eight entries' v in flight at a time
+    // lanes that hold row p's dot products; each v_l[p] is read once for all positions,
+    // eight entries in flight at a time (cw is zero past each position's window, v is
+    // zero past the unit's)
     auto emit = [&](int gi, bool from_tile_fp8) {
       if (MODE == kModeFlush) return;
 #pragma unroll
-      for (int s = 0; s < NQ; ++s) {
-        if (s < n) {
+      for (int i = 0; i < Red::kHeld; ++i) {
+        const int pr = gi * RGR + rbase + dbase + i;
+        if (dwr && pr < P) {
+          const float sc = from_tile_fp8 ? scale_tile[pr] : 1.f;
+          if (MODE == kModeReplay && NQR == 1) {
+            const int last = c - o0;  // the one position replays window entries 0 .. last
+            float b0 = 0.f, b1 = 0.f;
+            for (int l0 = 0; l0 <= last; l0 += 8) {
+              float vv[8];
 #pragma unroll
-          for (int i = 0; i < Red::kHeld; ++i) {
-            const int pr = gi * RGR + rbase + dbase + i;
-            if (dwr && pr < P) {
-              const float d = from_tile_fp8 ? dv[s][i] * scale_tile[pr] : dv[s][i];
-              if (MODE == kModeReplay) {
-                const int last = c + s - o0;
-                const float* cws = cw + s * kMaxWindow;
-                float b0 = 0.f, b1 = 0.f;
-                for (int l0 = 0; l0 <= last; l0 += 8) {
-                  float vv[8];
+              for (int r = 0; r < 8; ++r)
+                vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
 #pragma unroll
-                  for (int r = 0; r < 8; ++r)
-                    vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
-#pragma unroll
-                  for (int r = 0; r < 8; r += 2) {
-                    if (l0 + r <= last) b0 = fmaf(cws[l0 + r], vv[r], b0);
-                    if (l0 + r + 1 <= last) b1 = fmaf(cws[l0 + r + 1], vv[r + 1], b1);
-                  }
-                }
-                p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], d, b0 + b1);
-              } else {
-                p.y[bh * P + pr] = d;
+              for (int r = 0; r < 8; r += 2) {
+                if (l0 + r <= last) b0 = fmaf(cw[l0 + r], vv[r], b0);
+                if (l0 + r + 1 <= last) b1 = fmaf(cw[l0 + r + 1], vv[r + 1], b1);
               }
             }
+            p.y[(((size_t)pl.b * n) * p.H + pl.h) * P + pr] = fmaf(alpha[0], dv[0][i] * sc, b0 + b1);
+          } else if (MODE == kModeReplay) {
+            const int width = c + n - o0;
+            float b[NQR];
+#pragma unroll
+            for (int s = 0; s < NQR; ++s) b[s] = 0.f;
+            for (int l0 = 0; l0 < width; l0 += 8) {
+              float vv[8];
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+                vv[r] = (l0 + r < width) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
+#pragma unroll
+              for (int s = 0; s < NQR; ++s) {
+                if (s < n) {
+                  const float4 c0 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0);
+                  const float4 c1 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0 + 4);
+                  b[s] = fmaf(c0.x, vv[0], fmaf(c0.y, vv[1], fmaf(c0.z, vv[2], fmaf(c0.w, vv[3],
+                         fmaf(c1.x, vv[4], fmaf(c1.y, vv[5], fmaf(c1.z, vv[6], fmaf(c1.w, vv[7], b[s]))))))));
+                }
+              }
+            }
+#pragma unroll
+            for (int s = 0; s < NQR; ++s)
+              if (s < n) p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], dv[s][i] * sc, b[s]);
+          } else {
+            p.y[bh * P + pr] = dv[0][i] * sc;
           }
         }
       }

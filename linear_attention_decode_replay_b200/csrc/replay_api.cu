@@ -193,10 +193,14 @@ int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const voi
   pp.qpack = n_pos > 1 ? ctx->bufs.qpack : nullptr;
   pp.counts_in = p.counts_in;
   p.qpack = pp.qpack;
-  const long long tasks = (long long)p.B * p.H;
-  const long long blocks = (tasks + 7) / 8;
-  const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
-  if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
+  if (n_pos == 1) {
+    p.append_here = 1;  // the main kernel appends the one new entry itself
+  } else {
+    const long long tasks = (long long)p.B * p.H;
+    const long long blocks = (tasks + 7) / 8;
+    const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
+    if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
+  }
   const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
   if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos > 1 ? replay::kMaxPos : 1, ctx->num_sms, s) !=
       cudaSuccess)

@@ -20,6 +20,7 @@ constexpr int kMaxPos = 8;                       // query positions per verify c
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
 constexpr int kMaxStages = 8;
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
+constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
 constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 
@@ -126,6 +127,10 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // Named barrier `id` (1 + group) spans the `count` threads of one consumer group only.
 __device__ __forceinline__ void group_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Arrive on named barrier `id` (of `count` threads) without waiting.
+__device__ __forceinline__ void named_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 // Group barrier with an AND-vote across the group's threads.
 __device__ __forceinline__ bool group_all(bool v, int id, int count) {

@@ -118,6 +118,60 @@ struct Records {
   }
 };
 
+// ---------------------------------------------------------------------------- append
+// This CTA's units' new entries (one position) into their ring records, slot
+// (start + c) mod cap, by the consumer threads before any bulk copy is issued. The input
+// pieces do not depend on the pointer word, so both reads are in flight together.
+template <int S_IO>
+__device__ __forceinline__ void append_entries(const KParams& p) {
+  constexpr int kPool = kConsumerWarps * 32;
+  constexpr int kBatch = 8;  // pieces per thread in flight
+  const int R = p.rec_bytes;
+  const int kpe = p.N * S_IO / 16;  // 16-byte pieces of k, then of v
+  const int vpe = p.P * S_IO / 16;
+  const int per_unit = kpe + vpe + 1;
+  const int units = (p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int total = units * per_unit;
+  for (int t0 = threadIdx.x; t0 < total; t0 += kBatch * kPool) {
+    uint4 val[kBatch];
+    uint8_t* dst[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int t = t0 + r * kPool;
+      dst[r] = nullptr;
+      val[r] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < total) {
+        const int iu = t / per_unit;
+        const int ch = t - iu * per_unit;
+        const int u = (int)blockIdx.x + iu * (int)gridDim.x;
+        const int b = u / p.H;
+        const int h = u - b * p.H;
+        const int g = h / p.hpg;
+        const int32_t word = __ldg(p.counts_in + b);
+        if (ch < kpe) {
+          val[r] = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.k) + ((size_t)b * p.G + g) * p.N * S_IO)[ch];
+        } else if (ch < kpe + vpe) {
+          val[r] = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.v) + ((size_t)b * p.H + h) * p.P * S_IO)[ch - kpe];
+        } else {
+          val[r].x = __float_as_uint(__ldg(p.dt + (size_t)b * p.H + h));
+          val[r].y = __float_as_uint(__ldg(p.a + (size_t)b * p.H + h));
+        }
+        const int start = word >> 16;
+        const int c = word & 0xFFFF;
+        if (!(word < 0 || c > p.L || start >= p.cap)) {  // a bad word is reported by the consumers
+          int slot = start + c;
+          slot -= (slot >= p.cap) ? p.cap : 0;
+          dst[r] = static_cast<uint8_t*>(p.ring) + (((size_t)b * p.H + h) * p.cap + slot) * R + (size_t)ch * 16;
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r)
+      if (dst[r]) *reinterpret_cast<uint4*>(dst[r]) = val[r];
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------- producer
 // Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile, 1 the FP8 row
 // scales, 2-3 the live ring records [start, start + count) modulo cap, 4 the queries.
@@ -160,7 +214,7 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, 
 // count, and then one predicated bulk-copy instruction issues every copy of the batch
 // (lane = unit in batch * kCopyKinds + kind). Issuing costs the warp about as much for
 // one copy as for a whole batch, so batching is what keeps the stream fed.
-template <int MODE, int CKPT, int S_IO>
+template <int MODE, int CKPT, int S_IO, bool APPEND>
 __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   constexpr int U = kUnitsPerIssue;
   static_assert(U * kCopyKinds <= 32 && (32 % U) == 0, "a batch's copies must fit one warp and tile 32 units");
@@ -188,6 +242,33 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   load_words(32, w_nxt, m_nxt);
   const int j = lane / kCopyKinds;     // this lane's unit within the batch
   const int kind = lane % kCopyKinds;  // and its copy
+  // When the kernel appends this call's entries itself, the first stages' state tiles
+  // (and FP8 scales) go out at once and their records and queries once the entries are
+  // in the ring; every stage is armed with its unit's full byte count either way.
+  int pre = 0;
+  if (APPEND && p.append_here) {
+    pre = min(NS, total);
+    for (int i = 0; i < pre; ++i) {
+      const int32_t word = __shfl_sync(0xffffffffu, w_cur, i & 31);
+      const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), word, 1);
+      uint8_t* st = stages + (size_t)i * p.stage_bytes;
+      if (lane == 0) {
+        reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
+        reinterpret_cast<int32_t*>(st + p.off_meta)[1] = 1;
+        if (pl.corrupt) report_error(p.status, kErrPointer);
+        mbar_arrive_expect_tx(&bars->full[i], pl.bytes);
+      }
+      __syncwarp();
+      const uint8_t* src;
+      uint8_t* dst;
+      uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, st, lane, src, dst);
+      if (lane > 1) bytes = 0;
+      __syncwarp();
+      if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->full[i], lane == 0 ? stream_policy : keep_policy);
+      if (lane == 0) bars->last_fill[i] = i;
+    }
+    group_sync(kAppendBar, kThreads);  // the entries are in the ring
+  }
   for (int i0 = 0; i0 < total; i0 += U) {
     if ((i0 & 31) == 0 && i0 > 0) {
       w_cur = w_nxt;
@@ -219,7 +300,8 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     uint8_t* st = stages + (size_t)s * p.stage_bytes;
     uint64_t* bar = &bars->full[s];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), word, msk);
-    if (valid && kind == 0) {
+    const bool armed = i < pre;  // tile already issued, stage already armed
+    if (valid && kind == 0 && !armed) {
       reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
       reinterpret_cast<int32_t*>(st + p.off_meta)[1] = msk;
       if (pl.corrupt) report_error(p.status, kErrPointer);
@@ -229,7 +311,7 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     const uint8_t* src;
     uint8_t* dst;
     uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, st, kind, src, dst);
-    if (!valid) bytes = 0;
+    if (!valid || (armed && kind <= 1)) bytes = 0;
     __syncwarp();
     if (bytes) bulk_g2s_hint(dst, src, bytes, bar, kind == 0 ? stream_policy : keep_policy);
     if (valid && kind == 0) bars->last_fill[s] = i;
@@ -689,13 +771,23 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     fence_mbar_init();
   }
   __syncthreads();
+  if constexpr (MODE == kModeReplay && NQ == 1) {
+    // One-position calls append their entries here rather than in a pre-pass: each CTA
+    // writes the new ring record of each of its own units (k, v, then Delta and a in one
+    // 16-byte piece), makes the writes visible to the bulk copies that read them, and
+    // tells the producer, which meanwhile streams the first state tiles.
+    if (p.append_here && threadIdx.x < kConsumerWarps * 32) {
+      append_entries<S_IO>(p);
+      named_arrive(kAppendBar, kThreads);
+    }
+  }
 
   const int warp = threadIdx.x / 32;
   if (warp >= kConsumerWarps) {
     if constexpr (MODE == kModeEager)
       producer_loop_eager<CKPT, S_IO>(p, stages, bars);
     else
-      producer_loop<MODE, CKPT, S_IO>(p, stages, bars);
+      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, stages, bars);
     return;
   }
   const int g = warp / Gr::kWarps;  // consumer group

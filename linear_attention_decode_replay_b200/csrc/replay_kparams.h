@@ -12,6 +12,7 @@ struct KParams {
   // sizes
   int32_t B, H, G, P, N, L, cap, n_pos, hpg, num_units;
   int32_t commit;  // replay: 1 = step (new entries committed), 0 = verify (tentative)
+  int32_t append_here;  // replay, one position: the kernel appends the entries (no pre-pass)
   // this call's inputs and outputs
   const void* q;
   const void* k;

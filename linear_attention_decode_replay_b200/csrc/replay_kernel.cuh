@@ -421,62 +421,41 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
 // k_l . q_s is a private dot product (no cross-lane reduction). It leaves, per position
 // s, alpha_s and cw[s][l] = w_{s,l} (k_l . q_s); the row lanes then form
 // u_s[p] = sum_l cw[s][l] v_l[p] for the rows they hold.
-template <int N, typename IO, int NQ>
+// The coefficients of the positions s = s0, s0 + ds, ... (< n) by one warp: alpha_s and
+// cw[s][l] = w_{s,l} (k_l . q_s), lane l holding window entry o0 + l, so that k_l . q_s
+// is a private dot product (two independent chains over the row).
+template <int N, typename IO>
 __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
-                                             int n, int o0, float* alpha, float* cw, int lane) {
+                                             int n, int o0, int s0, int ds, float* alpha, float* cw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  constexpr int NQR = NQ > 0 ? NQ : 1;
-  const int width = c + n - o0;   // window entries (at most L): lane l holds entry o0 + l
+  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
+  const int width = c + n - o0;   // window entries (at most L)
   const bool mine = lane < width;
   float xa = 1.f, xd = 0.f;
   if (mine) {
     xa = rec.a(o0 + lane);
     xd = rec.dt(o0 + lane);
   }
-  // k_l . q_s: for one position two independent chains over the row; for several, each
-  // k element is read once for all positions (their chains are independent)
-  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
   const uint8_t* kr = rec.k(o0 + (mine ? lane : 0));
-  float d[NQR];
-#pragma unroll
-  for (int s = 0; s < NQR; ++s) d[s] = 0.f;
-  if constexpr (NQR == 1) {
-    float d1 = 0.f;
+  for (int s = s0; s < n; s += ds) {
+    const uint8_t* qs = qbuf + (size_t)s * N * S_IO;
+    float d0 = 0.f, d1 = 0.f;
 #pragma unroll
     for (int e = 0; e < N; e += 2 * EPV) {
-      d[0] += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qbuf + (size_t)e * S_IO));
-      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 4) * S_IO));
+      d0 += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qs + (size_t)e * S_IO));
+      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 4) * S_IO));
       if (EPV == 8) {
-        d[0] += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 8) * S_IO));
-        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qbuf + (size_t)(e + 12) * S_IO));
+        d0 += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 8) * S_IO));
+        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 12) * S_IO));
       }
     }
-    d[0] += d1;
-  } else {
-#pragma unroll 2
-    for (int e = 0; e < N; e += 8) {
-      const float4 k0 = IoT<IO>::load4(kr + (size_t)e * S_IO);
-      const float4 k1 = IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO);
-#pragma unroll
-      for (int s = 0; s < NQR; ++s) {
-        if (s < n) {
-          const uint8_t* qs = qbuf + ((size_t)s * N + e) * S_IO;
-          d[s] += dot4(k0, IoT<IO>::load4(qs)) + dot4(k1, IoT<IO>::load4(qs + 4 * S_IO));
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < NQR; ++s) {
-    if (s < n) {
-      const int last = c + s - o0;  // position s replays window entries 0 .. last
-      const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
-      float excl = __shfl_down_sync(0xffffffffu, incl, 1);
-      if (lane == 31) excl = 1.f;
-      if (lane == 0) alpha[s] = incl;
-      // w_{s,l} (k_l . q_s); zero past `last`, so that the row lanes may read whole vectors
-      cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * d[s] : 0.f;
-    }
+    const int last = c + s - o0;  // position s replays window entries 0 .. last
+    const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
+    float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+    if (lane == 31) excl = 1.f;
+    if (lane == 0) alpha[s] = incl;
+    // zero past `last`, so that the row lanes may read whole vectors
+    cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * (d0 + d1) : 0.f;
   }
 }
 
@@ -531,7 +510,8 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       fold_weights<N, IO, MODE>(rec, c, sig, lane);
       group_sync(bar_id, GT);
     }
-    if (MODE == kModeReplay) output_coefs<N, IO, NQ>(rec, qbuf, c, n, o0, alpha, cw, lane);
+    // the positions are spread over the group's warps: this warp takes 0, GW + 1, ...
+    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, lane);
     group_sync(bar_id, GT);
   } else {
     float4 qr[NQR];
@@ -639,6 +619,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       // terms; further row groups (P > one row group) follow with the terms in hand
       load_rows(x, 0, false);
       row_dots(x);
+      if (NQ > 1) output_coefs<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);  // positions gw+1, ...
       group_sync(bar_id, GT);
       emit(0, !pl.fp32_tile);
       for (int gi = 1; gi < ngroups; ++gi) {
@@ -722,6 +703,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
           }
         }
         if (MODE != kModeFlush) row_dots(x);
+        if (MODE == kModeReplay && NQ > 1 && gi == 0) output_coefs<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);
         if (gi == 0) group_sync(bar_id, GT);  // the outputs' buffer terms are in
         emit(gi, false);
       }

@@ -422,40 +422,51 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
 // s, alpha_s and cw[s][l] = w_{s,l} (k_l . q_s); the row lanes then form
 // u_s[p] = sum_l cw[s][l] v_l[p] for the rows they hold.
 // The coefficients of the positions s = s0, s0 + ds, ... (< n) by one warp: alpha_s and
-// cw[s][l] = w_{s,l} (k_l . q_s), lane l holding window entry o0 + l, so that k_l . q_s
-// is a private dot product (two independent chains over the row).
+// cw[s][l] = w_{s,l} (k_l . q_s). The dot products take eight entries per pass, four
+// lanes per entry (a quarter of the row each, two shuffles to combine); the decay
+// weights take one lane per entry.
 template <int N, typename IO>
 __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
                                              int n, int o0, int s0, int ds, float* alpha, float* cw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  constexpr int EPV = 16 / S_IO;  // io elements per 16-byte vector
-  const int width = c + n - o0;   // window entries (at most L)
-  const bool mine = lane < width;
+  constexpr int QN = N / 4;  // elements of a quarter row
+  const int width = c + n - o0;  // window entries (at most L)
   float xa = 1.f, xd = 0.f;
-  if (mine) {
+  if (lane < width) {
     xa = rec.a(o0 + lane);
     xd = rec.dt(o0 + lane);
   }
-  const uint8_t* kr = rec.k(o0 + (mine ? lane : 0));
-  for (int s = s0; s < n; s += ds) {
-    const uint8_t* qs = qbuf + (size_t)s * N * S_IO;
-    float d0 = 0.f, d1 = 0.f;
+  const int quarter = lane & 3;
+  // raw k_l . q_s into cw[s][l]
+  for (int l0 = 0; l0 < width; l0 += 8) {
+    const int l = l0 + (lane >> 2);
+    const uint8_t* kq = rec.k(o0 + (l < width ? l : 0)) + (size_t)quarter * QN * S_IO;
+    for (int s = s0; s < n; s += ds) {
+      const uint8_t* qq = qbuf + ((size_t)s * N + quarter * QN) * S_IO;
+      float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < N; e += 2 * EPV) {
-      d0 += dot4(IoT<IO>::load4(kr + (size_t)e * S_IO), IoT<IO>::load4(qs + (size_t)e * S_IO));
-      d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 4) * S_IO));
-      if (EPV == 8) {
-        d0 += dot4(IoT<IO>::load4(kr + (size_t)(e + 8) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 8) * S_IO));
-        d1 += dot4(IoT<IO>::load4(kr + (size_t)(e + 12) * S_IO), IoT<IO>::load4(qs + (size_t)(e + 12) * S_IO));
+      for (int e = 0; e < QN; e += 8) {
+        d0 += dot4(IoT<IO>::load4(kq + (size_t)e * S_IO), IoT<IO>::load4(qq + (size_t)e * S_IO));
+        if (e + 4 < QN)
+          d1 += dot4(IoT<IO>::load4(kq + (size_t)(e + 4) * S_IO), IoT<IO>::load4(qq + (size_t)(e + 4) * S_IO));
       }
+      float d = d0 + d1;
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
+      d += __shfl_xor_sync(0xffffffffu, d, 2);
+      if (quarter == 0 && l < width) cw[s * kMaxWindow + l] = d;
     }
+  }
+  __syncwarp();
+  for (int s = s0; s < n; s += ds) {
     const int last = c + s - o0;  // position s replays window entries 0 .. last
     const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
     float excl = __shfl_down_sync(0xffffffffu, incl, 1);
     if (lane == 31) excl = 1.f;
     if (lane == 0) alpha[s] = incl;
-    // zero past `last`, so that the row lanes may read whole vectors
-    cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * (d0 + d1) : 0.f;
+    // w_{s,l} (k_l . q_s); zero past `last`, so that the row lanes may read whole vectors
+    const float kqv = (lane <= last) ? cw[s * kMaxWindow + lane] : 0.f;
+    __syncwarp();
+    cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * kqv : 0.f;
   }
 }
 

@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
 # window) from an ncu capture, and the hash of the kernel sources it was taken on. When
 # the sources change the figure no longer applies and is reported as null.
-NCU_TRAFFIC = {"sources_sha256": "2518a94fa40f0118f48ceb870ae5e7986244fcc3d56c362e01d44820b0cc6fcf",
-               "bytes_per_launch": 597.0e6}
+NCU_TRAFFIC = {"sources_sha256": "77956a164585913156ad03ae2fcc9d862a8f3c2733cedcad88d805ee92f59ee3",
+               "bytes_per_launch": 597.6e6}
 
 
 def kernel_sources_hash() -> str:

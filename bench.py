@@ -7,6 +7,9 @@ path: append, decay scan, k.q products, output-only reads of S0, the fused flush
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+`--workload sweep` times replay_step against eager_step over the batch x window x
+head-layout sweep and prints one line with every point.
+
 Under torchrun every rank runs its own replica of the batch on its own GPU (sequences
 are independent; there is no collective on the data path) and the timing is the max
 over ranks. Rank 0 prints one JSON line.
@@ -224,31 +227,40 @@ def run_ours(args, rank, world, local):
 
     K = args.steps
     stream = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
     t_start.record(stream)
-    i = 0
     for _ in range(K):
-        for x in window:
-            ev[i][0].record(stream)
-            r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
-            ev[i][1].record(stream)
-            i += 1
+        one_window()
     t_stop.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier(world)
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), world, device)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    avg_launch_ms = max_over_ranks(sum(launch_ms) / len(launch_ms), world, device)
-    # in lockstep decode the first launch of every timed window folds the buffers
-    fold_ms = statistics.mean(launch_ms[0::L])
-    out_ms = statistics.mean([t for j, t in enumerate(launch_ms) if j % L]) if L > 1 else fold_ms
+    # one replay_kernel launch per step, back to back: the average launch over the timed
+    # region (gaps between launches included)
+    avg_launch_ms = elapsed_ms / (K * L)
     status = r.check_status()
     if status:
         raise RuntimeError(f"device status bits {status} after the timed region")
+
+    # ---- fold and output-only launches apart: an instrumented pass with an event pair
+    # around every launch (the events add gaps, so this pass is not the timed one); in
+    # lockstep decode the first launch of every window folds the buffers
+    Ki = max(3, min(K, 100))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ki * L)]
+    i = 0
+    for _ in range(Ki):
+        for x in window:
+            ev[i][0].record(stream)
+            r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+            ev[i][1].record(stream)
+            i += 1
+    torch.cuda.synchronize()
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    fold_ms = statistics.mean(launch_ms[0::L])
+    out_ms = statistics.mean([t for j, t in enumerate(launch_ms) if j % L]) if L > 1 else fold_ms
 
     bpt = algorithmic_bytes_per_token(shape)
     bytes_per_launch = bpt["replay"] * B  # one launch decodes one token of every sequence
@@ -336,6 +348,7 @@ def run_ours(args, rank, world, local):
                      "kernel": "replay_kernel (replay_step: appends the entries, then streams the state)",
                      "avg_launch_us": avg_launch_ms * 1e3,
                      "fold_launch_us": fold_ms * 1e3, "output_launch_us": out_ms * 1e3,
+                     "launch_split": f"fold / output-only launch times from {Ki} instrumented windows",
                      "algorithmic_bytes_per_launch": bytes_per_launch},
         "e2e": {"value": world * B * L / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -542,22 +555,122 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------------------ our arm, batch x window sweep
+
+SWEEP_METRIC = "decode tokens/s per SSM layer, replay vs the in-house eager kernel, over batch x window x head layout (1 B200)"
+
+
+def run_sweep_ours(args, rank, world, local):
+    """Every point of gen.sweep_shapes(): replay_step in lockstep windows and eager_step,
+    each over the same 256 decode steps (256 / L windows), the median of three timed
+    repetitions after one warm-up window. Per point: tokens/s of both, the replay/eager
+    ratio and the fraction of the measured HBM bandwidth by the algorithmic bytes. Points
+    whose checkpoint fits in L2 (126 MB) are marked: their steps re-read it from L2."""
+    import linear_attention_decode_replay_b200 as lar
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_hbm_peak()
+    steps = 256
+
+    def timed(fn, reps=3):
+        out = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1))
+        return statistics.median(out)
+
+    points = []
+    clocks = ClockSampler(local)
+    clocks.start()
+    for shape in gen.sweep_shapes(steps):
+        L, B = shape.L, shape.B
+        cfg = lar.Config(batch=B, heads=shape.H, groups=shape.G, P=shape.P, N=shape.N, L=L, max_pos=1,
+                         io=shape.io, ckpt=shape.ckpt)
+        bufs = lar.alloc_buffers(cfg, device)
+        S0 = gen.initial_state(shape, device=device)
+        bufs["S0"].copy_(S0)
+        r = lar.Replay(cfg, bufs)
+        window = [gen.step_inputs(shape, t, device=device) for t in range(L)]
+        y = torch.empty(B, shape.H, shape.P, device=device)
+
+        def replay_steps():
+            for _ in range(steps // L):
+                for x in window:
+                    r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+
+        for x in window:
+            r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+        replay_ms = max_over_ranks(timed(replay_steps), world, device)
+        if r.check_status():
+            raise RuntimeError(f"device status bits set at {shape.name}")
+        r.close()
+        del bufs
+        S = S0
+
+        def eager_steps():
+            for j in range(steps):
+                x = window[j % L]
+                lar.eager_step(cfg, S, x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+
+        for x in window:
+            lar.eager_step(cfg, S, x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+        eager_ms = max_over_ranks(timed(eager_steps), world, device)
+        bpt = algorithmic_bytes_per_token(shape)
+        tok = world * B * steps
+        state_bytes = B * shape.H * shape.P * shape.N * 4
+        points.append({
+            "batch": B, "L": L, "heads": shape.H, "P": shape.P, "N": shape.N,
+            "replay_tokens_s": tok / (replay_ms * 1e-3), "eager_tokens_s": tok / (eager_ms * 1e-3),
+            "speedup": eager_ms / replay_ms,
+            "replay_frac": bpt["replay"] * B * steps / (replay_ms * 1e-3) / 1e9 / peak,
+            "eager_frac": bpt["eager"] * B * steps / (eager_ms * 1e-3) / 1e9 / peak,
+            "l2_resident": state_bytes <= 126 * 2**20,
+        })
+        del S, S0, window, y
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    hbm = [p["speedup"] for p in points if not p["l2_resident"]]
+    geo = float(np.exp(np.mean(np.log(hbm))))
+    return {
+        "metric": SWEEP_METRIC, "value": geo, "unit": "x (replay / eager tokens/s, geometric mean over the points whose state exceeds L2)",
+        "n_gpus": world, "steps": steps, "warmup": 1, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "sweep", "batch": [1, 16, 64, 256, 1024], "L": [4, 8, 16, 32],
+                   "heads_P": [[64, 64], [32, 128]], "N": 128, "io": "bf16", "ckpt": "f32",
+                   "step": f"{steps} decode steps per point, median of 3",
+                   "l2": "points with a checkpoint under 126 MB are L2-resident and marked"},
+        "peak_gbs": peak, "peak_source": peak_kind, "clocks": clk, "points": points,
+        "gpu_launches": 3 * 2 * steps * len(points),
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1500, help="timed windows of L decode steps")
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mamba2_b256", choices=sorted(k for k in gen.SHAPES if k != "tiny"))
+    ap.add_argument("--workload", default="mamba2_b256",
+                    choices=sorted(k for k in gen.SHAPES if k != "tiny") + ["sweep"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.impl == "reference" and args.workload == "sweep":
+        ap.error("the sweep has no reference arm: --impl reference times the oracle on one workload")
     rank, world, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
             out = run_reference(args, rank, world)
+        elif args.workload == "sweep":
+            out = run_sweep_ours(args, rank, world, local)
         elif gen.SHAPES[args.workload].max_pos > 1:
             out = run_spec_ours(args, rank, world, local)
         else:

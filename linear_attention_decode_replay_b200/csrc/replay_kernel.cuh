@@ -417,17 +417,26 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
   if (lane == 0) sig[kMaxWindow] = incl;
 }
 
-// The coefficient warp keeps its dependent chains short: lane l holds entry o0 + l, so
-// k_l . q_s is a private dot product (no cross-lane reduction). It leaves, per position
-// s, alpha_s and cw[s][l] = w_{s,l} (k_l . q_s); the row lanes then form
-// u_s[p] = sum_l cw[s][l] v_l[p] for the rows they hold.
 // The coefficients of the positions s = s0, s0 + ds, ... (< n) by one warp: alpha_s and
-// cw[s][l] = w_{s,l} (k_l . q_s). The dot products take eight entries per pass, four
-// lanes per entry (a quarter of the row each, two shuffles to combine); the decay
-// weights take one lane per entry.
+// cw[s][l] = w_{s,l} (k_l . q_s) with w_{s,l} = Delta_l prod_{l < i <= last_s} a_i, zero
+// past the position's last entry so that the row lanes may read whole vectors. Two
+// forms, chosen by measurement:
+//  * output_coefs_pairs, for one-position calls on the FP32 checkpoint, where one warp
+//    per group forms the coefficients while four stream the state and its chain is on
+//    the unit's critical path: a lane pair per entry, sixteen entries per pass (half of k_l . q_s per lane,
+//    the second half one 4-element chunk rotated so that the pair's reads fall in
+//    different shared-memory banks, one shuffle to combine), and each lane forms its
+//    entry's decay weight itself from broadcast reads of the a_i. Its chain is one round
+//    of shared-memory reads, the products and one shuffle.
+//  * output_coefs_quarters, for multi-position calls, where all five warps of a group
+//    form coefficients at once and the shared-memory pipe, not one warp's chain, is the
+//    limit, and for the FP8 read copy, whose row warps (decoding the codes) rather than
+//    the coefficient warp set the pace: four lanes per entry, eight entries per pass,
+//    and the decay weights by a suffix-product scan across the lanes, which issues fewer
+//    shared-memory requests per position than the broadcast reads.
 template <int N, typename IO>
-__device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
-                                             int n, int o0, int s0, int ds, float* alpha, float* cw, int lane) {
+__device__ __forceinline__ void output_coefs_quarters(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
+                                                      int n, int o0, int s0, int ds, float* alpha, float* cw, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
   constexpr int QN = N / 4;  // elements of a quarter row
   const int width = c + n - o0;  // window entries (at most L)
@@ -467,6 +476,51 @@ __device__ __forceinline__ void output_coefs(const Records<N, IoT<IO>::bytes>& r
     const float kqv = (lane <= last) ? cw[s * kMaxWindow + lane] : 0.f;
     __syncwarp();
     cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * kqv : 0.f;
+  }
+}
+
+
+template <int N, typename IO>
+__device__ __forceinline__ void output_coefs_pairs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
+                                                   int n, int o0, int s0, int ds, float* alpha, float* cw, int lane) {
+  constexpr int S_IO = IoT<IO>::bytes;
+  constexpr int HN = N / 2;       // elements of half a row
+  constexpr int HC = HN / 4;      // 4-element chunks of half a row
+  constexpr int kBlock = 16;      // decay factors read per round
+  const int width = c + n - o0;   // window entries (at most kMaxWindow)
+  const int half = lane & 1;
+  for (int e0 = 0; e0 < width; e0 += 16) {
+    const int e = e0 + (lane >> 1);
+    const int er = (e < width) ? e : width - 1;  // lanes past the window read a valid record
+    const uint8_t* kh = rec.k(o0 + er) + (size_t)half * HN * S_IO;
+    const float xd = rec.dt(o0 + er);
+    for (int s = s0; s < n; s += ds) {
+      const int last = c + s - o0;  // position s replays window entries 0 .. last
+      const uint8_t* qh = qbuf + ((size_t)s * N + half * HN) * S_IO;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int t = 0; t < HC; ++t) {
+        const int off = ((t + half) % HC) * 4 * S_IO;
+        const float4 kk = IoT<IO>::load4(kh + off);
+        const float4 qq = IoT<IO>::load4(qh + off);
+        d[t & 3] = fmaf(kk.x, qq.x, fmaf(kk.y, qq.y, fmaf(kk.z, qq.z, fmaf(kk.w, qq.w, d[t & 3]))));
+      }
+      float kq = (d[0] + d[1]) + (d[2] + d[3]);
+      kq += __shfl_xor_sync(0xffffffffu, kq, 1);
+      // prod_{e < i <= last} a_i; i runs from e0 + 1 (i <= e0 never counts for this pass)
+      float w = 1.f;
+      float a_first = 1.f;  // a_{o0}, for alpha
+      for (int t0 = (e0 == 0) ? 0 : e0 + 1; t0 <= last; t0 += kBlock) {
+        float at[kBlock];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) at[r] = (t0 + r <= last) ? rec.a(o0 + t0 + r) : 1.f;
+        if (t0 == 0) a_first = at[0];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) w = (t0 + r > e) ? w * at[r] : w;
+      }
+      if (half == 0 && e < kMaxWindow) cw[s * kMaxWindow + e] = (e <= last) ? xd * w * kq : 0.f;
+      if (lane == 0 && e0 == 0) alpha[s] = a_first * w;  // prod_{0 <= i <= last} a_i
+    }
   }
 }
 
@@ -522,7 +576,12 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       group_sync(bar_id, GT);
     }
     // the positions are spread over the group's warps: this warp takes 0, GW + 1, ...
-    if (MODE == kModeReplay) output_coefs<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, lane);
+    if (MODE == kModeReplay) {
+      if (NQ > 1 || CKPT == kCkptFp8)
+        output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, lane);
+      else
+        output_coefs_pairs<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, lane);
+    }
     group_sync(bar_id, GT);
   } else {
     float4 qr[NQR];
@@ -568,21 +627,49 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         }
       }
     };
+    // Multi-position calls, where a lane ends with one row (N >= 64): the v_l[p] of the
+    // first kPre window entries and the row's scale are read into registers before the
+    // group barrier, while the group forms the coefficients; after the barrier only the
+    // coefficients are read. (One-position calls measured no gain from it.)
+    constexpr int kPre = (MODE == kModeReplay && NQ > 1 && Red::kHeld == 1) ? 16 : 0;  // 0 or 16
+    float vpre[16];  // the first kPre used
+    float scpre = 1.f;
+    auto preload = [&](int gi, bool from_tile_fp8) {
+      if constexpr (kPre > 0) {
+        const int pr = gi * RGR + rbase + dbase;
+        const bool own = dwr && pr < P;
+        const int width = c + n - o0;
+#pragma unroll
+        for (int r = 0; r < kPre; ++r)
+          vpre[r] = (own && r < width) ? IoT<IO>::load1(rec.v(o0 + r) + (size_t)pr * S_IO) : 0.f;
+        scpre = (own && from_tile_fp8) ? scale_tile[pr] : 1.f;
+      }
+    };
     // y_s[p] = alpha_s d + sum_l cw[s][l] v_l[p] (replay) or y[p] = d (eager), by the
     // lanes that hold row p's dot products; each v_l[p] is read once for all positions,
     // eight entries in flight at a time (cw is zero past each position's window, v is
-    // zero past the unit's)
-    auto emit = [&](int gi, bool from_tile_fp8) {
+    // zero past the unit's). `pre`: the preload above ran for this row group.
+    auto emit = [&](int gi, bool from_tile_fp8, bool pre) {
       if (MODE == kModeFlush) return;
 #pragma unroll
       for (int i = 0; i < Red::kHeld; ++i) {
         const int pr = gi * RGR + rbase + dbase + i;
         if (dwr && pr < P) {
-          const float sc = from_tile_fp8 ? scale_tile[pr] : 1.f;
+          const float sc = (kPre > 0 && pre) ? scpre : (from_tile_fp8 ? scale_tile[pr] : 1.f);
           if (MODE == kModeReplay && NQR == 1) {
             const int last = c - o0;  // the one position replays window entries 0 .. last
             float b0 = 0.f, b1 = 0.f;
-            for (int l0 = 0; l0 <= last; l0 += 8) {
+            int l0 = 0;
+            if (kPre > 0 && pre) {
+              const float4* c4 = reinterpret_cast<const float4*>(cw);
+              const float4 c0 = c4[0], c1 = c4[1], c2 = c4[2], c3 = c4[3];
+              b0 = fmaf(c0.x, vpre[0], fmaf(c0.y, vpre[1], fmaf(c0.z, vpre[2], fmaf(c0.w, vpre[3],
+                   fmaf(c1.x, vpre[4], fmaf(c1.y, vpre[5], fmaf(c1.z, vpre[6], c1.w * vpre[7])))))));
+              b1 = fmaf(c2.x, vpre[8], fmaf(c2.y, vpre[9], fmaf(c2.z, vpre[10], fmaf(c2.w, vpre[11],
+                   fmaf(c3.x, vpre[12], fmaf(c3.y, vpre[13], fmaf(c3.z, vpre[14], c3.w * vpre[15])))))));
+              l0 = kPre;
+            }
+            for (; l0 <= last; l0 += 8) {
               float vv[8];
 #pragma unroll
               for (int r = 0; r < 8; ++r)
@@ -599,7 +686,26 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
             float b[NQR];
 #pragma unroll
             for (int s = 0; s < NQR; ++s) b[s] = 0.f;
-            for (int l0 = 0; l0 < width; l0 += 8) {
+            int l0 = 0;
+            if (kPre > 0 && pre) {
+#pragma unroll
+              for (int h = 0; h < kPre; h += 8) {
+                if (h < width) {
+#pragma unroll
+                  for (int s = 0; s < NQR; ++s) {
+                    if (s < n) {
+                      const float4 c0 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + h);
+                      const float4 c1 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + h + 4);
+                      const float* vv = vpre + h;
+                      b[s] = fmaf(c0.x, vv[0], fmaf(c0.y, vv[1], fmaf(c0.z, vv[2], fmaf(c0.w, vv[3],
+                             fmaf(c1.x, vv[4], fmaf(c1.y, vv[5], fmaf(c1.z, vv[6], fmaf(c1.w, vv[7], b[s]))))))));
+                    }
+                  }
+                }
+              }
+              l0 = kPre;
+            }
+            for (; l0 < width; l0 += 8) {
               float vv[8];
 #pragma unroll
               for (int r = 0; r < 8; ++r)
@@ -630,13 +736,15 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       // terms; further row groups (P > one row group) follow with the terms in hand
       load_rows(x, 0, false);
       row_dots(x);
-      if (NQ > 1) output_coefs<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);  // positions gw+1, ...
+      preload(0, !pl.fp32_tile);
+      if (NQ > 1) output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);  // positions gw+1, ...
       group_sync(bar_id, GT);
-      emit(0, !pl.fp32_tile);
+      emit(0, !pl.fp32_tile, true);
       for (int gi = 1; gi < ngroups; ++gi) {
         load_rows(x, gi, false);
         row_dots(x);
-        emit(gi, !pl.fp32_tile);
+        preload(gi, !pl.fp32_tile);
+        emit(gi, !pl.fp32_tile, true);
       }
     } else {
       // ---- fold (state route), write the state back, outputs from the fresh rows
@@ -714,9 +822,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
           }
         }
         if (MODE != kModeFlush) row_dots(x);
-        if (MODE == kModeReplay && NQ > 1 && gi == 0) output_coefs<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);
+        if (MODE == kModeReplay && NQ > 1 && gi == 0) output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, lane);
         if (gi == 0) group_sync(bar_id, GT);  // the outputs' buffer terms are in
-        emit(gi, false);
+        emit(gi, false, false);
       }
     }
   }

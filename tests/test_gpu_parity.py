@@ -125,6 +125,58 @@ def test_eager_fp8_small():
     assert rep.max_err <= 1e-3, rep.max_err
 
 
+def _all_finite_e4m3_codes(P=16, N=16):
+    """The 256 e4m3 codes as a P x N block (byte 16 p + n), NaN codes 0x7F / 0xFF replaced
+    by +0 / -0 (the quantiser never writes NaN), and row scales 2^(p - 8)."""
+    codes = np.arange(256, dtype=np.uint8).reshape(P, N)
+    codes[codes == 0x7F] = 0x00
+    codes[codes == 0xFF] = 0x80
+    scale = np.exp2(np.arange(P) - 8.0).astype(np.float32)
+    return codes, scale
+
+
+def _one_hot_step(shape, n):
+    """Inputs under which y[p] = (state row p) . e_n exactly: query e_n, Delta 0, a 1."""
+    q = torch.zeros(shape.B, shape.G, shape.N, device="cuda")
+    q[:, :, n] = 1.0
+    k = torch.zeros_like(q)
+    v = torch.zeros(shape.B, shape.H, shape.P, device="cuda")
+    return q, k, v, torch.zeros(shape.B, shape.H, device="cuda"), torch.ones(shape.B, shape.H, device="cuda")
+
+
+def test_fp8_read_copy_decodes_every_code():
+    """The output-only route's decode of the e4m3 read copy, every code: with a one-hot
+    query, Delta = 0 and a = 1 every output is one decoded code times its row's scale,
+    exactly; all 254 finite codes against the oracle's table (OCP e4m3)."""
+    shape = gen.Shape("f4", B=1, H=1, G=1, P=16, N=16, L=16, io="f32", ckpt="f32_fp8read", seed=34)
+    cfg, bufs, r, _ = hx.setup(shape)
+    codes, scale = _all_finite_e4m3_codes()
+    bufs["S0_fp8"].copy_(torch.from_numpy(codes).view(1, 1, 16, 16))
+    bufs["S0_scale"].copy_(torch.from_numpy(scale).view(1, 1, 16))
+    want = ro.e4m3_decode(codes) * scale[:, None].astype(np.float64)
+    got = np.zeros((16, 16))
+    for n in range(16):  # 16 steps, no flush (the buffer holds L = 16 entries)
+        got[:, n] = r.step(*_one_hot_step(shape, n)).cpu().numpy()[0, 0]
+    assert r.check_status() == 0
+    assert r.read_counts() == [16]  # sixteen entries buffered: every step was output-only
+    np.testing.assert_array_equal(got, want)
+    r.close()
+
+
+def test_eager_fp8_decodes_every_code():
+    """The same block of codes through the shared-FP8 eager kernel (dequantise, update,
+    y = S q before the state is quantised again): y[p] = decoded code times scale."""
+    shape = gen.Shape("f5", B=1, H=1, G=1, P=16, N=16, L=4, io="f32", seed=35)
+    cfg = hx.lar_config(shape)
+    codes, scale = _all_finite_e4m3_codes()
+    want = ro.e4m3_decode(codes) * scale[:, None].astype(np.float64)
+    for n in (0, 5, 11, 15):
+        S8 = torch.from_numpy(codes).view(1, 1, 16, 16).cuda()
+        sc = torch.from_numpy(scale).view(1, 1, 16).cuda()
+        y = lar.eager_step_fp8(cfg, S8, sc, *_one_hot_step(shape, n))
+        np.testing.assert_array_equal(y.cpu().numpy()[0, 0], want[:, n])
+
+
 # ------------------------------------------------------------------ protocol and error paths
 
 def test_flush_mask_folds_only_selected_sequences():

@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
 # window) from an ncu capture, and the hash of the kernel sources it was taken on. When
 # the sources change the figure no longer applies and is reported as null.
-NCU_TRAFFIC = {"sources_sha256": "77956a164585913156ad03ae2fcc9d862a8f3c2733cedcad88d805ee92f59ee3",
-               "bytes_per_launch": 597.6e6}
+NCU_TRAFFIC = {"sources_sha256": "caaa1e6390b8ce13a8699743266b845fa98da1cad4d154d8bb24ab330ad164f5",
+               "bytes_per_launch": 597.2e6}
 
 
 def kernel_sources_hash() -> str:

@@ -561,11 +561,12 @@ SWEEP_METRIC = "decode tokens/s per SSM layer, replay vs the in-house eager kern
 
 
 def run_sweep_ours(args, rank, world, local):
-    """Every point of gen.sweep_shapes(): replay_step in lockstep windows and eager_step,
-    each over the same 256 decode steps (256 / L windows), the median of three timed
-    repetitions after one warm-up window. Per point: tokens/s of both, the replay/eager
-    ratio and the fraction of the measured HBM bandwidth by the algorithmic bytes. Points
-    whose checkpoint fits in L2 (126 MB) are marked: their steps re-read it from L2."""
+    """Every point of gen.sweep_shapes(): replay_step in lockstep windows (host calls, and
+    replays of one window captured in a CUDA graph) and eager_step, each over the same 256
+    decode steps (256 / L windows), the median of three timed repetitions after one
+    warm-up window. Per point: tokens/s of each, the replay/eager ratios and the fraction
+    of the measured HBM bandwidth by the algorithmic bytes. Points whose checkpoint fits
+    in L2 (126 MB) are marked: their steps re-read it from L2."""
     import linear_attention_decode_replay_b200 as lar
 
     device = torch.device("cuda", local)
@@ -607,8 +608,26 @@ def run_sweep_ours(args, rank, world, local):
         for x in window:
             r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
         replay_ms = max_over_ranks(timed(replay_steps), world, device)
+        # the same steps as replays of one captured window (one graph launch per window
+        # instead of one host call per step: the small-batch path)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.graph(g, stream=side):
+            for x in window:
+                r.step(x["q"], x["k"], x["v"], x["dt"], x["a"], y=y)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+
+        def graph_steps():
+            for _ in range(steps // L):
+                g.replay()
+
+        g.replay()
+        graph_ms = max_over_ranks(timed(graph_steps), world, device)
         if r.check_status():
             raise RuntimeError(f"device status bits set at {shape.name}")
+        del g
         r.close()
         del bufs
         S = S0
@@ -627,7 +646,8 @@ def run_sweep_ours(args, rank, world, local):
         points.append({
             "batch": B, "L": L, "heads": shape.H, "P": shape.P, "N": shape.N,
             "replay_tokens_s": tok / (replay_ms * 1e-3), "eager_tokens_s": tok / (eager_ms * 1e-3),
-            "speedup": eager_ms / replay_ms,
+            "replay_graph_tokens_s": tok / (graph_ms * 1e-3),
+            "speedup": eager_ms / replay_ms, "graph_speedup": eager_ms / graph_ms,
             "replay_frac": bpt["replay"] * B * steps / (replay_ms * 1e-3) / 1e9 / peak,
             "eager_frac": bpt["eager"] * B * steps / (eager_ms * 1e-3) / 1e9 / peak,
             "l2_resident": state_bytes <= 126 * 2**20,
@@ -646,7 +666,7 @@ def run_sweep_ours(args, rank, world, local):
                    "step": f"{steps} decode steps per point, median of 3",
                    "l2": "points with a checkpoint under 126 MB are L2-resident and marked"},
         "peak_gbs": peak, "peak_source": peak_kind, "clocks": clk, "points": points,
-        "gpu_launches": 3 * 2 * steps * len(points),
+        "gpu_launches": 3 * 3 * steps * len(points),
     }
 
 

@@ -31,6 +31,13 @@
  *    L = window, cap = replay_ring_capacity(cfg), R = replay_ring_record_bytes(cfg).
  *    "io" is the replay_config.io dtype.
  *  - A replay_ctx is not thread-safe; calls on one context must be serialised.
+ *  - replay_step and replay_flush queue kernels only, so a run of them can be captured
+ *    into a CUDA graph and replayed (a graph launch per window instead of a host call
+ *    per step), under three conditions: one call of the same kind has run outside the
+ *    capture (the first launch of a kernel sets its shared-memory limit); the inputs
+ *    and outputs are the buffers named at capture; and the run holds an even number of
+ *    calls, because each call flips which half of `counts` holds the pointer words and
+ *    the graph keeps the halves it was captured with.
  */
 #ifndef REPLAY_H
 #define REPLAY_H

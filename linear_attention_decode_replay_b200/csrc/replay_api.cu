@@ -90,7 +90,10 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
     lfold = 1;
   }
   p->rec_bytes = record_bytes(c);
-  const int tile = fp8_eager ? round_up(P * N + P * 4, 16) : P * N * 4;
+  // a unit is one row group of a head (all of it when P is smaller): its tile is at most
+  // 64 rows x 128 floats, whatever P
+  const int UR = P < replay::row_group_rows(N) ? P : replay::row_group_rows(N);
+  const int tile = fp8_eager ? round_up(UR * N + UR * 4, 16) : UR * N * 4;
   p->off_rec = round_up(tile, 16);
   p->off_q = p->off_rec + jmax * p->rec_bytes;
   p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
@@ -98,8 +101,8 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
 
   // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
   // abar, the outputs' entry coefficients [kMaxPos][kMaxWindow], and the fold weights
-  // times v, [lfold][wt_stride] (rows padded to a multiple of kRowsPerThread)
-  p->wt_stride = round_up(c.P, replay::kRowsPerThread);
+  // times v, [lfold][wt_stride] (a unit's rows, padded to a multiple of kRowsPerThread)
+  p->wt_stride = round_up(UR, replay::kRowsPerThread);
   p->ws_alpha = 0;
   p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
   p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
@@ -122,13 +125,16 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->L = c.L;
   p->cap = cap;
   p->hpg = c.heads / c.groups;
-  p->num_units = c.batch * c.heads;
+  p->rows_unit = UR;
+  p->row_blocks = (P + UR - 1) / UR;
+  p->num_bh = c.batch * c.heads;
+  p->num_units = p->num_bh * p->row_blocks;
   return REPLAY_OK;
 }
 
 cudaError_t launch_main(const KParams& p, const replay_config& c, int ckpt, int mode, int nq, int num_sms,
                         cudaStream_t s) {
-  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  const int grid = p.num_bh < num_sms ? p.num_bh : num_sms;  // every CTA holds whole heads
   switch (c.N) {
     case 16: return replay::launch_replay_n16(p, c.io, ckpt, mode, nq, grid, s);
     case 32: return replay::launch_replay_n32(p, c.io, ckpt, mode, nq, grid, s);

@@ -22,6 +22,11 @@ constexpr int kMaxStages = 8;
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
 constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
 constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
+// State rows of one row group: kGroupGemvWarps warps, 128/N rows per warp pass (a row of
+// N floats takes N/4 lanes), kRowsPerThread rows per lane. A unit covers one row group of
+// a head (or the whole head when it has fewer rows), so that every unit's tile is at most
+// 32 KiB of FP32 and as many stages fit in shared memory whatever the head's P.
+constexpr int row_group_rows(int N) { return kGroupGemvWarps * (128 / N) * kRowsPerThread; }
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 
 // status word bits (device-detected errors; the host reads them with replay_check_status)

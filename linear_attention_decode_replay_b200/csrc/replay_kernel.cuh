@@ -58,18 +58,34 @@ struct Bars {
 static_assert(sizeof(Bars) <= 256, "the barrier header must fit the 256 bytes the host layout reserves");
 
 struct Plan {
-  int b, h, g, start, c;
+  int b, h, g, rb, r0, rows, start, c;  // rows r0 .. r0 + rows - 1 of head h of sequence b
   bool fold, corrupt, active, fp32_tile;
   uint32_t bytes;
 };
 
+// This CTA's units, in the order its producer fills them and its groups take them: the
+// heads blockIdx.x, blockIdx.x + gridDim.x, ..., each with its row blocks in a row, so
+// that one CTA holds every unit of a head (the in-kernel append writes a head's new
+// record once, before any copy of it).
+__device__ __forceinline__ int cta_units(const KParams& p) {
+  return (p.num_bh - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x * p.row_blocks;
+}
+__device__ __forceinline__ int cta_unit(const KParams& p, int i) {
+  const int bh = (int)blockIdx.x + (i / p.row_blocks) * (int)gridDim.x;
+  return bh * p.row_blocks + (i % p.row_blocks);
+}
+
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word, int msk) {
   Plan pl;
-  pl.b = u / p.H;
-  pl.h = u - pl.b * p.H;
+  const int bh = u / p.row_blocks;
+  pl.rb = u - bh * p.row_blocks;
+  pl.b = bh / p.H;
+  pl.h = bh - pl.b * p.H;
   pl.g = pl.h / p.hpg;
-  const uint32_t P = p.P, N = p.N;
+  pl.r0 = pl.rb * p.rows_unit;
+  pl.rows = min(p.rows_unit, p.P - pl.r0);
+  const uint32_t P = pl.rows, N = p.N;  // the unit's rows
   if (MODE == kModeEager) {
     pl.start = 0;
     pl.c = 0;
@@ -130,8 +146,8 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
   const int kpe = p.N * S_IO / 16;  // 16-byte pieces of k, then of v
   const int vpe = p.P * S_IO / 16;
   const int per_unit = kpe + vpe + 1;
-  const int units = (p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  const int total = units * per_unit;
+  const int heads = (p.num_bh - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // this CTA's
+  const int total = heads * per_unit;
   for (int t0 = threadIdx.x; t0 < total; t0 += kBatch * kPool) {
     uint4 val[kBatch];
     uint8_t* dst[kBatch];
@@ -143,9 +159,9 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
       if (t < total) {
         const int iu = t / per_unit;
         const int ch = t - iu * per_unit;
-        const int u = (int)blockIdx.x + iu * (int)gridDim.x;
-        const int b = u / p.H;
-        const int h = u - b * p.H;
+        const int bh = (int)blockIdx.x + iu * (int)gridDim.x;
+        const int b = bh / p.H;
+        const int h = bh - b * p.H;
         const int g = h / p.hpg;
         const int32_t word = __ldg(p.counts_in + b);
         if (ch < kpe) {
@@ -173,15 +189,17 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
 }
 
 // ---------------------------------------------------------------------------- producer
-// Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile, 1 the FP8 row
-// scales, 2-3 the live ring records [start, start + count) modulo cap, 4 the queries.
+// Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile (the unit's rows),
+// 1 their FP8 row scales, 2-3 the live ring records [start, start + count) modulo cap
+// (whole records: every row block reads all of k and its rows of v), 4 the queries.
 // Returns the bytes of copy `kind` (0 if none) and its addresses.
 constexpr int kCopyKinds = 5;
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, uint8_t* st, int kind,
                                               const uint8_t*& src, uint8_t*& dst) {
-  const size_t P = p.P, N = p.N;
+  const size_t P = pl.rows, N = p.N;
   const size_t bh = (size_t)pl.b * p.H + pl.h;
+  const size_t row0 = bh * p.P + pl.r0;  // the unit's first state row
   const int R = p.rec_bytes;
   const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
   const int first = min(cnt, p.cap - pl.start);
@@ -189,14 +207,14 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, 
   const size_t bg = (size_t)pl.b * p.G + pl.g;
   const uint8_t* qsrc = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
                                 : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
-  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + bh * P * N) : p.S8 + bh * P * N;
+  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + row0 * N) : p.S8 + row0 * N;
   src = (kind == 0)   ? tsrc
-        : (kind == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + bh * P)
+        : (kind == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + row0)
         : (kind == 2) ? ring + (size_t)pl.start * R
         : (kind == 3) ? ring
                       : qsrc;
   dst = (kind == 0)   ? st
-        : (kind == 1) ? st + P * N
+        : (kind == 1) ? st + (size_t)p.rows_unit * N  // the scales follow a full unit's codes
         : (kind == 2) ? st + p.off_rec
         : (kind == 3) ? st + p.off_rec + (size_t)first * R
                       : st + p.off_q;
@@ -222,16 +240,15 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   const int NS = p.num_stages;
   const uint64_t stream_policy = l2_evict_first_policy();
   const uint64_t keep_policy = l2_evict_normal_policy();
-  const int total = (p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  auto unit_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
+  const int total = cta_units(p);
+  auto unit_of = [&](int i) { return cta_unit(p, i); };
   // pointer words (and flush masks) 32 units at a time, one chunk ahead: lane j of a
   // chunk holds the word of the chunk's j-th unit
   auto load_words = [&](int i0, int32_t& w, int& msk) {
     w = 0;
     msk = 1;
-    const int uu = unit_of(i0 + lane);
-    if (uu < p.num_units) {
-      const int b = uu / p.H;
+    if (i0 + lane < total) {
+      const int b = unit_of(i0 + lane) / p.row_blocks / p.H;
       w = __ldg(p.counts_in + b);
       if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
     }
@@ -334,8 +351,9 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bar
   const int NS = p.num_stages;
   const uint64_t stream_policy = l2_evict_first_policy();
   const size_t P = p.P, N = p.N;
-  int i = 0;
-  for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++i) {
+  const int total = cta_units(p);
+  for (int i = 0; i < total; ++i) {
+    const int u = cta_unit(p, i);
     const int s = i % NS;
     const int k = i / NS;
     if (k > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1))) {
@@ -352,13 +370,15 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bar
     uint64_t* bar = &bars->full[s];
     const size_t bh = (size_t)pl.b * p.H + pl.h;
     const size_t bg = (size_t)pl.b * p.G + pl.g;
+    const size_t row0 = bh * P + pl.r0;  // the unit's rows
+    const uint32_t rows = (uint32_t)pl.rows;
     uint8_t* recbuf = st + p.off_rec;
     if (lane == 0) mbar_arrive_expect_tx(bar, pl.bytes);
     __syncwarp();
     if (lane == 0)
-      bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + bh * P * N) : (const void*)(p.S8 + bh * P * N),
-                    pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * N), bar, stream_policy);
-    if (lane == 1 && !pl.fp32_tile) bulk_g2s(st + P * N, p.Sscale + bh * P, (uint32_t)(P * 4), bar);
+      bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + row0 * N) : (const void*)(p.S8 + row0 * N),
+                    pl.fp32_tile ? (uint32_t)(rows * N * 4) : (uint32_t)(rows * N), bar, stream_policy);
+    if (lane == 1 && !pl.fp32_tile) bulk_g2s(st + (size_t)p.rows_unit * N, p.Sscale + row0, rows * 4u, bar);
     const int kpe = (int)(N * S_IO / 16);
     const int vpe = (int)(P * S_IO / 16);
     for (int idx = lane; idx < 2 * kpe + vpe; idx += 32) {
@@ -550,7 +570,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   // fold reads their weights as four 16-byte vectors)
   const int rbase = (gw * RPW + lane / TPR) * RT;
   const int col = (lane % TPR) * 4;
-  const int P = p.P;
+  const int P = pl.rows;  // the unit's rows: r0 .. r0 + P - 1 of the head's PH
+  const int PH = p.P;
+  const int r0 = pl.r0;
   const int c = pl.c;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
@@ -558,8 +580,8 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const int wts = p.wt_stride;  // row stride of the fold weight table, >= P, multiple of RT
   const uint8_t* tile = st;
   const uint8_t* qbuf = st + p.off_q;
-  const Records<N, S_IO> rec{st + p.off_rec, P, p.rec_bytes};
-  const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)P * N);
+  const Records<N, S_IO> rec{st + p.off_rec, PH, p.rec_bytes};  // whole records: v_j[0 .. PH)
+  const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)p.rows_unit * N);
   float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);  // [kMaxPos]
   float* sig = reinterpret_cast<float*>(ws + p.ws_sig);      // fold weights; [kMaxWindow] = abar
   float* cw = reinterpret_cast<float*>(ws + p.ws_cw);        // [kMaxPos][kMaxWindow] entry coefficients
@@ -641,7 +663,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         const int width = c + n - o0;
 #pragma unroll
         for (int r = 0; r < kPre; ++r)
-          vpre[r] = (own && r < width) ? IoT<IO>::load1(rec.v(o0 + r) + (size_t)pr * S_IO) : 0.f;
+          vpre[r] = (own && r < width) ? IoT<IO>::load1(rec.v(o0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
         scpre = (own && from_tile_fp8) ? scale_tile[pr] : 1.f;
       }
     };
@@ -673,14 +695,14 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
               float vv[8];
 #pragma unroll
               for (int r = 0; r < 8; ++r)
-                vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
+                vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
 #pragma unroll
               for (int r = 0; r < 8; r += 2) {
                 if (l0 + r <= last) b0 = fmaf(cw[l0 + r], vv[r], b0);
                 if (l0 + r + 1 <= last) b1 = fmaf(cw[l0 + r + 1], vv[r + 1], b1);
               }
             }
-            p.y[(((size_t)pl.b * n) * p.H + pl.h) * P + pr] = fmaf(alpha[0], dv[0][i] * sc, b0 + b1);
+            p.y[(((size_t)pl.b * n) * p.H + pl.h) * PH + r0 + pr] = fmaf(alpha[0], dv[0][i] * sc, b0 + b1);
           } else if (MODE == kModeReplay) {
             const int width = c + n - o0;
             float b[NQR];
@@ -709,7 +731,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
               float vv[8];
 #pragma unroll
               for (int r = 0; r < 8; ++r)
-                vv[r] = (l0 + r < width) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)pr * S_IO) : 0.f;
+                vv[r] = (l0 + r < width) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
 #pragma unroll
               for (int s = 0; s < NQR; ++s) {
                 if (s < n) {
@@ -722,9 +744,9 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
             }
 #pragma unroll
             for (int s = 0; s < NQR; ++s)
-              if (s < n) p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * P + pr] = fmaf(alpha[s], dv[s][i] * sc, b[s]);
+              if (s < n) p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * PH + r0 + pr] = fmaf(alpha[s], dv[s][i] * sc, b[s]);
           } else {
-            p.y[bh * P + pr] = dv[0][i] * sc;
+            p.y[bh * PH + r0 + pr] = dv[0][i] * sc;
           }
         }
       }
@@ -760,7 +782,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           const int jj = min(j8 * 8 + r, cf - 1);
-          wv[r] = sig[jj] * IoT<IO>::load1(rec.v(jj) + pv * S_IO);
+          wv[r] = sig[jj] * IoT<IO>::load1(rec.v(jj) + (size_t)(r0 + pv) * S_IO);
         }
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
@@ -810,14 +832,14 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           const int pr = gi * RGR + rbase + r;
-          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * P + pr) * N + col), x[r]);
+          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * PH + r0 + pr) * N + col), x[r]);
           if (store_fp8) {
             const float am = seg_allmax<TPR>(amax4(x[r]));
             float sc, inv;
             e4m3_row_scale(am, sc, inv);
             if (pr < P) {
-              __stcs(reinterpret_cast<unsigned int*>(p.S8 + (bh * P + pr) * N + col), quant4_e4m3(x[r], inv));
-              if ((lane % TPR) == 0) p.Sscale[bh * P + pr] = sc;
+              __stcs(reinterpret_cast<unsigned int*>(p.S8 + (bh * PH + r0 + pr) * N + col), quant4_e4m3(x[r], inv));
+              if ((lane % TPR) == 0) p.Sscale[bh * PH + r0 + pr] = sc;
             }
           }
         }
@@ -833,7 +855,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   const int start = pl.start;
   const int cap = p.cap;
   if (MODE == kModeReplay) {
-    if (pl.h == 0 && gtid == 0) {
+    if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
       int start2 = fold ? start + c : start;
       start2 -= (start2 >= cap) ? cap : 0;
       const int base = fold ? 0 : c;
@@ -842,7 +864,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       if (p.flushed) p.flushed[pl.b] = fold ? 1 : 0;
     }
   } else if (MODE == kModeFlush) {
-    if (pl.h == 0 && gtid == 0) {
+    if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
       int start2 = start + c;
       start2 -= (start2 >= cap) ? cap : 0;
       p.counts_out[pl.b] = start2 << 16;
@@ -897,8 +919,9 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   const int gemv_bar_id = 1 + NG + g;       // the group's row warps only
   uint8_t* ws = smem + p.ws_off + (size_t)g * p.ws_group_bytes;
   const int NS = p.num_stages;
-  int i = g;
-  for (int u = blockIdx.x + g * gridDim.x; u < p.num_units; u += NG * gridDim.x, i += NG) {
+  const int total = cta_units(p);
+  for (int i = g; i < total; i += NG) {
+    const int u = cta_unit(p, i);
     const int s = i % NS;
     const int k = i / NS;  // this is the k-th use of stage s
     // Parity waits only tell apart a phase and the one just before it, so before waiting
@@ -923,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u, word, msk);
     if (pl.active) {
       consume_unit<N, IO, CKPT, MODE, NQ, NG>(p, pl, st, ws, gtid, bar_id, gemv_bar_id);
-    } else if (pl.h == 0 && gtid == 0) {
+    } else if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
       p.counts_out[pl.b] = word;  // nothing to fold: the pointer word carries over
       if (MODE == kModeFlush && p.flushed && !pl.corrupt) p.flushed[pl.b] = 0;
     }

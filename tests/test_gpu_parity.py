@@ -64,6 +64,8 @@ RAGGED = [
     gen.Shape("r4", B=2, H=2, G=2, P=8, N=16, L=1, io="f32", seed=14),
     # one head, one group, prefill-shaped checkpoint
     gen.Shape("r5", B=4, H=1, G=1, P=64, N=128, L=16, io="bf16", s0="prefill", seed=15),
+    # two row-block units per head (N = 64: 128 rows per unit), a group shared by two heads
+    gen.Shape("r6", B=3, H=2, G=1, P=256, N=64, L=4, io="bf16", seed=16),
 ]
 
 
@@ -74,7 +76,7 @@ def test_ragged_shapes_match_oracle(shape):
     _check_decode(rep)
 
 
-@pytest.mark.parametrize("shape", RAGGED[:3], ids=[s.name for s in RAGGED[:3]])
+@pytest.mark.parametrize("shape", RAGGED[:3] + RAGGED[5:], ids=[s.name for s in RAGGED[:3] + RAGGED[5:]])
 def test_ragged_eager_matches_oracle(shape):
     rep = hx.run_eager(shape, 9, np.arange(shape.B))
     assert rep.max_err <= hx.TOL_F32 and rep.ckpt_err <= hx.TOL_F32, (rep.max_err, rep.ckpt_err)
@@ -84,6 +86,8 @@ SPEC = [
     gen.Shape("s1", B=4, H=4, G=2, P=16, N=32, L=8, io="bf16", max_pos=5, seed=21),
     gen.Shape("s2", B=3, H=2, G=2, P=24, N=16, L=5, io="f32", max_pos=5, seed=22),
     gen.Shape("s3", B=2, H=2, G=1, P=64, N=128, L=16, io="bf16", max_pos=8, seed=23),
+    # two row-block units per head: every unit replays the same records for its rows
+    gen.Shape("s5", B=3, H=2, G=2, P=128, N=128, L=8, io="bf16", max_pos=5, seed=25),
 ]
 
 
@@ -100,8 +104,9 @@ def test_verify_with_fewer_positions(n_pos):
     _check_decode(rep)
 
 
-def test_fp8_read_copy_small():
-    shape = gen.Shape("f1", B=3, H=2, G=2, P=32, N=64, L=4, io="f32", ckpt="f32_fp8read", seed=31)
+@pytest.mark.parametrize("P,N", [(32, 64), (96, 128)], ids=["one_unit", "row_blocks_64_32"])
+def test_fp8_read_copy_small(P, N):
+    shape = gen.Shape("f1", B=3, H=2, G=2, P=P, N=N, L=4, io="f32", ckpt="f32_fp8read", seed=31)
     rep = hx.run_decode(shape, 21, np.arange(shape.B), fp8_emulation=True)
     assert rep.max_err_fp8_emul <= 1e-3, rep.max_err_fp8_emul
     assert rep.fro_err <= hx.TOL_FP8, rep.fro_err
@@ -119,8 +124,9 @@ def test_fp8_init_copy_bit_exact():
     r.close()
 
 
-def test_eager_fp8_small():
-    shape = gen.Shape("f3", B=2, H=2, G=2, P=32, N=64, L=4, io="f32", seed=33)
+@pytest.mark.parametrize("P,N", [(32, 64), (96, 128)], ids=["one_unit", "row_blocks_64_32"])
+def test_eager_fp8_small(P, N):
+    shape = gen.Shape("f3", B=2, H=2, G=2, P=P, N=N, L=4, io="f32", seed=33)
     rep = hx.run_eager(shape, 12, np.arange(shape.B), fp8=True)
     assert rep.max_err <= 1e-3, rep.max_err
 

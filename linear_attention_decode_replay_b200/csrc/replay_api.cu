@@ -126,7 +126,9 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->cap = cap;
   p->hpg = c.heads / c.groups;
   p->rows_unit = UR;
-  p->row_blocks = (P + UR - 1) / UR;
+  p->row_blocks = (P + UR - 1) / UR;  // 1 or 2: P <= 65536 / (4 N) <= 2 row groups
+  p->rb_shift = p->row_blocks == 1 ? 0 : 1;
+  if (p->row_blocks > 2) return REPLAY_EINVAL;
   p->num_bh = c.batch * c.heads;
   p->num_units = p->num_bh * p->row_blocks;
   return REPLAY_OK;

@@ -68,18 +68,18 @@ struct Plan {
 // that one CTA holds every unit of a head (the in-kernel append writes a head's new
 // record once, before any copy of it).
 __device__ __forceinline__ int cta_units(const KParams& p) {
-  return (p.num_bh - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x * p.row_blocks;
+  return ((p.num_bh - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) << p.rb_shift;
 }
 __device__ __forceinline__ int cta_unit(const KParams& p, int i) {
-  const int bh = (int)blockIdx.x + (i / p.row_blocks) * (int)gridDim.x;
-  return bh * p.row_blocks + (i % p.row_blocks);
+  const int bh = (int)blockIdx.x + (i >> p.rb_shift) * (int)gridDim.x;
+  return (bh << p.rb_shift) | (i & (p.row_blocks - 1));
 }
 
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word, int msk) {
   Plan pl;
-  const int bh = u / p.row_blocks;
-  pl.rb = u - bh * p.row_blocks;
+  const int bh = u >> p.rb_shift;
+  pl.rb = u & (p.row_blocks - 1);
   pl.b = bh / p.H;
   pl.h = bh - pl.b * p.H;
   pl.g = pl.h / p.hpg;
@@ -248,7 +248,7 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     w = 0;
     msk = 1;
     if (i0 + lane < total) {
-      const int b = unit_of(i0 + lane) / p.row_blocks / p.H;
+      const int b = (unit_of(i0 + lane) >> p.rb_shift) / p.H;
       w = __ldg(p.counts_in + b);
       if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
     }

@@ -12,8 +12,9 @@ struct KParams {
   // sizes
   int32_t B, H, G, P, N, L, cap, n_pos, hpg;
   // units: a unit is rows [rb * rows_unit, min(P, (rb + 1) * rows_unit)) of one head of one
-  // sequence, u = (b * H + h) * row_blocks + rb; all row blocks of a head go to one CTA
-  int32_t rows_unit, row_blocks, num_bh, num_units;
+  // sequence, u = (b * H + h) * row_blocks + rb with row_blocks = 1 << rb_shift (1 or 2);
+  // all row blocks of a head go to one CTA
+  int32_t rows_unit, row_blocks, rb_shift, num_bh, num_units;
   int32_t commit;  // replay: 1 = step (new entries committed), 0 = verify (tentative)
   int32_t append_here;  // replay, one position: the kernel appends the entries (no pre-pass)
   // this call's inputs and outputs

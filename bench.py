@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
 # window) from an ncu capture, and the hash of the kernel sources it was taken on. When
 # the sources change the figure no longer applies and is reported as null.
-NCU_TRAFFIC = {"sources_sha256": "caaa1e6390b8ce13a8699743266b845fa98da1cad4d154d8bb24ab330ad164f5",
-               "bytes_per_launch": 597.2e6}
+NCU_TRAFFIC = {"sources_sha256": "02e754b9f0ac5f3f23f0ef3b60c8386e72f01b065fcf05a98a712ee408d5eafb",
+               "bytes_per_launch": 597.3e6}
 
 
 def kernel_sources_hash() -> str:

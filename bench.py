@@ -41,9 +41,10 @@ SPEC_METRIC = "speculative decode tokens/s per SSM layer at batch 256, L=16, dra
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of one replay_step launch (flush and output-only launches averaged over a
-# window) from an ncu capture, and the hash of the kernel sources it was taken on. When
-# the sources change the figure no longer applies and is reported as null.
-NCU_TRAFFIC = {"sources_sha256": "02e754b9f0ac5f3f23f0ef3b60c8386e72f01b065fcf05a98a712ee408d5eafb",
+# window) of the workload it was captured on, from an ncu capture, and the hash of the
+# kernel sources it was taken on. For another workload, or once the sources change, the
+# figure does not apply and is reported as null.
+NCU_TRAFFIC = {"workload": "mamba2_b256", "sources_sha256": "02e754b9f0ac5f3f23f0ef3b60c8386e72f01b065fcf05a98a712ee408d5eafb",
                "bytes_per_launch": 597.3e6}
 
 
@@ -267,7 +268,7 @@ def run_ours(args, rank, world, local):
     achieved_gbs = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_peak()
     traffic = None
-    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_hash():
+    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_hash() and NCU_TRAFFIC["workload"] == shape.name:
         traffic = NCU_TRAFFIC["bytes_per_launch"]
 
     tokens = world * B * L * K

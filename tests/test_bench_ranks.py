@@ -55,7 +55,7 @@ def test_single_rank_max_is_identity():
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
 
 
-def test_algorithmic_bytes_match_the_survey_figures():
+def test_algorithmic_bytes_per_token_of_the_b256_layer():
     """Per-token bytes of the B=256, L=16 layer: 2,228,224 state bytes for replay vs
     4,194,304 for eager (a 32/17 cut), 2,524,416 in total."""
     sys.path.insert(0, ROOT)

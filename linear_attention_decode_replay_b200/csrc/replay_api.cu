@@ -210,7 +210,7 @@ int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const voi
     if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
   }
   const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
-  if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos > 1 ? replay::kMaxPos : 1, ctx->num_sms, s) !=
+  if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos, ctx->num_sms, s) !=
       cudaSuccess)
     return REPLAY_ECUDA;
   ctx->parity ^= 1;
@@ -559,7 +559,7 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
   const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
   if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
   const int ckpt = cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
-  if (launch_main(p, cfg, ckpt, replay::kModeReplay, replay::kMaxPos, ctx->num_sms, s) != cudaSuccess)
+  if (launch_main(p, cfg, ckpt, replay::kModeReplay, n_pos, ctx->num_sms, s) != cudaSuccess)
     return REPLAY_ECUDA;
   ctx->parity ^= 1;
   ctx->pending = n_pos;

@@ -33,11 +33,17 @@ cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+constexpr int kVerifyPosSmall = 5;  // positions of the smaller multi-position instance
+
 template <typename IO, int CKPT>
 cudaError_t launch_mode(const KParams& p, int mode, int nq, int grid, cudaStream_t s) {
   if (mode == kModeReplay) {
-    return nq > 1 ? launch_one<IO, CKPT, kModeReplay, kMaxPos>(p, grid, s)
-                  : launch_one<IO, CKPT, kModeReplay, 1>(p, grid, s);
+    // multi-position calls: an instance unrolled over five positions for the common
+    // draft of four (n_pos <= 5), whose code fits the instruction cache better than the
+    // eight-position one (measured: 327 against 372 us per verify round of five positions)
+    return nq > 5 ? launch_one<IO, CKPT, kModeReplay, kMaxPos>(p, grid, s)
+           : nq > 1 ? launch_one<IO, CKPT, kModeReplay, kVerifyPosSmall>(p, grid, s)
+                    : launch_one<IO, CKPT, kModeReplay, 1>(p, grid, s);
   }
   if (mode == kModeFlush) return launch_one<IO, CKPT, kModeFlush, 0>(p, grid, s);
   return launch_one<IO, CKPT, kModeEager, 1>(p, grid, s);

@@ -8,7 +8,8 @@
 namespace replay {
 
 // mode: kModeReplay / kModeFlush / kModeEager; ckpt: kCkptF32 / kCkptFp8;
-// io: 0 = FP32, 1 = BF16; nq: query registers (1, or kMaxPos for multi-position verify)
+// io: 0 = FP32, 1 = BF16; nq: the call's query positions (1; 2..5 run the five-position
+// instance, more the kMaxPos one)
 cudaError_t launch_replay_n16(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
 cudaError_t launch_replay_n32(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);
 cudaError_t launch_replay_n64(const KParams& p, int io, int ckpt, int mode, int nq, int grid, cudaStream_t s);

@@ -68,3 +68,24 @@ def test_algorithmic_bytes_per_token_of_the_b256_layer():
     assert b["eager_state"] / b["replay_state"] == pytest.approx(32 / 17)
     f = bench.algorithmic_bytes_per_token(gen.SHAPES["mamba2_b256_fp8"])
     assert f["replay_state"] == 802_816
+
+
+def test_verify_round_bytes_by_hand():
+    """Bytes of one verify round, counted by hand for two sequences of the B=256 layer's
+    head shape: one that folds (12 committed + 5 positions > L = 16) and one that does
+    not (3 + 5)."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from workloads import gen
+
+    s = gen.SHAPES["mamba2_b256_spec"]
+    assert (s.H, s.G, s.P, s.N, s.L, s.io_bytes) == (64, 64, 64, 128, 16, 2)
+    entry = 64 * 128 * 2 + 64 * 64 * 2 + 8 * 64        # k, v, Delta and a of all heads
+    state = 64 * 64 * 128 * 4
+    q5 = 5 * 64 * 128 * 2
+    y5 = 5 * 4 * 64 * 64
+    fold = 2 * state + (12 + 5) * entry + 5 * entry + q5 + y5
+    no_fold = state + (3 + 5) * entry + 5 * entry + q5 + y5
+    assert bench.verify_round_bytes(s, np.array([12, 3]), 5) == float(fold + no_fold)

@@ -13,6 +13,16 @@ provides device memory and streams.
     y = r.verify(q5, k5, v5, dt5, a5)          # 5 speculative positions, output-only
     r.rollback(n_keep)                         # keep n_keep[b] of them (pointer move)
     r.flush()                                  # fold every buffer into the checkpoint
+
+Small batches are bound by the host's launch rate; an even number of ``step`` calls on
+fixed input and output tensors can be captured in a CUDA graph once one call has run
+outside the capture (the conditions are in ``include/replay.h``):
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for t in range(cfg.L):
+            r.step(q[t], k[t], v[t], dt[t], a[t], y=y[t])
+    g.replay()                                 # one window, one graph launch
 """
 
 from __future__ import annotations

@@ -419,6 +419,44 @@ def pin_dual_precision_master_is_exact():
     assert np.max(np.abs(deq - S)) > 0
 
 
+def _fp8_fixture():
+    rows = _read_fixture("fp8_hand_example.txt")
+    codes = {k: np.array([int(x, 16) for x in v], dtype=np.uint8) for k, v in rows.items() if "codes" in k}
+    vals = {k: np.array([float(x) for x in v]) for k, v in rows.items() if "codes" not in k}
+    return codes, vals
+
+
+def pin_shared_fp8_hand_example():
+    """Shared-FP8 eager step worked by hand from the OCP table (fixture, example A): the
+    initial codes, the output taken from the updated values before re-quantising, and
+    the re-quantised codes and scale."""
+    codes, fx = _fp8_fixture()
+    S = fx["A_S"].reshape(1, 1, 1, 4)
+    c0, s0 = ro.quantize_rows_e4m3(S)
+    assert np.array_equal(c0.ravel(), codes["A_codes0"]) and s0.ravel()[0] == fx["A_scale"][0]
+    one = lambda x: np.asarray(x, np.float64).reshape(1, 1, -1)  # noqa: E731 - [B=1][H or G=1][...]
+    c1, s1, y = ro.eager_fp8_batch_step(c0, s0, one(fx["A_q"]), one(fx["A_k"]), one(fx["A_v"]),
+                                        fx["A_dt"].reshape(1, 1), fx["A_a"].reshape(1, 1), 1)
+    assert abs(y.ravel()[0] - fx["A_y"][0]) < 1e-12, y
+    assert np.array_equal(c1.ravel(), codes["A_codes1"]), [hex(x) for x in c1.ravel()]
+    assert s1.ravel()[0] == fx["A_scale"][0]
+
+
+def pin_dual_precision_hand_example():
+    """Dual precision with L = 1 (fixture, example B): a step that does not flush reads
+    the FP8 copy, the step that flushes reads the fresh master."""
+    codes, fx = _fp8_fixture()
+    seq = ro.ReplaySeq(fx["B_S0"].reshape(1, 1, 4), G=1, L=1, ckpt="f32_fp8read")
+    assert np.array_equal(seq.codes.ravel(), codes["B_codes"])
+    q = fx["B_q"].reshape(1, 4)
+    zero_k, zero_v, one, zero = np.zeros((1, 4)), np.zeros((1, 1)), np.ones(1), np.zeros(1)
+    y0, f0 = seq.step(q, zero_k, zero_v, zero, one)
+    y1, f1 = seq.step(q, zero_k, zero_v, zero, one)
+    assert not f0 and f1
+    assert y0.ravel()[0] == fx["B_y0"][0], y0
+    assert abs(y1.ravel()[0] - fx["B_y1"][0]) < 1e-12, y1
+
+
 def pin_relative_error_metric():
     """The error metric is the max over vectors of the relative L2 error."""
     y_ref = np.array([[3.0, 4.0], [0.0, 1.0]])

@@ -3,8 +3,9 @@
 Every mutation below replaces one oracle function (on the CPU, inside this test only)
 with a plausibly wrong version: a dropped term, an off-by-one in a decay product, a
 wrong sign, a transposed operand, a wrong flush or rollback boundary, a wrong rounding
-or scale in the FP8 encoder. If no pin noticed one of them, the pins would not be
-pinning that part of the oracle.
+or scale in the FP8 encoder, an FP8 state read at the wrong moment or never
+re-quantised. If no pin noticed one of them, the pins would not be pinning that part
+of the oracle.
 """
 
 import numpy as np
@@ -14,7 +15,7 @@ import pins
 from oracle import replay_oracle as ro
 
 _orig = {name: getattr(ro, name) for name in dir(ro)}
-_orig_seq = {name: getattr(ro.ReplaySeq, name) for name in ("step", "verify", "rollback", "fold")}
+_orig_seq = {name: getattr(ro.ReplaySeq, name) for name in ("step", "verify", "rollback", "fold", "_output")}
 
 
 def m_decay_includes_own_a(a_buf, dt_buf):
@@ -104,6 +105,10 @@ def m_fold_keeps_buffer(self):
         self.k, self.v, self.dt, self.a = k[-1:], v[-1:], dt[-1:], a[-1:]
 
 
+def m_output_reads_copy_at_flush(self, q, t, from_master):
+    return _orig_seq["_output"](self, q, t, False)
+
+
 def m_e4m3_round_half_up(x):
     x = np.asarray(x, dtype=np.float64)
     sign = np.signbit(x).astype(np.int64) << 7
@@ -138,6 +143,20 @@ def m_quantize_scale_256(S):
     return _orig["e4m3_encode"]((x * inv[..., None]).astype(np.float32)), scale
 
 
+def m_eager_fp8_output_after_requantise(codes, scale, q, k, v, dt, a, G):
+    codes2, scale2, _ = _orig["eager_fp8_batch_step"](codes, scale, q, k, v, dt, a, G)
+    S = ro.dequantize_rows_e4m3(codes2, scale2)
+    B, H = S.shape[:2]
+    gh = np.arange(H) // (H // G)
+    y = np.stack([np.einsum("hpn,hn->hp", S[b], q[b][gh]) for b in range(B)])
+    return codes2, scale2, y
+
+
+def m_eager_fp8_never_requantises(codes, scale, q, k, v, dt, a, G):
+    _, _, y = _orig["eager_fp8_batch_step"](codes, scale, q, k, v, dt, a, G)
+    return codes, scale, y
+
+
 def m_route_flops_counts_outer_twice(P, N, entries):
     f = _orig["route_flops"](P, N, entries)
     return {"outer": 2 * f["outer"], "inner": f["inner"]}
@@ -161,12 +180,15 @@ MODULE_MUTATIONS = [
     ("e4m3_decode", m_e4m3_decode_bias8),
     ("quantize_rows_e4m3", m_quantize_scale_256),
     ("route_flops", m_route_flops_counts_outer_twice),
+    ("eager_fp8_batch_step", m_eager_fp8_output_after_requantise),
+    ("eager_fp8_batch_step", m_eager_fp8_never_requantises),
 ]
 SEQ_MUTATIONS = [
     ("step", m_step_flushes_early),
     ("rollback", m_rollback_keeps_one_less),
     ("verify", m_verify_no_causal_mask),
     ("fold", m_fold_keeps_buffer),
+    ("_output", m_output_reads_copy_at_flush),
 ]
 
 

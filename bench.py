@@ -179,29 +179,48 @@ def measured_hbm_peak():
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def cpu_oracle_rate(shape: gen.Shape, budget_s: float, windows_per_seq: int = 1):
-    """Tokens/s of the CPU oracle (float64, one thread) on sequences of the workload's
-    shape: each sample is one sequence, all heads, `windows_per_seq` windows of L steps
-    (one flush each). Runs whole samples until `budget_s` seconds have passed."""
-    from threadpoolctl import threadpool_limits
-
-    from oracle import replay_oracle as ro
-
+def _oracle_sample_inputs(shape: gen.Shape):
+    """One sequence of the workload (all heads) and the inputs of one oracle sample: one
+    window of L decode steps plus the step that folds it, or, for verify workloads, L
+    verify rounds with their n_keep. Returns (S0 [H,P,N], inputs, keeps or None, tokens)."""
     one = shape.replace(B=1)
-    S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))
-    steps = windows_per_seq * shape.L
-    xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()} for t in range(steps)]
-    tokens, elapsed, samples = 0, 0.0, 0
-    with threadpool_limits(1):
-        while elapsed < budget_s or samples == 0:
-            t0 = time.perf_counter()
-            seq = ro.ReplayBatch(S0, shape.G, shape.L)
-            for x in xs:
-                seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
-            elapsed += time.perf_counter() - t0
-            tokens += steps
-            samples += 1
-    return tokens / elapsed, samples, steps, elapsed
+    S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))[0]
+    if shape.max_pos > 1:
+        xs = [{k: gen.to_numpy64(v) for k, v in gen.verify_inputs(one, t, shape.max_pos, device="cpu").items()}
+              for t in range(shape.L)]
+        keeps = [gen.accepted_lengths(one, t, shape.max_pos, device="cpu").numpy().astype(np.int64) + 1
+                 for t in range(shape.L)]
+        return S0, xs, keeps, int(sum(k.sum() for k in keeps))
+    xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()}
+          for t in range(shape.L)]
+    return S0, xs + xs[:1], None, shape.L + 1
+
+
+def _sample_text(shape: gen.Shape, tokens: int) -> str:
+    if shape.max_pos > 1:
+        return (f"1 sequence x {shape.H} heads x {shape.L} verify rounds of {shape.max_pos} positions "
+                f"({tokens} accepted tokens) of {shape.name}")
+    return f"1 sequence x {shape.H} heads x {shape.L + 1} decode steps (one window and its fold) of {shape.name}"
+
+
+def cpu_oracle_rate(shape: gen.Shape, budget_s: float):
+    """Tokens/s of the CPU oracle (float64 numpy) on sequences of the workload's shape,
+    on all host cores (one process per core, each replaying whole sequences with one
+    BLAS thread; sequences are independent) and on one core, each for about budget_s
+    seconds of wall time. Returns the cpu_baseline record."""
+    from oracle.pool import OraclePool, cpu_model, host_cores
+
+    S0, xs, keeps, tokens = _oracle_sample_inputs(shape)
+    cores = host_cores()
+    with OraclePool(1, S0, xs, keeps, shape.G, shape.L) as pool:
+        s1, t1 = pool.run_for(budget_s / 2)
+    with OraclePool(cores, S0, xs, keeps, shape.G, shape.L) as pool:
+        sn, tn = pool.run_for(budget_s / 2)
+    return {"value": sn * tokens / tn, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"{sn} samples on {cores} processes in {tn:.1f} s, each {_sample_text(shape, tokens)}, "
+                       f"float64 numpy, one BLAS thread per process"),
+            "one_core": {"value": s1 * tokens / t1, "cores": 1, "sample": f"{s1} samples in {t1:.1f} s"},
+            "cpu_model": cpu_model()}
 
 
 # ------------------------------------------------------------------ our arm
@@ -462,10 +481,7 @@ def run_ours(args, rank, world, local):
                                   "cut": bpt["eager_state"] / bpt["replay_state"]},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, samples, steps, secs = cpu_oracle_rate(shape, args.cpu_seconds)
-        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                  "sample": f"{samples} x (1 sequence x {shape.H} heads x {steps} steps) of "
-                                            f"{shape.name}, float64 numpy, {secs:.1f} s"}
+        result["cpu_baseline"] = cpu_oracle_rate(shape, args.cpu_seconds)
     return result
 
 
@@ -572,7 +588,9 @@ def run_spec_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(x0.elapsed_time(x1) / Kx, world, device)
     r.close()
 
+    cpu = cpu_oracle_rate(shape, args.cpu_seconds) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
     return {
+        "cpu_baseline": cpu,
         "metric": SPEC_METRIC,
         "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -597,59 +615,40 @@ def run_spec_ours(args, rank, world, local):
 # ------------------------------------------------------------------ reference arm (the oracle)
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle (there is no reference implementation to
+    install: the reference holds only web pages). Each step, every one of the host's
+    cores (one spawned process each) replays one sample of the workload."""
     if rank != 0:
         return None
     shape = gen.SHAPES[args.workload]
-    from threadpoolctl import threadpool_limits
+    from oracle.pool import OraclePool, cpu_model, host_cores
 
-    from oracle import replay_oracle as ro
-
-    one = shape.replace(B=1)
-    S0 = gen.to_numpy64(gen.initial_state(one, device="cpu"))
-    spec = shape.max_pos > 1
-    if spec:
-        # one step: L verify rounds of max_pos positions, each rolled back to 1 + accepted
-        xs = [{k: gen.to_numpy64(v) for k, v in gen.verify_inputs(one, t, shape.max_pos, device="cpu").items()}
-              for t in range(shape.L)]
-        keeps = [gen.accepted_lengths(one, t, shape.max_pos, device="cpu").numpy().astype(np.int64) + 1
-                 for t in range(shape.L)]
-        step_tokens = int(sum(k.sum() for k in keeps))
-    else:
-        xs = [{k: gen.to_numpy64(v) for k, v in gen.step_inputs(one, t, device="cpu").items()}
-              for t in range(shape.L)]
-        step_tokens = shape.L + 1
-
-    def step():
-        seq = ro.ReplayBatch(S0, shape.G, shape.L)
-        if spec:
-            for x, nk in zip(xs, keeps):
-                seq.verify(x["q"], x["k"], x["v"], x["dt"], x["a"])
-                seq.rollback(nk)
-        else:
-            for x in xs + xs[:1]:  # one window plus the step that folds it
-                seq.step(x["q"], x["k"], x["v"], x["dt"], x["a"])
-
-    with threadpool_limits(1):
+    S0, xs, keeps, tokens = _oracle_sample_inputs(shape)
+    cores = host_cores()
+    with OraclePool(cores, S0, xs, keeps, shape.G, shape.L) as pool:
+        # a step gives every process about half a second of samples (sized in warm-up),
+        # so that handing out the work is a small part of it
+        per = 1
         for _ in range(args.warmup):
-            step()
+            t0 = time.perf_counter()
+            pool.run_each(per)
+            per = max(1, min(1000, round(per * 0.5 / max(time.perf_counter() - t0, 1e-3))))
         t0 = time.perf_counter()
+        samples = 0
         for _ in range(args.steps):
-            step()
+            samples += pool.run_each(per)
         secs = time.perf_counter() - t0
-    tokens = step_tokens * args.steps
-    value = tokens / secs
-    if spec:
-        sample = (f"each step: 1 sequence x {shape.H} heads x {shape.L} verify rounds of {shape.max_pos} positions "
-                  f"({step_tokens} accepted tokens) of {shape.name}")
-    else:
-        sample = f"each step: 1 sequence x {shape.H} heads x {shape.L + 1} decode steps of {shape.name}"
+    value = samples * tokens / secs
+    sample = f"each step: {cores} processes x {per} x ({_sample_text(shape, tokens)})"
+    spec = shape.max_pos > 1
     return {
-        "impl": "reference", "metric": SPEC_METRIC if spec else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True,
+        "impl": "reference", "metric": SPEC_METRIC if spec else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": shape.name, "batch": shape.B, "heads": shape.H, "groups": shape.G, "P": shape.P,
                    "N": shape.N, "L": shape.L, "io": shape.io, "ckpt": shape.ckpt},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -218,16 +218,24 @@ int replay_quantize_rows_e4m3(const float* x, int64_t rows, int32_t n, uint8_t* 
  *  - Limit: B * G * n_pos * N * s bytes (s = 2 for BF16, 4 for FP32) must not exceed
  *    REPLAY_STATIC_SCRATCH_BYTES, else REPLAY_ESCRATCH is returned and nothing is queued.
  *  - 1 <= n_pos <= min(L, 8), even above the context's max_pos. When n_pos > max_pos the
- *    ring (L + max_pos records) has room for n_pos new entries only beside an empty
- *    buffer, so the call first folds every sequence's buffer into its checkpoint, as
- *    replay_flush(ctx, NULL, stream) does: one more state read and write, not reported
- *    in `flushed`.
+ *    ring (cap = L + max_pos records per head) has room for the n_pos new entries only
+ *    where the buffer holds c <= cap - n_pos entries, so the call first folds the
+ *    buffers of the sequences with more (one more launch, which reads and writes only
+ *    their states); the verify then folds the others itself where c + n_pos > L, as
+ *    replay_verify does. `flushed` (if not NULL) reports both folds: 1 where either ran.
+ *    With the FP8 read copy, a pre-folded sequence's outputs are read from its freshly
+ *    re-quantised copy rather than from the fresh master (replay_verify, folding inside
+ *    the verify, reads the master), so they differ from replay_verify's within the FP8
+ *    error; with the FP32 checkpoint the two give the same outputs.
  *  - Allocation: none, on the device or the host. The array is part of the library's
  *    device code, so every GPU that loads libreplay.so holds its 32 MiB until the process
  *    exits.
- *  - Set-up: the first call with n_pos > 1 on a device looks up that device's copy of the
- *    array (cudaGetSymbolAddress); it must run with the context's device current (else
- *    REPLAY_EINVAL), and it should come before any stream capture.
+ *  - Set-up: the first call with n_pos > 1 in a CUDA context (the device's primary
+ *    context, as the runtime uses it) looks up that context's copy of the array
+ *    (cudaGetSymbolAddress) and keeps it for later calls in the same context; after a
+ *    device reset the next call looks it up again. The call must run with the context's
+ *    device current (else REPLAY_EINVAL), and its first call should come before any
+ *    stream capture.
  *  - Sharing: every call on a device, from any context, stream or thread, uses the same
  *    array. Calls whose work overlaps on the GPU race and corrupt each other's queries;
  *    order them (one stream, or events). The array keeps the last call's contents, but

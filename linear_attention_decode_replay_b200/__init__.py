@@ -16,13 +16,16 @@ provides device memory and streams.
 
 Small batches are bound by the host's launch rate; an even number of ``step`` calls on
 fixed input and output tensors can be captured in a CUDA graph once one call has run
-outside the capture (the conditions are in ``include/replay.h``):
+outside the capture (the conditions are in ``include/replay.h``). Each call flips which
+half of the pointer words is current, so capture two windows when L is odd:
 
+    r.step(q[0], k[0], v[0], dt[0], a[0], y=y[0])   # one call outside the capture
+    n = cfg.L if cfg.L % 2 == 0 else 2 * cfg.L      # an even number of calls
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        for t in range(cfg.L):
-            r.step(q[t], k[t], v[t], dt[t], a[t], y=y[t])
-    g.replay()                                 # one window, one graph launch
+        for t in range(n):
+            r.step(q[t % cfg.L], k[t % cfg.L], v[t % cfg.L], dt[t % cfg.L], a[t % cfg.L], y=y[t % cfg.L])
+    g.replay()                                       # n decode steps, one graph launch
 """
 
 from __future__ import annotations
@@ -186,9 +189,9 @@ class Replay:
     def verify_static_scratch(self, q, k, v, dt, a, y=None, flushed=None, stream=None):
         """verify() for callers that cannot allocate device memory: the queries are packed
         into the library's fixed 32 MiB device array instead of the qpack buffer, so the
-        layer needs no qpack (max_pos = 1 works; n_pos above max_pos first folds every
-        buffer). Calls that overlap on the GPU share that array and race. Pass `y` to
-        keep this binding from allocating the output itself."""
+        layer needs no qpack (max_pos = 1 works; n_pos above max_pos first folds the
+        buffers too full to take the new entries). Calls that overlap on the GPU share
+        that array and race. Pass `y` to keep this binding from allocating the output."""
         n_pos = q.shape[1]
         qs, vs, ds = self._token_shapes(n_pos)
         t = self.cfg.io_dtype

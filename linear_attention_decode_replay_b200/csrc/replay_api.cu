@@ -24,6 +24,9 @@ struct replay_ctx {
   int num_sms;
   KParams kp_step, kp_verify, kp_flush;  // prebuilt launch layouts (pointers filled per call)
   int verify_ok;                          // kp_verify was built (max_pos > 1)
+  int smem_optin;                         // the device's per-block shared-memory limit
+  KParams kp_static[replay::kMaxPos + 1]; // replay_verify_static_scratch layouts, by n_pos
+  int kp_static_ok[replay::kMaxPos + 1];  // ... built on first use
 };
 
 namespace {
@@ -299,6 +302,7 @@ int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_str
   ctx->cap = ring_capacity(*cfg);
   ctx->device = d.device;
   ctx->num_sms = d.num_sms;
+  ctx->smem_optin = d.smem_optin;
   replay_config one = *cfg;
   one.max_pos = 1;
   if ((rc = build_layout(&ctx->kp_step, one, replay::kModeReplay, 0, ctx->cap, d.smem_optin)) ||
@@ -306,6 +310,7 @@ int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_str
     delete ctx;
     return rc;
   }
+  ctx->kp_flush.fold_min = 1;  // a flush folds every selected buffer that holds an entry
   if (cfg->max_pos > 1) {
     if ((rc = build_layout(&ctx->kp_verify, *cfg, replay::kModeReplay, 0, ctx->cap, d.smem_optin))) {
       delete ctx;
@@ -472,18 +477,58 @@ namespace {
 
 constexpr int kScratchDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kScratchDevices];  // per device: its copy of replay_static_qpack
+struct ScratchSlot {
+  unsigned long long ctx_id;  // the CUDA context the address belongs to (0: none yet)
+  void* addr;                 // that context's copy of replay_static_qpack
+};
+ScratchSlot g_scratch[kScratchDevices];
 
-// Set-up, once per device, with that device current: its address of the scratch array.
+// The unique id of the calling thread's current CUDA context, 0 if it cannot be had.
+// The driver calls are looked up through the runtime, so the library needs no link to
+// the driver library.
+unsigned long long current_context_id() {
+  typedef int (*GetCurrentFn)(void**);
+  typedef int (*GetIdFn)(void*, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {  // under g_scratch_mu
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess && q2 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(f1);
+      get_id = reinterpret_cast<GetIdFn>(f2);
+    }
+    looked_up = true;
+  }
+  if (!get_current || !get_id) return 0;
+  void* cu_ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&cu_ctx) != 0 || !cu_ctx || get_id(cu_ctx, &id) != 0) return 0;
+  return id;
+}
+
+// Set-up, once per device and CUDA context, with that device current: the context's
+// address of the scratch array. A device reset ends the context that held the array; the
+// next call sees a new context id and looks the address up again. Where the id cannot be
+// had, the address is looked up on every call.
 int static_scratch_address(int device, void** out) {
   if (device < 0 || device >= kScratchDevices) return REPLAY_EINVAL;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[device]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress((void**)&ptr, replay_static_qpack) != cudaSuccess || !ptr) return REPLAY_ECUDA;
-    g_scratch_addr[device] = ptr;
+  ScratchSlot& slot = g_scratch[device];
+  const unsigned long long id = current_context_id();
+  if (id != 0 && slot.addr && slot.ctx_id == id) {
+    *out = slot.addr;
+    return REPLAY_OK;
   }
-  *out = g_scratch_addr[device];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress((void**)&ptr, replay_static_qpack) != cudaSuccess || !ptr) return REPLAY_ECUDA;
+  slot.ctx_id = current_context_id();  // the lookup above made the context current if it was not
+  slot.addr = ptr;
+  *out = ptr;
   return REPLAY_OK;
 }
 
@@ -508,24 +553,38 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
     if (rc == REPLAY_OK) ctx->pending = 1;
     return rc;
   }
-  DeviceInfo d;
-  if ((rc = device_info(&d))) return rc;
-  if (d.device != ctx->device) return REPLAY_EINVAL;
+  int device = -1;
+  if (cudaGetDevice(&device) != cudaSuccess) return REPLAY_ECUDA;
+  if (device != ctx->device) return REPLAY_EINVAL;
   void* scratch = nullptr;
-  if ((rc = static_scratch_address(d.device, &scratch))) return rc;
-  replay_config c = cfg;
-  c.max_pos = n_pos;
-  KParams p;
-  if ((rc = build_layout(&p, c, replay::kModeReplay, 0, ctx->cap, d.smem_optin))) return rc;
-  if (cfg.max_pos < n_pos) {
-    // a ring of L + max_pos records holds n_pos new entries only beside an empty buffer
-    if ((rc = replay_flush(ctx, nullptr, stream))) return rc;
+  if ((rc = static_scratch_address(device, &scratch))) return rc;
+  if (!ctx->kp_static_ok[n_pos]) {
+    replay_config c = cfg;
+    c.max_pos = n_pos;
+    if ((rc = build_layout(&ctx->kp_static[n_pos], c, replay::kModeReplay, 0, ctx->cap, ctx->smem_optin))) return rc;
+    ctx->kp_static_ok[n_pos] = 1;
+  }
+  KParams p = ctx->kp_static[n_pos];
+  const int ckpt = cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
+  const bool prefold = cfg.max_pos < n_pos;
+  if (prefold) {
+    // The ring holds cap = L + max_pos records per head, so a buffer of c entries has room
+    // for the n_pos new ones only while c <= cap - n_pos: fold just the fuller buffers
+    // first (the verify folds the others itself when c + n_pos > L). The flush writes
+    // `flushed` for every sequence; the verify then ORs its own folds into it.
+    KParams f = ctx->kp_flush;
+    set_state(&f, ctx);
+    f.flushed = flushed;
+    f.fold_min = ctx->cap - n_pos + 1;
+    if (launch_main(f, cfg, ckpt, replay::kModeFlush, 0, ctx->num_sms, s) != cudaSuccess) return REPLAY_ECUDA;
+    ctx->parity ^= 1;
   }
   set_state(&p, ctx);
   p.qpack = scratch;
   p.qpack_pos = n_pos;
   p.n_pos = n_pos;
   p.commit = 0;
+  p.flushed_or = prefold ? 1 : 0;
   p.q = q;
   p.k = k;
   p.v = v;
@@ -558,7 +617,6 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
   const long long blocks = (tasks + 7) / 8;
   const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
   if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
-  const int ckpt = cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
   if (launch_main(p, cfg, ckpt, replay::kModeReplay, n_pos, ctx->num_sms, s) != cudaSuccess)
     return REPLAY_ECUDA;
   ctx->parity ^= 1;

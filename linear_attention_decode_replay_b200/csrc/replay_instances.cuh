@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "replay_kernel.cuh"
 #include "replay_launch.h"
 
@@ -20,14 +22,20 @@ cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
   constexpr int NG = kGroups;  // consumer groups (the host layout reserves one workspace per group)
   auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ, NG>;
   // the dynamic shared-memory opt-in is per function and device; remember the largest set
+  // (under a lock: calls may come from several threads, and a smaller concurrent setting
+  // must not lower the limit below what another launch needs)
   static int configured[kMaxDevices] = {0};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices || configured[dev] < p.smem_bytes) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices) configured[dev] = p.smem_bytes;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= kMaxDevices || configured[dev] < p.smem_bytes) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < kMaxDevices) configured[dev] = p.smem_bytes;
+    }
   }
   kern<<<grid, kThreads, p.smem_bytes, s>>>(p);
   return cudaGetLastError();

@@ -103,7 +103,7 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
     pl.fold = pl.c + p.n_pos > p.L;
     pl.active = true;
   } else {
-    pl.fold = msk != 0 && pl.c > 0;
+    pl.fold = msk != 0 && pl.c > 0 && pl.c >= p.fold_min;
     pl.active = pl.fold;
   }
   pl.fp32_tile = (CKPT == kCkptF32) || pl.fold;
@@ -861,7 +861,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
       const int base = fold ? 0 : c;
       const int cnt2 = base + (p.commit ? n : 0);
       p.counts_out[pl.b] = (start2 << 16) | cnt2;
-      if (p.flushed) p.flushed[pl.b] = fold ? 1 : 0;
+      if (p.flushed && (!p.flushed_or || fold)) p.flushed[pl.b] = fold ? 1 : 0;
     }
   } else if (MODE == kModeFlush) {
     if (pl.h == 0 && pl.rb == 0 && gtid == 0) {

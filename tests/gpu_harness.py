@@ -49,6 +49,9 @@ class Report:
     fro_err: float = 0.0          # max over steps of ||Y - Y_ref||_F / ||Y_ref||_F (sampled batch)
     shared_fro_err: float = 0.0   # same for the shared-FP8 eager kernel
     per_vector: list = field(default_factory=list)  # every per-(sequence, head) error
+    shared_per_vector: list = field(default_factory=list)  # the same for the shared-FP8 eager kernel
+    per_step_fro: list = field(default_factory=list)
+    shared_per_step_fro: list = field(default_factory=list)
 
 
 def frobenius_error(y, y_ref) -> float:
@@ -92,9 +95,11 @@ def run_decode(shape: gen.Shape, steps: int, rows, flush_at_end=True, fp8_emulat
         e = ro.relative_error(y_gpu, y_ref)
         rep.per_step.append(e)
         rep.max_err = max(rep.max_err, e)
-        rep.fro_err = max(rep.fro_err, frobenius_error(y_gpu, y_ref))
+        fro = frobenius_error(y_gpu, y_ref)
+        rep.fro_err = max(rep.fro_err, fro)
         if shared_fp8:
             rep.per_vector.append(vector_errors(y_gpu, y_ref))
+            rep.per_step_fro.append(fro)
         if emu is not None:
             y_emu, _ = emu.step(xs["q"], xs["k"], xs["v"], xs["dt"], xs["a"])
             rep.max_err_fp8_emul = max(rep.max_err_fp8_emul, ro.relative_error(y_gpu, y_emu))
@@ -102,7 +107,10 @@ def run_decode(shape: gen.Shape, steps: int, rows, flush_at_end=True, fp8_emulat
             y_sh = lar.eager_step_fp8(cfg, codes_d, scale_d, x["q"], x["k"], x["v"], x["dt"], x["a"])
             y_sh_np = _np(y_sh, rows)
             rep.max_err_shared_fp8 = max(rep.max_err_shared_fp8, ro.relative_error(y_sh_np, y_ref))
-            rep.shared_fro_err = max(rep.shared_fro_err, frobenius_error(y_sh_np, y_ref))
+            sh_fro = frobenius_error(y_sh_np, y_ref)
+            rep.shared_fro_err = max(rep.shared_fro_err, sh_fro)
+            rep.shared_per_step_fro.append(sh_fro)
+            rep.shared_per_vector.append(vector_errors(y_sh_np, y_ref))
         f_gpu = fl.cpu().numpy()
         all_flags.append(f_gpu.copy())
         if not np.array_equal(f_gpu[rows], f_ref):

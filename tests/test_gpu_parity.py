@@ -1,6 +1,9 @@
 """CUDA path (through the C ABI) against the CPU oracle, element by element on the same
 seeded inputs: small shapes in full, the full-size workloads on sampled sequences."""
 
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -249,26 +252,43 @@ def test_mamba2_b256_decode_sampled():
     assert rep.max_err <= hx.TOL_BF16
 
 
+def _error_summary(per_vector, per_step_fro):
+    errs = np.concatenate(per_vector)
+    fro = np.asarray(per_step_fro)
+    return {"per_vector_median": float(np.median(errs)), "per_vector_p99": float(np.quantile(errs, 0.99)),
+            "per_vector_max": float(errs.max()), "per_step_frobenius_median": float(np.median(fro)),
+            "per_step_frobenius_max": float(fro.max()), "per_step_frobenius_last": float(fro[-1])}
+
+
 def test_mamba2_b256_fp8_sampled():
-    """Dual precision at full size over 2048 steps. Parity: the FP8-read path against the
-    oracle's emulation of the same FP8-read method, within the 6e-2 bar (measured ~5e-3;
-    the FP32 and FP64 masters can round a row to neighbouring codes). Reported beside it,
-    the method's own output error against the unquantised oracle and that of the
-    shared-FP8 eager kernel: the dual-precision error stays bounded (per-step Frobenius
-    error under the 6e-2 bar, the master exact) while the shared-FP8 state drifts."""
+    """Dual precision at full size over 2048 steps, six sampled sequences. Parity: the
+    FP8-read path against the oracle's emulation of the same FP8-read method, per output
+    vector, within 1e-2 (the FP32 and FP64 masters can round a row to neighbouring codes).
+    The method's own error against the unquantised FP32 oracle is held to the 6e-2 bar as
+    a per-step Frobenius error (a per-vector relative error against FP32 has no bound for
+    any FP8 copy: an output vector with a small norm still carries the copy's absolute
+    error). Beside it, the shared-FP8 eager kernel on the same inputs: its error grows,
+    the dual-precision error does not, and the master stays exact. With REPLAY_REPORT_DIR
+    set, the figures are written to fp8_error_mamba2_b256.json there."""
     shape = gen.SHAPES["mamba2_b256_fp8"]
-    rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 3), fp8_emulation=True,
-                        shared_fp8=True)
+    rows = hx.sample_rows(shape.B, 6)
+    rep = hx.run_decode(shape, shape.steps, rows, fp8_emulation=True, shared_fp8=True)
     assert rep.max_err_fp8_emul <= hx.TOL_FP8 and rep.max_err_fp8_emul <= 1e-2, rep.max_err_fp8_emul
     assert rep.fro_err <= hx.TOL_FP8, rep.fro_err
     assert rep.flags_equal and rep.counts_equal
     assert rep.ckpt_err <= hx.TOL_F32  # the master never sees FP8 rounding
     assert rep.shared_fro_err > rep.fro_err  # shared low precision compounds, dual does not
-    errs = np.concatenate(rep.per_vector)
-    print(f"fp8 read vs emulation {rep.max_err_fp8_emul:.3e}; vs FP32 oracle: per-step Frobenius "
-          f"{rep.fro_err:.3e}, per-vector median {np.median(errs):.3e} p99 {np.quantile(errs, 0.99):.3e} "
-          f"max {rep.max_err:.3e}; shared-FP8 eager: Frobenius {rep.shared_fro_err:.3e} max "
-          f"{rep.max_err_shared_fp8:.3e}")
+    report = {"workload": shape.name, "steps": shape.steps, "sampled_sequences": [int(r) for r in rows],
+              "dual_precision_vs_fp8_emulation_max": rep.max_err_fp8_emul,
+              "dual_precision_vs_fp32_oracle": _error_summary(rep.per_vector, rep.per_step_fro),
+              "shared_fp8_eager_vs_fp32_oracle": _error_summary(rep.shared_per_vector, rep.shared_per_step_fro),
+              "master_checkpoint_vs_fp32_oracle": rep.ckpt_err}
+    print(json.dumps(report))
+    out_dir = os.environ.get("REPLAY_REPORT_DIR")
+    if out_dir:
+        os.makedirs(out_dir, exist_ok=True)
+        with open(os.path.join(out_dir, "fp8_error_mamba2_b256.json"), "w") as f:
+            json.dump(report, f, indent=1)
 
 
 def test_mamba2_b256_spec_sampled():

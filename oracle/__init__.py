@@ -15,7 +15,10 @@ from .replay_oracle import (  # noqa: F401
     ReplayBatch,
     ReplaySeq,
     decay_weights,
+    dequantize_rows_e2m1,
     dequantize_rows_e4m3,
+    e2m1_decode,
+    e2m1_encode,
     e4m3_decode,
     e4m3_encode,
     eager_batch_step,
@@ -23,6 +26,7 @@ from .replay_oracle import (  # noqa: F401
     eager_step,
     history_state,
     output_only,
+    quantize_rows_e2m1,
     quantize_rows_e4m3,
     relative_error,
     route_flops,

@@ -176,6 +176,63 @@ def dequantize_rows_e4m3(codes, scale):
 
 
 # --------------------------------------------------------------------------------------
+# FP4 e2m1 (OCP Microscaling formats, FP4 E2M1 element) -- the 4-bit read copy
+# --------------------------------------------------------------------------------------
+
+E2M1_MAX = 6.0
+
+
+def e2m1_decode(codes):
+    """Value of each 4-bit e2m1 code: sign bit, 2 exponent bits (bias 1), 1 mantissa bit.
+    Exponent field 0 is subnormal (M * 0.5); every code is finite (largest 6)."""
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    E = (c >> 1) & 0x3
+    M = c & 0x1
+    mag = np.where(E == 0, M * 0.5, (1.0 + M / 2.0) * np.exp2(E - 1.0))
+    return sign * mag
+
+
+def e2m1_encode(x):
+    """Round each value to the nearest e2m1 value (ties to the even mantissa), saturating
+    beyond +-6. Returns 4-bit codes (uint8, one per value)."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.signbit(x).astype(np.int64) << 3
+    mag = np.minimum(np.abs(x), E2M1_MAX)
+    # spacing of representable values in the binade of mag: 2^(e-1) for mag in [2^e, 2^(e+1)),
+    # held at 0.5 below 1 (subnormal spacing)
+    _, e = np.frexp(mag)
+    e = np.maximum(e - 1, 0)
+    quantum = np.exp2(e - 1.0)
+    val = np.rint(mag / quantum) * quantum  # half to even on the mantissa bit
+    f2, e2 = np.frexp(val)
+    normal = val >= 1.0
+    E = np.where(normal, e2, 0)  # val = 2^(E-1) * (1 + M/2): E = e2 for val in [2^(e2-1), 2^e2)
+    M = np.where(normal, (2.0 * f2 - 1.0) * 2.0, val / 0.5)
+    return (sign | (E.astype(np.int64) << 1) | M.astype(np.int64)).astype(np.uint8)
+
+
+def quantize_rows_e2m1(S):
+    """Per-row FP4 read copy, the FP8 copy's recipe with the e2m1 range: scale = amax / 6
+    in FP32 (1 for an all-zero row), codes = e2m1(x * (6 / amax)) with the product rounded
+    to FP32 first. Returns (codes uint8 [..., N], one 4-bit code per value; scale float32
+    [...])."""
+    x = np.asarray(S).astype(np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    zero = amax == 0
+    safe = np.where(zero, np.float32(1), amax).astype(np.float32)
+    scale = np.where(zero, np.float32(1), safe / np.float32(E2M1_MAX)).astype(np.float32)
+    inv = np.where(zero, np.float32(1), np.float32(E2M1_MAX) / safe).astype(np.float32)
+    codes = e2m1_encode((x * inv[..., None]).astype(np.float32))
+    return codes, scale
+
+
+def dequantize_rows_e2m1(codes, scale):
+    """FP4 read copy back to values: e2m1 value times its row's scale."""
+    return e2m1_decode(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+# --------------------------------------------------------------------------------------
 # One sequence with a checkpoint and a buffer (blog, "Decodificacion estandar",
 # "Rollback", "Paralelismo"; arXiv abstract)
 # --------------------------------------------------------------------------------------
@@ -186,6 +243,7 @@ class ReplaySeq:
     ckpt="f32":          every output reads the master S0.
     ckpt="f32_fp8read":  outputs read an e4m3 copy of S0 (per-row scale); the flush
                          updates the master and re-quantises the copy.
+    ckpt="f32_fp4read":  the same with an e2m1 copy (video takeaways: FP8/FP4).
     Counters: state_reads / state_writes count full passes over the per-head state."""
 
     def __init__(self, S0, G, L, ckpt="f32"):
@@ -201,8 +259,14 @@ class ReplaySeq:
         self.state_reads = 0
         self.state_writes = 0
         self._read_copy = None  # dequantised FP8 copy, kept until the next flush
-        if ckpt == "f32_fp8read":
-            self.codes, self.scale = quantize_rows_e4m3(self.S0)
+        if ckpt not in ("f32", "f32_fp8read", "f32_fp4read"):
+            raise ValueError(f"unknown checkpoint kind {ckpt}")
+        self._quantize, self._dequantize = {
+            "f32_fp8read": (quantize_rows_e4m3, dequantize_rows_e4m3),
+            "f32_fp4read": (quantize_rows_e2m1, dequantize_rows_e2m1),
+        }.get(ckpt, (None, None))
+        if self._quantize is not None:
+            self.codes, self.scale = self._quantize(self.S0)
 
     @property
     def count(self):
@@ -230,8 +294,8 @@ class ReplaySeq:
             ab, db, vb, kb = self._buffer(c)
             abar, s = decay_weights(ab, db)
             self.S0 = state_route(self.S0, abar, s, vb, kb)
-            if self.ckpt == "f32_fp8read":
-                self.codes, self.scale = quantize_rows_e4m3(self.S0)
+            if self._quantize is not None:
+                self.codes, self.scale = self._quantize(self.S0)
                 self._read_copy = None
             self.state_reads += 1
             self.state_writes += 1
@@ -245,7 +309,7 @@ class ReplaySeq:
             S_read = self.S0
         else:
             if self._read_copy is None:
-                self._read_copy = dequantize_rows_e4m3(self.codes, self.scale)
+                self._read_copy = self._dequantize(self.codes, self.scale)
             S_read = self._read_copy
         return output_only(S_read, abar, s, vb, kb, np.asarray(q, np.float64)[self.group_of_head])
 

@@ -457,6 +457,72 @@ def pin_dual_precision_hand_example():
     assert abs(y1.ravel()[0] - fx["B_y1"][0]) < 1e-12, y1
 
 
+def pin_dual_precision_fp4_hand_example():
+    """The same split with the FP4 e2m1 copy (fixture, example C): codes worked by hand,
+    the copy read by a step without a flush, the master by the flushing step."""
+    codes, fx = _fp8_fixture()
+    seq = ro.ReplaySeq(fx["C_S0"].reshape(1, 1, 4), G=1, L=1, ckpt="f32_fp4read")
+    assert np.array_equal(seq.codes.ravel(), codes["C_codes"]) and seq.scale.ravel()[0] == 1.0
+    q = fx["C_q"].reshape(1, 4)
+    zero_k, zero_v, one, zero = np.zeros((1, 4)), np.zeros((1, 1)), np.ones(1), np.zeros(1)
+    y0, f0 = seq.step(q, zero_k, zero_v, zero, one)
+    y1, f1 = seq.step(q, zero_k, zero_v, zero, one)
+    assert not f0 and f1
+    assert y0.ravel()[0] == fx["C_y0"][0], y0
+    assert abs(y1.ravel()[0] - fx["C_y1"][0]) < 1e-12, y1
+
+
+def pin_e2m1_table():
+    """Every e2m1 code decodes to the OCP MX table value (golden fixture) and encodes
+    back to itself (the two zeros to themselves)."""
+    rows = _read_fixture("e2m1_table.txt")
+    assert len(rows) == 16
+    for code, val in rows.items():
+        c = int(code, 16)
+        got = ro.e2m1_decode(np.array([c], dtype=np.uint8))[0]
+        assert got == float(val[0]) and math.copysign(1, got) == math.copysign(1, float(val[0])), code
+        assert ro.e2m1_encode(np.array([float(val[0])]))[0] == c, code
+
+
+def pin_e2m1_nearest_by_brute_force():
+    """Encoding = the nearest of the 16 table values by exhaustive search (ties to the
+    code with the even mantissa bit, beyond +-6 to +-6), over a dense sweep with every
+    midpoint and its neighbours."""
+    table = {int(k, 16): float(v[0]) for k, v in _read_fixture("e2m1_table.txt").items()}
+    pos = sorted((v, c) for c, v in table.items() if c < 8)
+    mids = [(pos[i][0] + pos[i + 1][0]) / 2 for i in range(7)]
+    rng = _rng(15)
+    x = np.concatenate([rng.uniform(-8, 8, 4000), np.array(mids), -np.array(mids), np.nextafter(mids, 0),
+                        np.nextafter(mids, 10), [6.0, 6.5, 7.9, 100.0, -7.0, 0.0]])
+
+    def brute(xi):
+        m = min(abs(xi), 6.0)
+        best = min(pos, key=lambda vc: (abs(vc[0] - m), vc[1] & 1))  # nearest, then even mantissa
+        return best[1] | (8 if math.copysign(1, xi) < 0 else 0)
+
+    want = np.array([brute(xi) for xi in x], dtype=np.uint8)
+    assert np.array_equal(ro.e2m1_encode(x), want), np.flatnonzero(ro.e2m1_encode(x) != want)[:5]
+
+
+def pin_row_quantiser_e2m1():
+    """Per-row FP4 scale: the row's largest magnitude maps to 6 (code 0x7); an all-zero
+    row has scale 1 and zero codes; dequantised values lie within half a code spacing."""
+    rng = _rng(16)
+    S = rng.standard_normal((5, 32)) * np.array([[1e-3], [1.0], [30.0], [0.0], [2.5]])
+    codes, scale = ro.quantize_rows_e2m1(S)
+    assert scale.dtype == np.float32 and codes.dtype == np.uint8 and codes.max() <= 0xF
+    assert np.all((codes[3] & 0x7) == 0) and scale[3] == 1.0
+    for r in (0, 1, 2, 4):
+        amax = np.max(np.abs(S[r].astype(np.float32)))
+        assert scale[r] == np.float32(amax) / np.float32(6)
+        assert (codes[r] & 0x7).max() == 0x7
+    deq = ro.dequantize_rows_e2m1(codes, scale)
+    x = S.astype(np.float32).astype(np.float64)
+    # normal range (|x| >= scale): relative error <= 2^-2; below it: absolute <= 0.25 * scale
+    bound = np.maximum(np.abs(x) * 0.25, 0.25 * scale[:, None]) * (1 + 1e-6)
+    assert np.all(np.abs(deq - x) <= bound)
+
+
 def pin_relative_error_metric():
     """The error metric is the max over vectors of the relative L2 error."""
     y_ref = np.array([[3.0, 4.0], [0.0, 1.0]])

@@ -157,6 +157,38 @@ def m_eager_fp8_never_requantises(codes, scale, q, k, v, dt, a, G):
     return codes, scale, y
 
 
+def m_e2m1_round_half_up(x):
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.signbit(x).astype(np.int64) << 3
+    mag = np.minimum(np.abs(x), 6.0)
+    _, e = np.frexp(mag)
+    quantum = np.exp2(np.maximum(e - 1, 0) - 1.0)
+    val = np.floor(mag / quantum + 0.5) * quantum
+    f2, e2 = np.frexp(val)
+    normal = val >= 1.0
+    E = np.where(normal, e2, 0)
+    M = np.where(normal, (2.0 * f2 - 1.0) * 2.0, val / 0.5)
+    return (sign | (E.astype(np.int64) << 1) | np.minimum(M, 1).astype(np.int64)).astype(np.uint8)
+
+
+def m_e2m1_decode_bias2(codes):
+    return _orig["e2m1_decode"](codes) / 2.0
+
+
+def m_quantize_e2m1_scale_4(S):
+    x = np.asarray(S).astype(np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    safe = np.where(amax == 0, np.float32(1), amax).astype(np.float32)
+    scale = np.where(amax == 0, np.float32(1), safe / np.float32(4)).astype(np.float32)
+    inv = np.where(amax == 0, np.float32(1), np.float32(4) / safe).astype(np.float32)
+    return _orig["e2m1_encode"]((x * inv[..., None]).astype(np.float32)), scale
+
+
+def m_e2m1_no_saturation(x):
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(np.abs(x) > 6.0, 0, _orig["e2m1_encode"](x)).astype(np.uint8)
+
+
 def m_route_flops_counts_outer_twice(P, N, entries):
     f = _orig["route_flops"](P, N, entries)
     return {"outer": 2 * f["outer"], "inner": f["inner"]}
@@ -182,6 +214,10 @@ MODULE_MUTATIONS = [
     ("route_flops", m_route_flops_counts_outer_twice),
     ("eager_fp8_batch_step", m_eager_fp8_output_after_requantise),
     ("eager_fp8_batch_step", m_eager_fp8_never_requantises),
+    ("e2m1_encode", m_e2m1_round_half_up),
+    ("e2m1_encode", m_e2m1_no_saturation),
+    ("e2m1_decode", m_e2m1_decode_bias2),
+    ("quantize_rows_e2m1", m_quantize_e2m1_scale_4),
 ]
 SEQ_MUTATIONS = [
     ("step", m_step_flushes_early),

@@ -66,7 +66,9 @@ def kernel_sources_hash() -> str:
 def algorithmic_bytes_per_token(s: gen.Shape) -> dict:
     """Bytes a decoded token must move, per sequence (steady state, lazy flush once per
     window of L tokens):
-      replay: state (L+1)/L * H*P*N*4 (L-1 output-only reads + one fused read+write),
+      replay: state (L+1)/L * H*P*N*4 (L-1 output-only reads + one fused read+write; with
+              a read copy, L-1 reads of the codes and scales, and the fold reads and writes
+              the master and writes the copy),
               buffer re-reads (L+1)/2 * E, new inputs q + E, entry write E, output 4*H*P,
               with E = G*N*s + H*P*s + 8*H (one entry: k, v, Delta, a);
       eager:  state 2 * H*P*N*4 (read + write), inputs q + E, output 4*H*P."""
@@ -75,8 +77,9 @@ def algorithmic_bytes_per_token(s: gen.Shape) -> dict:
     q = s.G * s.N * sio
     y = 4 * s.H * s.P
     state = s.H * s.P * s.N * 4
-    if s.ckpt == "f32_fp8read":
-        copy = s.H * s.P * (s.N + 4)  # e4m3 codes + per-row scales
+    if s.ckpt in ("f32_fp8read", "f32_fp4read"):
+        code_bytes = s.N if s.ckpt == "f32_fp8read" else s.N // 2
+        copy = s.H * s.P * (code_bytes + 4)  # e4m3 or e2m1 codes + per-row scales
         replay_state = ((s.L - 1) * copy + 2 * state + copy) / s.L
     else:
         replay_state = (s.L + 1) / s.L * state

@@ -67,16 +67,20 @@ typedef enum {
 typedef enum { REPLAY_F32 = 0, REPLAY_BF16 = 1 } replay_dtype;
 
 typedef enum {
-  REPLAY_CKPT_F32 = 0,         /* outputs and flushes use the FP32 checkpoint */
-  REPLAY_CKPT_F32_FP8READ = 1  /* outputs read an FP8 e4m3 copy; flushes update the FP32
-                                  master and re-quantise the copy (abstract: separate
-                                  state precisions; video takeaways: dual precision) */
+  REPLAY_CKPT_F32 = 0,          /* outputs and flushes use the FP32 checkpoint */
+  REPLAY_CKPT_F32_FP8READ = 1,  /* outputs read an FP8 e4m3 copy; flushes update the FP32
+                                   master and re-quantise the copy (abstract: separate
+                                   state precisions; video takeaways: dual precision) */
+  REPLAY_CKPT_F32_FP4READ = 2   /* the same with an FP4 e2m1 copy (video takeaways: FP8/FP4):
+                                   one FP32 scale per row, scale = amax/6 */
 } replay_ckpt;
 
 /* Device-detected error bits OR-ed into the status word. */
 #define REPLAY_DEV_WAIT_TIMEOUT 1 /* a pipeline wait gave up after ~2 s (results invalid) */
 #define REPLAY_DEV_POINTER 2      /* a buffer pointer word was out of range */
 #define REPLAY_DEV_ROLLBACK 4     /* n_keep outside [0, n_pos]; that sequence kept none */
+#define REPLAY_DEV_SNAPSHOT 8     /* replay_import: a snapshot or sequence id did not match
+                                     the layer; that snapshot was skipped */
 
 typedef struct {
   int32_t batch;   /* B >= 1 */
@@ -93,15 +97,20 @@ typedef struct {
 /* Caller-owned device buffers of one decode layer. All 16-byte aligned except counts and
  * status (4-byte). P*N*4 bytes per head must not exceed 65536.
  *
- * The buffer of recent inputs is a ring of `cap` records per (sequence, head); record j
- * holds one buffered input as R bytes: k (N io values), v (P io values), Delta (FP32),
- * a (FP32), zero padding to a multiple of 16 bytes. Keeping an entry's pieces together
- * lets a unit's whole buffer arrive in one or two bulk copies. */
+ * The buffer of recent inputs is a ring of `cap` records per sequence: one k record per
+ * k/q group and one record per head. A group's heads share its k (blog, end of "Ruta
+ * 'solo salida'": k and q belong to the group), so k is stored once per group. k record
+ * j of (b, g): RK bytes, k (N io values). Head record j of (b, h): R bytes, v (P io values),
+ * Delta (FP32), a (FP32), zero padding to a multiple of 16 bytes. Keeping an entry's pieces
+ * together lets a unit's whole buffer arrive in one or two bulk copies per ring. */
 typedef struct {
   float* S0;         /* [B][H][P][N] FP32 checkpoint (master); row p of N floats contiguous */
-  uint8_t* S0_fp8;   /* [B][H][P][N] e4m3 read copy (ckpt = REPLAY_CKPT_F32_FP8READ, else NULL) */
+  uint8_t* S0_codes; /* the read copy's codes: FP8 [B][H][P][N] bytes; FP4 [B][H][P][N/2] bytes,
+                        element 2i of a row in the low nibble of byte i, 2i+1 in the high
+                        nibble; NULL for REPLAY_CKPT_F32 */
   float* S0_scale;   /* [B][H][P] FP32 per-row scale of the copy (same condition) */
-  void* ring;        /* [B][H][cap] records of R bytes (see above) */
+  void* ring_k;      /* [B][G][cap] k records of RK bytes */
+  void* ring;        /* [B][H][cap] head records of R bytes (v, Delta, a) */
   void* qpack;       /* [B][G][max_pos][N] io scratch for verify queries (max_pos > 1, else NULL) */
   int32_t* counts;   /* [2][B] buffer pointer words, double-buffered (the library alternates
                         halves each call so that no launch reads what it writes) */
@@ -110,18 +119,25 @@ typedef struct {
 
 typedef struct replay_ctx replay_ctx;
 
-/* Records the ring holds per (sequence, head): L + max_pos. A flush and the appends of
- * the same call touch disjoint records. Returns a negative replay_status on a bad config. */
+/* Records the ring holds per (sequence, group) and per (sequence, head): L + max_pos. A
+ * flush and the appends of the same call touch disjoint records. Returns a negative
+ * replay_status on a bad config. */
 int32_t replay_ring_capacity(const replay_config* cfg);
 
-/* Bytes of one ring record: N*s + P*s + 8 rounded up to a multiple of 16, s = 2 (BF16) or
- * 4 (FP32). Returns a negative replay_status on a bad config. */
+/* Bytes of one head record: P*s + 8 rounded up to a multiple of 16, s = 2 (BF16) or 4
+ * (FP32). Returns a negative replay_status on a bad config. */
 int32_t replay_ring_record_bytes(const replay_config* cfg);
 
+/* Bytes of one k record: N*s (a multiple of 16). Returns a negative replay_status on a
+ * bad config. */
+int32_t replay_ring_k_record_bytes(const replay_config* cfg);
+
 /* Validates cfg and bufs, zeroes both halves of counts (every buffer empty) and the
- * status word, and for REPLAY_CKPT_F32_FP8READ fills S0_fp8 / S0_scale from S0 (per-row
- * e4m3, scale = amax/448). S0 must already hold the initial checkpoint. On success
- * *out receives a context owned by the caller (free with replay_destroy). */
+ * status word, and with a read copy fills S0_codes / S0_scale from S0 (per-row e4m3 with
+ * scale = amax/448, or e2m1 with scale = amax/6). S0 must already hold the initial
+ * checkpoint. On success *out receives a context owned by the caller (free with
+ * replay_destroy). REPLAY_EINVAL also when two pipeline stages of one unit do not fit in
+ * shared memory (only the largest P, L and max_pos together with FP32 inputs). */
 int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_stream_t stream,
                 replay_ctx** out);
 
@@ -152,6 +168,38 @@ int replay_verify(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k, 
                   const float* dt, const float* a, float* y, uint8_t* flushed,
                   replay_stream_t stream);
 
+/* ---- Zero-copy appends: the caller writes the entries straight into the ring ----
+ * The buffer holds the raw inputs of the recent tokens (blog "Decodificacion estandar";
+ * video takeaways: a ring buffer of the last L inputs). A caller whose projection kernel
+ * produces k, v, Delta and a can write them directly into their ring records instead of
+ * into separate input tensors that replay_step then copies: ask for the slots, write
+ * the records, then call the resident variant, which reads the entries from the ring.
+ *
+ * replay_append_slots writes, for every sequence b, the ring record of its next entry:
+ *   slots[b] = (start + count) mod cap   (device int32 [B], written on the stream),
+ * from the current buffer pointer word. The entry of position s (0 for a step, 0..n_pos-1
+ * for a verify) of sequence b goes to record (slots[b] + s) mod cap: its k into
+ * ring_k[b][g] for every group g, its v, Delta and a into ring[b][h] for every head h
+ * (layouts: see replay_buffers). slots[b] is -1 (and REPLAY_DEV_POINTER is set) for a
+ * pointer word out of
+ * range. The slots stay valid until the next step, verify, rollback or flush; a call
+ * that folds reads records [start, start + count) and appends after them, so writing the
+ * new records before that call never overwrites a buffered entry. Returns
+ * REPLAY_EPENDING while a verify awaits its rollback. */
+int replay_append_slots(replay_ctx* ctx, int32_t* slots, replay_stream_t stream);
+
+/* replay_step whose entry is already in the ring (written at replay_append_slots' record
+ * on this stream, or ordered before this call): only the query is passed.
+ *   q: device [B][G][N] io   y: device [B][H][P] FP32   flushed: device [B] uint8 or NULL */
+int replay_step_resident(replay_ctx* ctx, const void* q, float* y, uint8_t* flushed,
+                         replay_stream_t stream);
+
+/* replay_verify whose n_pos entries are already in the ring (records slots[b] + s mod
+ * cap); only the queries are passed. Must be followed by replay_rollback.
+ *   q: device [B][n_pos][G][N] io   y: device [B][n_pos][H][P] FP32   flushed: [B] or NULL */
+int replay_verify_resident(replay_ctx* ctx, int32_t n_pos, const void* q, float* y, uint8_t* flushed,
+                           replay_stream_t stream);
+
 /* Resolves the pending verify (blog "Rollback (deshacer)"; video takeaways: rollback is a
  * pointer move): sequence b keeps the first n_keep[b] of the n_pos tentative entries
  * (device int32 [B], values in [0, n_pos]); the rest are dropped by moving the buffer end
@@ -162,6 +210,44 @@ int replay_rollback(replay_ctx* ctx, const int32_t* n_keep, replay_stream_t stre
 /* Folds the buffer of every sequence with mask[b] != 0 (device uint8 [B]; NULL = all)
  * into the checkpoint (state route) and empties it; also refreshes the FP8 copy. */
 int replay_flush(replay_ctx* ctx, const uint8_t* mask, replay_stream_t stream);
+
+/* ---- Snapshots of single sequences (export / import) ----
+ * A sequence's decode state is its checkpoint, its committed buffer entries and their
+ * count, nothing else (blog "Decodificacion estandar"; abstract: the buffer keeps the
+ * raw inputs since the checkpoint). A snapshot holds exactly that, as one self-describing
+ * block per sequence: a prefix-cache or migration unit (the hamidun.com page and the video
+ * takeaways on snapshots and prefix caching). Layout of one block, replay_snapshot_bytes
+ * long, all little-endian:
+ *   int32[16] header: magic 0x4E535052, count c, H, P, N, L, R, G, RK, then zeros;
+ *   FP32 [H][P][N]: the checkpoint S0 (the FP32 master);
+ *   [G][L] k records of RK bytes, then [H][L] head records of R bytes: the committed
+ *   entries, oldest first, in records 0 .. c-1 (the ring layouts; records c .. L-1 are
+ *   unspecified).
+ * The read copy is not stored: it is a function of the master (replay_init's per-row
+ * quantiser), and import recomputes it. */
+
+/* Bytes of one sequence's snapshot: 64 + H*P*N*4 + G*L*RK + H*L*R (a multiple of 16).
+ * Returns a negative replay_status on a bad config. */
+int64_t replay_snapshot_bytes(const replay_config* cfg);
+
+/* Writes the snapshots of the n sequences seqs[0 .. n) (device int32 [n]) into dst
+ * (device, [n][replay_snapshot_bytes], 16-byte aligned), on the stream. The state is
+ * read, not changed. A sequence id out of range (or a corrupt pointer word) writes a
+ * header with magic 0 and sets REPLAY_DEV_POINTER. Returns REPLAY_EPENDING while a verify
+ * awaits its rollback (tentative entries are not part of a snapshot). */
+int replay_export(replay_ctx* ctx, const int32_t* seqs, int32_t n, void* dst, replay_stream_t stream);
+
+/* Restores snapshot i of src (device, [n][replay_snapshot_bytes], as replay_export wrote
+ * it, from a context of the same H, G, P, N, L and io; batch and max_pos may differ) into
+ * sequence seqs[i] of this context: its S0, its rings (entries in records 0 .. c-1) and
+ * its pointer word; with a read copy also its codes and row scales, quantised from the
+ * restored master. Decoding then continues exactly as it would have in the exporting
+ * context (with the same checkpoint kind). A snapshot whose header does not match this
+ * layer, or a
+ * sequence id out of range, is skipped and sets REPLAY_DEV_SNAPSHOT. The seqs must be
+ * distinct. Returns REPLAY_EPENDING while a verify awaits its rollback. */
+int replay_import(replay_ctx* ctx, const int32_t* seqs, int32_t n, const void* src,
+                  replay_stream_t stream);
 
 /* Copies the committed entry count of every sequence to host_counts (host int32 [B]);
  * synchronises the stream. */
@@ -190,6 +276,15 @@ int eager_step(const replay_config* cfg, float* S, const void* q, const void* k,
 int eager_step_fp8(const replay_config* cfg, uint8_t* S8, float* scale, const void* q,
                    const void* k, const void* v, const float* dt, const float* a, float* y,
                    replay_stream_t stream);
+
+/* Per-row e2m1 quantisation used for the FP4 read copy: for each row of n FP32 values,
+ * scale = amax/6 (1 for an all-zero row) and code = e2m1(x * (6/amax)) with the product
+ * rounded to FP32, round-to-nearest-even, saturating to +-6; codes packed two per byte
+ * (element 2i in the low nibble).
+ *   x: device [rows][n] FP32   codes: device [rows][n/2] uint8   scale: device [rows] FP32
+ *   n: 16, 32, 64 or 128. */
+int replay_quantize_rows_e2m1(const float* x, int64_t rows, int32_t n, uint8_t* codes,
+                              float* scale, replay_stream_t stream);
 
 /* Per-row e4m3 quantisation used for the FP8 read copy: for each row of n FP32 values,
  * scale = amax/448 (1 for an all-zero row) and code = e4m3(x * (448/amax)) with the

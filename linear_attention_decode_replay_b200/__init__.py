@@ -39,6 +39,7 @@ from . import _abi
 from ._abi import (  # noqa: F401
     DEV_POINTER,
     DEV_ROLLBACK,
+    DEV_SNAPSHOT,
     DEV_WAIT_TIMEOUT,
     ReplayError,
     check,
@@ -46,8 +47,13 @@ from ._abi import (  # noqa: F401
     strerror,
 )
 
-__all__ = ["Config", "Replay", "alloc_buffers", "ring_capacity", "ring_record_bytes", "eager_step", "eager_step_fp8",
-           "quantize_rows_e4m3", "ReplayError", "load", "strerror"]
+__all__ = ["Config", "Replay", "alloc_buffers", "ring_capacity", "ring_record_bytes", "ring_k_record_bytes",
+           "code_shape", "snapshot_bytes", "eager_step", "eager_step_fp8", "quantize_rows_e4m3", "quantize_rows_e2m1",
+           "ReplayError", "load", "strerror"]
+
+
+_CKPT = {"f32": _abi.REPLAY_CKPT_F32, "f32_fp8read": _abi.REPLAY_CKPT_F32_FP8READ,
+         "f32_fp4read": _abi.REPLAY_CKPT_F32_FP4READ}
 
 
 @dataclass(frozen=True)
@@ -62,12 +68,12 @@ class Config:
     L: int
     max_pos: int = 1
     io: str = "bf16"  # "bf16" or "f32": dtype of q, k, v
-    ckpt: str = "f32"  # "f32" or "f32_fp8read"
+    ckpt: str = "f32"  # "f32", "f32_fp8read" or "f32_fp4read"
 
     def c(self) -> _abi.CConfig:
         return _abi.CConfig(self.batch, self.heads, self.groups, self.P, self.N, self.L, self.max_pos,
                             _abi.REPLAY_BF16 if self.io == "bf16" else _abi.REPLAY_F32,
-                            _abi.REPLAY_CKPT_F32_FP8READ if self.ckpt == "f32_fp8read" else _abi.REPLAY_CKPT_F32)
+                            _CKPT[self.ckpt])
 
     @property
     def io_dtype(self) -> torch.dtype:
@@ -82,9 +88,32 @@ def ring_capacity(cfg: Config) -> int:
 
 
 def ring_record_bytes(cfg: Config) -> int:
+    """Bytes of one head record of the ring (v, Delta, a)."""
     r = load().replay_ring_record_bytes(ctypes.byref(cfg.c()))
     if r < 0:
         raise ReplayError(r, "replay_ring_record_bytes")
+    return r
+
+
+def ring_k_record_bytes(cfg: Config) -> int:
+    """Bytes of one k record of the ring (one per k/q group)."""
+    r = load().replay_ring_k_record_bytes(ctypes.byref(cfg.c()))
+    if r < 0:
+        raise ReplayError(r, "replay_ring_k_record_bytes")
+    return r
+
+
+def code_shape(cfg: Config):
+    """Shape of the read copy's codes (uint8): FP8 one byte per value, FP4 two values per byte."""
+    n = cfg.N // 2 if cfg.ckpt == "f32_fp4read" else cfg.N
+    return (cfg.batch, cfg.heads, cfg.P, n)
+
+
+def snapshot_bytes(cfg: Config) -> int:
+    """Bytes of one sequence's snapshot (replay_export / replay_import)."""
+    r = load().replay_snapshot_bytes(ctypes.byref(cfg.c()))
+    if r < 0:
+        raise ReplayError(r, "replay_snapshot_bytes")
     return r
 
 
@@ -92,17 +121,19 @@ def alloc_buffers(cfg: Config, device="cuda") -> dict:
     """Allocates the caller-owned device buffers of one layer (S0 left uninitialised)."""
     cap = ring_capacity(cfg)
     rec = ring_record_bytes(cfg)
+    rk = ring_k_record_bytes(cfg)
     B, H, G, P, N = cfg.batch, cfg.heads, cfg.groups, cfg.P, cfg.N
     bufs = {
         "S0": torch.empty(B, H, P, N, device=device, dtype=torch.float32),
+        "ring_k": torch.zeros(B, G, cap, rk, device=device, dtype=torch.uint8),
         "ring": torch.zeros(B, H, cap, rec, device=device, dtype=torch.uint8),
         "counts": torch.zeros(2, B, device=device, dtype=torch.int32),
         "status": torch.zeros(1, device=device, dtype=torch.int32),
     }
     if cfg.max_pos > 1:
         bufs["qpack"] = torch.empty(B, G, cfg.max_pos, N, device=device, dtype=cfg.io_dtype)
-    if cfg.ckpt == "f32_fp8read":
-        bufs["S0_fp8"] = torch.empty(B, H, P, N, device=device, dtype=torch.uint8)
+    if cfg.ckpt != "f32":
+        bufs["S0_codes"] = torch.empty(code_shape(cfg), device=device, dtype=torch.uint8)
         bufs["S0_scale"] = torch.empty(B, H, P, device=device, dtype=torch.float32)
     return bufs
 
@@ -138,12 +169,14 @@ class Replay:
         lib = load()
         B, H, G, P, N = cfg.batch, cfg.heads, cfg.groups, cfg.P, cfg.N
         cap = ring_capacity(cfg)
-        fp8 = cfg.ckpt == "f32_fp8read"
+        copy = cfg.ckpt != "f32"
         rec = ring_record_bytes(cfg)
+        rk = ring_k_record_bytes(cfg)
         cb = _abi.CBuffers(
             _ptr(buffers["S0"], (B, H, P, N), torch.float32, "S0"),
-            _ptr(buffers.get("S0_fp8"), (B, H, P, N), torch.uint8, "S0_fp8") if fp8 else None,
-            _ptr(buffers.get("S0_scale"), (B, H, P), torch.float32, "S0_scale") if fp8 else None,
+            _ptr(buffers.get("S0_codes"), code_shape(cfg), torch.uint8, "S0_codes") if copy else None,
+            _ptr(buffers.get("S0_scale"), (B, H, P), torch.float32, "S0_scale") if copy else None,
+            _ptr(buffers["ring_k"], (B, G, cap, rk), torch.uint8, "ring_k"),
             _ptr(buffers["ring"], (B, H, cap, rec), torch.uint8, "ring"),
             _ptr(buffers.get("qpack"), (B, G, cfg.max_pos, N), cfg.io_dtype, "qpack") if cfg.max_pos > 1 else None,
             _ptr(buffers["counts"], (2, B), torch.int32, "counts"),
@@ -203,6 +236,58 @@ class Replay:
             _ptr(flushed, (self.cfg.batch,), torch.uint8, "flushed"), _stream(stream)),
             "replay_verify_static_scratch")
         return y
+
+    def append_slots(self, slots=None, stream=None):
+        """Ring record of every sequence's next entry (int32 [B] on the device, written on
+        the stream): position s of head h of sequence b goes to record (slots[b] + s) % cap
+        of ring[b][h]. For callers that write the entries there themselves and then call
+        step_resident / verify_resident."""
+        if slots is None:
+            slots = torch.empty(self.cfg.batch, device=self.buffers["counts"].device, dtype=torch.int32)
+        check(self._lib.replay_append_slots(self._ctx, _ptr(slots, (self.cfg.batch,), torch.int32, "slots"),
+                                            _stream(stream)), "replay_append_slots")
+        return slots
+
+    def step_resident(self, q, y=None, flushed=None, stream=None):
+        """step() whose entry the caller already wrote into the ring at append_slots()."""
+        qs, vs, _ = self._token_shapes(None)
+        if y is None:
+            y = torch.empty(vs, device=q.device, dtype=torch.float32)
+        check(self._lib.replay_step_resident(self._ctx, _ptr(q, qs, self.cfg.io_dtype, "q"),
+                                             _ptr(y, vs, torch.float32, "y"),
+                                             _ptr(flushed, (self.cfg.batch,), torch.uint8, "flushed"),
+                                             _stream(stream)), "replay_step_resident")
+        return y
+
+    def verify_resident(self, q, y=None, flushed=None, stream=None):
+        """verify() whose n_pos = q.shape[1] entries the caller already wrote into the ring."""
+        n_pos = q.shape[1]
+        qs, vs, _ = self._token_shapes(n_pos)
+        if y is None:
+            y = torch.empty(vs, device=q.device, dtype=torch.float32)
+        check(self._lib.replay_verify_resident(self._ctx, n_pos, _ptr(q, qs, self.cfg.io_dtype, "q"),
+                                               _ptr(y, vs, torch.float32, "y"),
+                                               _ptr(flushed, (self.cfg.batch,), torch.uint8, "flushed"),
+                                               _stream(stream)), "replay_verify_resident")
+        return y
+
+    def export(self, seqs, dst=None, stream=None):
+        """Snapshots of the sequences seqs (int32 [n] on the device) into dst (uint8 [n,
+        snapshot_bytes] on the device, allocated here if None); returns dst."""
+        n = seqs.shape[0]
+        nb = snapshot_bytes(self.cfg)
+        if dst is None:
+            dst = torch.empty(n, nb, device=seqs.device, dtype=torch.uint8)
+        check(self._lib.replay_export(self._ctx, _ptr(seqs, (n,), torch.int32, "seqs"), n,
+                                      _ptr(dst, (n, nb), torch.uint8, "dst"), _stream(stream)), "replay_export")
+        return dst
+
+    def import_(self, seqs, src, stream=None):
+        """Restores snapshot i of src (uint8 [n, snapshot_bytes]) into sequence seqs[i]."""
+        n = seqs.shape[0]
+        check(self._lib.replay_import(self._ctx, _ptr(seqs, (n,), torch.int32, "seqs"), n,
+                                      _ptr(src, (n, snapshot_bytes(self.cfg)), torch.uint8, "src"), _stream(stream)),
+              "replay_import")
 
     def rollback(self, n_keep, stream=None):
         """Keep n_keep[b] (int32 [B] on the device) of the pending verify's positions."""
@@ -266,6 +351,23 @@ def eager_step_fp8(cfg: Config, S8, scale, q, k, v, dt, a, y=None, stream=None):
                                 _ptr(dt, (B, H), torch.float32, "dt"), _ptr(a, (B, H), torch.float32, "a"),
                                 _ptr(y, (B, H, P), torch.float32, "y"), _stream(stream)), "eager_step_fp8")
     return y
+
+
+def quantize_rows_e2m1(x, codes=None, scale=None, stream=None):
+    """Per-row e2m1 codes (two per byte, element 2i in the low nibble) and FP32 scales of
+    x [..., n] (FP32, n in 16/32/64/128)."""
+    n = x.shape[-1]
+    rows = x.numel() // n
+    cshape = (*x.shape[:-1], n // 2)
+    if codes is None:
+        codes = torch.empty(cshape, device=x.device, dtype=torch.uint8)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], device=x.device, dtype=torch.float32)
+    check(load().replay_quantize_rows_e2m1(_ptr(x, None, torch.float32, "x"), rows, n,
+                                           _ptr(codes, cshape, torch.uint8, "codes"),
+                                           _ptr(scale, x.shape[:-1], torch.float32, "scale"), _stream(stream)),
+          "replay_quantize_rows_e2m1")
+    return codes, scale
 
 
 def quantize_rows_e4m3(x, codes=None, scale=None, stream=None):

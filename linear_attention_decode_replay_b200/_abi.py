@@ -28,10 +28,12 @@ REPLAY_F32 = 0
 REPLAY_BF16 = 1
 REPLAY_CKPT_F32 = 0
 REPLAY_CKPT_F32_FP8READ = 1
+REPLAY_CKPT_F32_FP4READ = 2
 
 DEV_WAIT_TIMEOUT = 1
 DEV_POINTER = 2
 DEV_ROLLBACK = 4
+DEV_SNAPSHOT = 8
 
 
 class ReplayError(RuntimeError):
@@ -47,9 +49,9 @@ class CConfig(ctypes.Structure):
 
 
 class CBuffers(ctypes.Structure):
-    _fields_ = [("S0", ctypes.c_void_p), ("S0_fp8", ctypes.c_void_p), ("S0_scale", ctypes.c_void_p),
-                ("ring", ctypes.c_void_p), ("qpack", ctypes.c_void_p), ("counts", ctypes.c_void_p),
-                ("status", ctypes.c_void_p)]
+    _fields_ = [("S0", ctypes.c_void_p), ("S0_codes", ctypes.c_void_p), ("S0_scale", ctypes.c_void_p),
+                ("ring_k", ctypes.c_void_p), ("ring", ctypes.c_void_p), ("qpack", ctypes.c_void_p),
+                ("counts", ctypes.c_void_p), ("status", ctypes.c_void_p)]
 
 
 _lib = None
@@ -69,11 +71,18 @@ def load() -> ctypes.CDLL:
     sig = {
         "replay_ring_capacity": (i32, [cfgp]),
         "replay_ring_record_bytes": (i32, [cfgp]),
+        "replay_ring_k_record_bytes": (i32, [cfgp]),
         "replay_init": (ctypes.c_int, [cfgp, ctypes.POINTER(CBuffers), vp, ctypes.POINTER(vp)]),
         "replay_step": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_verify": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_verify_static_scratch": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_rollback": (ctypes.c_int, [vp, vp, vp]),
+        "replay_append_slots": (ctypes.c_int, [vp, vp, vp]),
+        "replay_snapshot_bytes": (i64, [cfgp]),
+        "replay_export": (ctypes.c_int, [vp, vp, i32, vp, vp]),
+        "replay_import": (ctypes.c_int, [vp, vp, i32, vp, vp]),
+        "replay_step_resident": (ctypes.c_int, [vp, vp, vp, vp, vp]),
+        "replay_verify_resident": (ctypes.c_int, [vp, i32, vp, vp, vp, vp]),
         "replay_flush": (ctypes.c_int, [vp, vp, vp]),
         "replay_read_counts": (ctypes.c_int, [vp, vp, vp]),
         "replay_check_status": (ctypes.c_int, [vp, ctypes.POINTER(i32), vp]),
@@ -81,6 +90,7 @@ def load() -> ctypes.CDLL:
         "eager_step": (ctypes.c_int, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "eager_step_fp8": (ctypes.c_int, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "replay_quantize_rows_e4m3": (ctypes.c_int, [vp, i64, i32, vp, vp, vp]),
+        "replay_quantize_rows_e2m1": (ctypes.c_int, [vp, i64, i32, vp, vp, vp]),
         "replay_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():

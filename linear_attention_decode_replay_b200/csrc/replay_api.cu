@@ -13,6 +13,7 @@
 #include "replay_launch.h"
 
 using replay::KParams;
+using replay::SnapParams;
 
 struct replay_ctx {
   replay_config cfg;
@@ -31,8 +32,7 @@ struct replay_ctx {
 
 namespace {
 
-constexpr int kHeaderBytes = 256;  // the kernel's mbarriers and abort flag
-constexpr int kGroups = replay::kGroups;  // consumer groups per CTA
+constexpr int kHeaderBytes = replay::kHeaderBytes;  // the kernel's mbarriers and flags
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -48,15 +48,22 @@ int validate_config(const replay_config* c, bool needs_window) {
   if (needs_window) {
     if (c->L < 1 || c->L > replay::kMaxWindow) return REPLAY_EINVAL;
     if (c->max_pos < 1 || c->max_pos > replay::kMaxPos || c->max_pos > c->L) return REPLAY_EINVAL;
-    if (c->ckpt != REPLAY_CKPT_F32 && c->ckpt != REPLAY_CKPT_F32_FP8READ) return REPLAY_EINVAL;
+    if (c->ckpt != REPLAY_CKPT_F32 && c->ckpt != REPLAY_CKPT_F32_FP8READ && c->ckpt != REPLAY_CKPT_F32_FP4READ)
+      return REPLAY_EINVAL;
   }
   return REPLAY_OK;
 }
 
 int ring_capacity(const replay_config& c) { return c.L + c.max_pos; }
+// head record: v (P io values), Delta, a; k record: k (N io values)
 int record_bytes(const replay_config& c) {
   const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
-  return round_up((c.N + c.P) * s_io + 8, 16);
+  return round_up(c.P * s_io + 8, 16);
+}
+int record_k_bytes(const replay_config& c) { return c.N * (c.io == REPLAY_BF16 ? 2 : 4); }
+int ckpt_kind(int ckpt) {
+  return ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : ckpt == REPLAY_CKPT_F32_FP4READ ? replay::kCkptFp4
+                                                                                              : replay::kCkptF32;
 }
 
 struct DeviceInfo {
@@ -73,7 +80,8 @@ int device_info(DeviceInfo* d) {
 }
 
 // Shared-memory layout of one launch mode. nq_alloc = query slots per stage, jmax =
-// entries a stage holds (buffer + new), lfold = most entries one unit folds.
+// entries a stage holds (buffer + new), lfold = most entries one unit folds; fp8_eager:
+// the eager launch on a shared FP8 state (its tile is the codes and scales).
 int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, int cap, int smem_optin) {
   std::memset(p, 0, sizeof(*p));
   const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
@@ -93,26 +101,32 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
     lfold = 1;
   }
   p->rec_bytes = record_bytes(c);
+  p->rec_k_bytes = record_k_bytes(c);
   // a unit is one row group of a head (all of it when P is smaller): its tile is at most
   // 64 rows x 128 floats, whatever P
   const int UR = P < replay::row_group_rows(N) ? P : replay::row_group_rows(N);
   const int tile = fp8_eager ? round_up(UR * N + UR * 4, 16) : UR * N * 4;
-  p->off_rec = round_up(tile, 16);
+  p->off_krec = round_up(tile, 16);
+  p->off_rec = p->off_krec + jmax * p->rec_k_bytes;
   p->off_q = p->off_rec + jmax * p->rec_bytes;
   p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
-  p->stage_bytes = round_up(p->off_meta + 16, 128);
+  // the stage's coefficient area, written by a coefficient warp for the row warps:
+  // alpha[kMaxPos], the fold weights [kMaxWindow] + abar, the buffer terms u[nq][UR] and
+  // the fold weight table wt[lfold][UR] (a unit's rows, zero past the head's)
+  p->off_coef = p->off_meta + 16;
+  p->co_alpha = 0;
+  p->co_sig = replay::kMaxPos * 4;
+  p->co_u = round_up(p->co_sig + (replay::kMaxWindow + 1) * 4, 16);
+  p->u_stride = UR;
+  p->co_wt = round_up(p->co_u + nq_alloc * UR * 4, 16);
+  p->wt_stride = UR;
+  p->stage_bytes = round_up(p->off_coef + p->co_wt + lfold * UR * 4, 128);
 
-  // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
-  // abar, the outputs' entry coefficients [kMaxPos][kMaxWindow], and the fold weights
-  // times v, [lfold][wt_stride] (a unit's rows, padded to a multiple of kRowsPerThread)
-  p->wt_stride = round_up(UR, replay::kRowsPerThread);
-  p->ws_alpha = 0;
-  p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
-  p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
-  p->ws_wt = round_up(p->ws_cw + replay::kMaxPos * replay::kMaxWindow * 4, 16);
-  p->ws_group_bytes = round_up(p->ws_wt + lfold * p->wt_stride * 4, 128);
+  // one scratch area per coefficient warp: the group's k . q products and the head's entry
+  // coefficients, [nq][kMaxWindow] each
   p->ws_off = kHeaderBytes;
-  p->stages_off = round_up(p->ws_off + kGroups * p->ws_group_bytes, 128);
+  p->ws_bytes = 2 * (nq_alloc > 0 ? nq_alloc : 1) * replay::kMaxWindow * 4;
+  p->stages_off = round_up(p->ws_off + replay::kCoefWarps * p->ws_bytes, 128);
   const int avail = smem_optin - p->stages_off;
   int ns = avail / p->stage_bytes;
   if (ns > replay::kMaxStages) ns = replay::kMaxStages;
@@ -151,9 +165,10 @@ cudaError_t launch_main(const KParams& p, const replay_config& c, int ckpt, int 
 
 void set_state(KParams* p, const replay_ctx* ctx) {
   p->S = ctx->bufs.S0;
-  p->S8 = ctx->bufs.S0_fp8;
+  p->S8 = ctx->bufs.S0_codes;
   p->Sscale = ctx->bufs.S0_scale;
   p->ring = ctx->bufs.ring;
+  p->ring_k = ctx->bufs.ring_k;
   p->qpack = nullptr;
   p->qpack_pos = ctx->cfg.max_pos;
   p->counts_in = ctx->bufs.counts + (size_t)ctx->parity * ctx->cfg.batch;
@@ -168,8 +183,11 @@ int check_inputs(const void* q, const void* k, const void* v, const float* dt, c
   return REPLAY_OK;
 }
 
+// One step or verify call. resident: the call's entries are already in the ring (the
+// caller wrote them at replay_append_slots' records), so nothing is appended.
 int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const void* k, const void* v,
-                const float* dt, const float* a, float* y, uint8_t* flushed, cudaStream_t s) {
+                const float* dt, const float* a, float* y, uint8_t* flushed, cudaStream_t s,
+                bool resident = false) {
   KParams p = (n_pos > 1) ? ctx->kp_verify : ctx->kp_step;
   set_state(&p, ctx);
   p.n_pos = n_pos;
@@ -193,6 +211,7 @@ int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const voi
   pp.n_pos = n_pos;
   pp.hpg = p.hpg;
   pp.rec_bytes = p.rec_bytes;
+  pp.rec_k_bytes = p.rec_k_bytes;
   pp.io_bytes = ctx->cfg.io == REPLAY_BF16 ? 2 : 4;
   pp.qpack_pos = ctx->cfg.max_pos;
   pp.q = q;
@@ -201,19 +220,20 @@ int replay_call(replay_ctx* ctx, int n_pos, int commit, const void* q, const voi
   pp.dt = dt;
   pp.a = a;
   pp.ring = ctx->bufs.ring;
+  pp.ring_k = ctx->bufs.ring_k;
   pp.qpack = n_pos > 1 ? ctx->bufs.qpack : nullptr;
   pp.counts_in = p.counts_in;
+  pp.write_entries = resident ? 0 : 1;
   p.qpack = pp.qpack;
   if (n_pos == 1) {
-    p.append_here = 1;  // the main kernel appends the one new entry itself
+    p.append_here = resident ? 0 : 1;  // the main kernel appends the one new entry itself
   } else {
     const long long tasks = (long long)p.B * p.H;
     const long long blocks = (tasks + 7) / 8;
     const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);
     if (replay::launch_pack_entries(pp, grid, s) != cudaSuccess) return REPLAY_ECUDA;
   }
-  const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
-  if (launch_main(p, ctx->cfg, ckpt, replay::kModeReplay, n_pos, ctx->num_sms, s) !=
+  if (launch_main(p, ctx->cfg, ckpt_kind(ctx->cfg.ckpt), replay::kModeReplay, n_pos, ctx->num_sms, s) !=
       cudaSuccess)
     return REPLAY_ECUDA;
   ctx->parity ^= 1;
@@ -258,6 +278,41 @@ int eager_call(const replay_config* cfg, float* S, uint8_t* S8, float* scale, co
   return REPLAY_OK;
 }
 
+int64_t snapshot_bytes(const replay_config& c) {
+  return replay::kSnapHeaderBytes + (int64_t)c.heads * c.P * c.N * 4 + (int64_t)c.groups * c.L * record_k_bytes(c) +
+         (int64_t)c.heads * c.L * record_bytes(c);
+}
+
+int snapshot_params(replay_ctx* ctx, const int32_t* seqs, int32_t n, void* snap, SnapParams* sp) {
+  if (!ctx || n < 0 || (n > 0 && (!seqs || !snap))) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  if (n > 0 && (!aligned(seqs, 4) || !aligned(snap, 16))) return REPLAY_EALIGN;
+  const replay_config& c = ctx->cfg;
+  if ((int64_t)n * c.heads > INT32_MAX) return REPLAY_EINVAL;
+  sp->B = c.batch;
+  sp->H = c.heads;
+  sp->P = c.P;
+  sp->N = c.N;
+  sp->L = c.L;
+  sp->cap = ctx->cap;
+  sp->rec_bytes = record_bytes(c);
+  sp->rec_k_bytes = record_k_bytes(c);
+  sp->G = c.groups;
+  sp->ckpt = ckpt_kind(c.ckpt);
+  sp->n = n;
+  sp->snap_bytes = snapshot_bytes(c);
+  sp->seqs = seqs;
+  sp->snap = snap;
+  sp->S = ctx->bufs.S0;
+  sp->S8 = ctx->bufs.S0_codes;
+  sp->Sscale = ctx->bufs.S0_scale;
+  sp->ring = ctx->bufs.ring;
+  sp->ring_k = ctx->bufs.ring_k;
+  sp->counts = ctx->bufs.counts + (size_t)ctx->parity * c.batch;
+  sp->status = ctx->bufs.status;
+  return REPLAY_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -274,18 +329,25 @@ int32_t replay_ring_record_bytes(const replay_config* cfg) {
   return record_bytes(*cfg);
 }
 
+int32_t replay_ring_k_record_bytes(const replay_config* cfg) {
+  const int rc = validate_config(cfg, true);
+  if (rc) return rc;
+  return record_k_bytes(*cfg);
+}
+
 int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_stream_t stream, replay_ctx** out) {
   if (!out) return REPLAY_EINVAL;
   *out = nullptr;
   int rc = validate_config(cfg, true);
   if (rc) return rc;
-  if (!bufs || !bufs->S0 || !bufs->ring || !bufs->counts || !bufs->status) return REPLAY_EINVAL;
-  const bool fp8 = cfg->ckpt == REPLAY_CKPT_F32_FP8READ;
-  if (fp8 && (!bufs->S0_fp8 || !bufs->S0_scale)) return REPLAY_EINVAL;
+  if (!bufs || !bufs->S0 || !bufs->ring || !bufs->ring_k || !bufs->counts || !bufs->status) return REPLAY_EINVAL;
+  const bool copy = cfg->ckpt != REPLAY_CKPT_F32;  // a low-precision read copy
+  if (copy && (!bufs->S0_codes || !bufs->S0_scale)) return REPLAY_EINVAL;
   if (cfg->max_pos > 1 && !bufs->qpack) return REPLAY_EINVAL;
-  if (!aligned(bufs->S0, 16) || !aligned(bufs->ring, 16) || !aligned(bufs->counts, 4) || !aligned(bufs->status, 4))
+  if (!aligned(bufs->S0, 16) || !aligned(bufs->ring, 16) || !aligned(bufs->ring_k, 16) ||
+      !aligned(bufs->counts, 4) || !aligned(bufs->status, 4))
     return REPLAY_EALIGN;
-  if (fp8 && (!aligned(bufs->S0_fp8, 16) || !aligned(bufs->S0_scale, 16))) return REPLAY_EALIGN;
+  if (copy && (!aligned(bufs->S0_codes, 16) || !aligned(bufs->S0_scale, 16))) return REPLAY_EALIGN;
   if (cfg->max_pos > 1 && !aligned(bufs->qpack, 16)) return REPLAY_EALIGN;
 
   DeviceInfo d;
@@ -295,8 +357,8 @@ int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_str
   std::memset(ctx, 0, sizeof(*ctx));
   ctx->cfg = *cfg;
   ctx->bufs = *bufs;
-  if (!fp8) {
-    ctx->bufs.S0_fp8 = nullptr;
+  if (!copy) {
+    ctx->bufs.S0_codes = nullptr;
     ctx->bufs.S0_scale = nullptr;
   }
   ctx->cap = ring_capacity(*cfg);
@@ -326,12 +388,15 @@ int replay_init(const replay_config* cfg, const replay_buffers* bufs, replay_str
     delete ctx;
     return REPLAY_ECUDA;
   }
-  if (fp8) {
+  if (copy) {
     const long long rows = (long long)cfg->batch * cfg->heads * cfg->P;
     const long long passes = (rows + (256 / (cfg->N / 4)) - 1) / (256 / (cfg->N / 4));
     const int grid = (int)(passes < (long long)d.num_sms * 8 ? passes : (long long)d.num_sms * 8);
-    if (replay::launch_quantize_rows(bufs->S0, rows, cfg->N, bufs->S0_fp8, bufs->S0_scale, grid, s) !=
-        cudaSuccess) {
+    const cudaError_t e =
+        cfg->ckpt == REPLAY_CKPT_F32_FP4READ
+            ? replay::launch_quantize_rows_e2m1(bufs->S0, rows, cfg->N, bufs->S0_codes, bufs->S0_scale, grid, s)
+            : replay::launch_quantize_rows(bufs->S0, rows, cfg->N, bufs->S0_codes, bufs->S0_scale, grid, s);
+    if (e != cudaSuccess) {
       delete ctx;
       return REPLAY_ECUDA;
     }
@@ -362,6 +427,60 @@ int replay_verify(replay_ctx* ctx, int32_t n_pos, const void* q, const void* k, 
   return rc;
 }
 
+int replay_append_slots(replay_ctx* ctx, int32_t* slots, replay_stream_t stream) {
+  if (!ctx || !slots) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  if (!aligned(slots, 4)) return REPLAY_EALIGN;
+  const int B = ctx->cfg.batch;
+  if (replay::launch_append_slots(ctx->bufs.counts + (size_t)ctx->parity * B, slots, B, ctx->cfg.L, ctx->cap,
+                                  ctx->bufs.status, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return REPLAY_ECUDA;
+  return REPLAY_OK;
+}
+
+int replay_step_resident(replay_ctx* ctx, const void* q, float* y, uint8_t* flushed, replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  if (!q || !y) return REPLAY_EINVAL;
+  if (!aligned(q, 16) || !aligned(y, 4)) return REPLAY_EALIGN;
+  return replay_call(ctx, 1, 1, q, nullptr, nullptr, nullptr, nullptr, y, flushed,
+                     reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int replay_verify_resident(replay_ctx* ctx, int32_t n_pos, const void* q, float* y, uint8_t* flushed,
+                           replay_stream_t stream) {
+  if (!ctx) return REPLAY_EINVAL;
+  if (ctx->pending) return REPLAY_EPENDING;
+  if (n_pos < 1 || n_pos > ctx->cfg.max_pos || n_pos > ctx->cfg.L) return REPLAY_EINVAL;
+  if (!q || !y) return REPLAY_EINVAL;
+  if (!aligned(q, 16) || !aligned(y, 4)) return REPLAY_EALIGN;
+  if (n_pos > 1 && !ctx->verify_ok) return REPLAY_EINVAL;
+  const int rc = replay_call(ctx, n_pos, 0, q, nullptr, nullptr, nullptr, nullptr, y, flushed,
+                             reinterpret_cast<cudaStream_t>(stream), true);
+  if (rc == REPLAY_OK) ctx->pending = n_pos;
+  return rc;
+}
+
+int64_t replay_snapshot_bytes(const replay_config* cfg) {
+  const int rc = validate_config(cfg, true);
+  if (rc) return rc;
+  return snapshot_bytes(*cfg);
+}
+
+int replay_export(replay_ctx* ctx, const int32_t* seqs, int32_t n, void* dst, replay_stream_t stream) {
+  SnapParams sp;
+  const int rc = snapshot_params(ctx, seqs, n, dst, &sp);
+  if (rc || n == 0) return rc;
+  return replay::launch_export(sp, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? REPLAY_OK : REPLAY_ECUDA;
+}
+
+int replay_import(replay_ctx* ctx, const int32_t* seqs, int32_t n, const void* src, replay_stream_t stream) {
+  SnapParams sp;
+  const int rc = snapshot_params(ctx, seqs, n, const_cast<void*>(src), &sp);
+  if (rc || n == 0) return rc;
+  return replay::launch_import(sp, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? REPLAY_OK : REPLAY_ECUDA;
+}
+
 int replay_rollback(replay_ctx* ctx, const int32_t* n_keep, replay_stream_t stream) {
   if (!ctx || !n_keep) return REPLAY_EINVAL;
   if (!ctx->pending) return REPLAY_ENOPENDING;
@@ -383,9 +502,8 @@ int replay_flush(replay_ctx* ctx, const uint8_t* mask, replay_stream_t stream) {
   KParams p = ctx->kp_flush;
   set_state(&p, ctx);
   p.mask = mask;
-  const int ckpt = ctx->cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
-  if (launch_main(p, ctx->cfg, ckpt, replay::kModeFlush, 0, ctx->num_sms, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  if (launch_main(p, ctx->cfg, ckpt_kind(ctx->cfg.ckpt), replay::kModeFlush, 0, ctx->num_sms,
+                  reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return REPLAY_ECUDA;
   ctx->parity ^= 1;
   return REPLAY_OK;
@@ -441,6 +559,24 @@ int replay_quantize_rows_e4m3(const float* x, int64_t rows, int32_t n, uint8_t* 
   const long long passes = (rows + rpb - 1) / rpb;
   const int grid = (int)(passes < (long long)d.num_sms * 8 ? passes : (long long)d.num_sms * 8);
   if (replay::launch_quantize_rows(x, rows, n, codes, scale, grid, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return REPLAY_ECUDA;
+  return REPLAY_OK;
+}
+
+int replay_quantize_rows_e2m1(const float* x, int64_t rows, int32_t n, uint8_t* codes, float* scale,
+                              replay_stream_t stream) {
+  if (!x || !codes || !scale || rows < 0) return REPLAY_EINVAL;
+  if (n != 16 && n != 32 && n != 64 && n != 128) return REPLAY_EINVAL;
+  if (!aligned(x, 16) || !aligned(codes, 2) || !aligned(scale, 4)) return REPLAY_EALIGN;
+  if (rows == 0) return REPLAY_OK;
+  DeviceInfo d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  const long long rpb = 256 / (n / 4);
+  const long long passes = (rows + rpb - 1) / rpb;
+  const int grid = (int)(passes < (long long)d.num_sms * 8 ? passes : (long long)d.num_sms * 8);
+  if (replay::launch_quantize_rows_e2m1(x, rows, n, codes, scale, grid, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return REPLAY_ECUDA;
   return REPLAY_OK;
@@ -565,7 +701,7 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
     ctx->kp_static_ok[n_pos] = 1;
   }
   KParams p = ctx->kp_static[n_pos];
-  const int ckpt = cfg.ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : replay::kCkptF32;
+  const int ckpt = ckpt_kind(cfg.ckpt);
   const bool prefold = cfg.max_pos < n_pos;
   if (prefold) {
     // The ring holds cap = L + max_pos records per head, so a buffer of c entries has room
@@ -603,6 +739,7 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
   pp.n_pos = n_pos;
   pp.hpg = p.hpg;
   pp.rec_bytes = p.rec_bytes;
+  pp.rec_k_bytes = p.rec_k_bytes;
   pp.io_bytes = (int)s_io;
   pp.qpack_pos = n_pos;
   pp.q = q;
@@ -611,8 +748,10 @@ extern "C" int replay_verify_static_scratch(replay_ctx* ctx, int32_t n_pos, cons
   pp.dt = dt;
   pp.a = a;
   pp.ring = ctx->bufs.ring;
+  pp.ring_k = ctx->bufs.ring_k;
   pp.qpack = scratch;
   pp.counts_in = p.counts_in;
+  pp.write_entries = 1;
   const long long tasks = (long long)p.B * p.H;
   const long long blocks = (tasks + 7) / 8;
   const int grid = (int)(blocks < (long long)ctx->num_sms * 16 ? blocks : (long long)ctx->num_sms * 16);

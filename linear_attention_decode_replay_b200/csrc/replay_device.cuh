@@ -10,29 +10,36 @@
 
 namespace replay {
 
-constexpr int kGroupGemvWarps = 4;              // per consumer group: warps that stream the state rows
-constexpr int kGroupWarps = kGroupGemvWarps + 1; // ... plus one warp for the buffer coefficients
-constexpr int kGroups = 2;                       // consumer groups per CTA
-constexpr int kConsumerWarps = kGroups * kGroupWarps;
+constexpr int kRowWarps = 8;                     // warps that stream a unit's state rows
+constexpr int kCoefWarps = 7;                    // warps that form the units' coefficients and buffer terms
+                                                 // (16 warps in all: 4 per scheduler, 128 registers each)
+constexpr int kWorkerWarps = kRowWarps + kCoefWarps;
 constexpr int kProducerWarps = 1;                // the warp that fills stages, in unit order
-constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
+constexpr int kThreads = (kWorkerWarps + kProducerWarps) * 32;
 constexpr int kMaxPos = 8;                       // query positions per verify call
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
 constexpr int kMaxStages = 8;
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
 constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
-constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
-// State rows of one row group: kGroupGemvWarps warps, 128/N rows per warp pass (a row of
-// N floats takes N/4 lanes), kRowsPerThread rows per lane. A unit covers one row group of
-// a head (or the whole head when it has fewer rows), so that every unit's tile is at most
-// 32 KiB of FP32 and as many stages fit in shared memory whatever the head's P.
-constexpr int row_group_rows(int N) { return kGroupGemvWarps * (128 / N) * kRowsPerThread; }
+constexpr int kRowsPerThread = 8;                // state rows one thread covers in a unit
+constexpr int kHeaderBytes = 512;                // the mbarriers and flags at the start of shared memory
+// State rows of one unit: kRowWarps warps, 128/N rows per warp pass (a row of N floats
+// takes N/4 lanes), kRowsPerThread rows per lane. A unit covers this many rows of a head
+// (or the whole head when it has fewer), so that every unit's tile is at most 32 KiB of
+// FP32 and as many stages fit in shared memory whatever the head's P.
+constexpr int row_group_rows(int N) { return kRowWarps * (128 / N) * kRowsPerThread; }
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 
 // status word bits (device-detected errors; the host reads them with replay_check_status)
 constexpr int32_t kErrWaitTimeout = 1 << 0;   // an mbarrier wait gave up
 constexpr int32_t kErrPointer = 1 << 1;       // a buffer pointer word was out of range
 constexpr int32_t kErrRollback = 1 << 2;      // n_keep outside [0, n_pos]
+constexpr int32_t kErrSnapshot = 1 << 3;      // an imported snapshot does not match the layer (skipped)
+
+// snapshot block of one sequence: a header of kSnapHeaderBytes (int32: magic, count, H, P,
+// N, L, record bytes, 0), then the FP32 state [H][P][N], then [H][L] ring records
+constexpr int kSnapHeaderBytes = 64;
+constexpr int32_t kSnapMagic = 0x4E535052;  // "RPSN"
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -204,6 +211,44 @@ __device__ __forceinline__ void e4m3_row_scale(float amax, float& scale, float& 
   if (amax > 0.f) {
     scale = __fdiv_rn(amax, 448.f);
     inv = __fdiv_rn(448.f, amax);
+  } else {
+    scale = 1.f;
+    inv = 1.f;
+  }
+}
+
+// FP4 e2m1 read copy: four codes in 16 bits, element 2i in the low nibble of byte i, 2i+1
+// in its high nibble; the hardware conversions (cvt .e2m1x2) pack the first operand into
+// the upper nibble and unpack the upper nibble into the upper half.
+__device__ __forceinline__ float4 e2m1x4_to_float4(uint32_t w16) {
+  uint32_t h01, h23;
+  asm("{\n\t.reg .b8 lo, hi;\n\t"
+      "mov.b16 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, hi;\n\t}"
+      : "=r"(h01), "=r"(h23)
+      : "h"(static_cast<unsigned short>(w16)));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+// four values of one row, times that row's inverse scale, to e2m1 codes (round to nearest
+// even, saturating to +-6); returns 16 bits
+__device__ __forceinline__ uint32_t quant4_e2m1(float4 x, float inv) {
+  unsigned short out;
+  asm("{\n\t.reg .b8 lo, hi;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 hi, %4, %3;\n\t"
+      "mov.b16 %0, {lo, hi};\n\t}"
+      : "=h"(out)
+      : "f"(__fmul_rn(x.x, inv)), "f"(__fmul_rn(x.y, inv)), "f"(__fmul_rn(x.z, inv)), "f"(__fmul_rn(x.w, inv)));
+  return out;
+}
+// row scale and its inverse for the e2m1 copy (largest magnitude 6; 1 and 1 for a zero row)
+__device__ __forceinline__ void e2m1_row_scale(float amax, float& scale, float& inv) {
+  if (amax > 0.f) {
+    scale = __fdiv_rn(amax, 6.f);
+    inv = __fdiv_rn(6.f, amax);
   } else {
     scale = 1.f;
     inv = 1.f;

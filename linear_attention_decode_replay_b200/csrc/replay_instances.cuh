@@ -19,8 +19,7 @@ constexpr int kMaxDevices = 64;
 
 template <typename IO, int CKPT, int MODE, int NQ>
 cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
-  constexpr int NG = kGroups;  // consumer groups (the host layout reserves one workspace per group)
-  auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ, NG>;
+  auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ>;
   // the dynamic shared-memory opt-in is per function and device; remember the largest set
   // (under a lock: calls may come from several threads, and a smaller concurrent setting
   // must not lower the limit below what another launch needs)
@@ -54,13 +53,15 @@ cudaError_t launch_mode(const KParams& p, int mode, int nq, int grid, cudaStream
                     : launch_one<IO, CKPT, kModeReplay, 1>(p, grid, s);
   }
   if (mode == kModeFlush) return launch_one<IO, CKPT, kModeFlush, 0>(p, grid, s);
-  return launch_one<IO, CKPT, kModeEager, 1>(p, grid, s);
+  if constexpr (CKPT == kCkptFp4) return cudaErrorInvalidValue;  // no eager baseline on an FP4 state
+  else return launch_one<IO, CKPT, kModeEager, 1>(p, grid, s);
 }
 
 template <typename IO>
 cudaError_t launch_ckpt(const KParams& p, int ckpt, int mode, int nq, int grid, cudaStream_t s) {
-  return ckpt == kCkptFp8 ? launch_mode<IO, kCkptFp8>(p, mode, nq, grid, s)
-                          : launch_mode<IO, kCkptF32>(p, mode, nq, grid, s);
+  return ckpt == kCkptFp8   ? launch_mode<IO, kCkptFp8>(p, mode, nq, grid, s)
+         : ckpt == kCkptFp4 ? launch_mode<IO, kCkptFp4>(p, mode, nq, grid, s)
+                            : launch_mode<IO, kCkptF32>(p, mode, nq, grid, s);
 }
 
 }  // namespace

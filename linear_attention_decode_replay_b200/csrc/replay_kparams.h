@@ -6,7 +6,7 @@
 namespace replay {
 
 enum { kModeReplay = 0, kModeFlush = 1, kModeEager = 2 };
-enum { kCkptF32 = 0, kCkptFp8 = 1 };
+enum { kCkptF32 = 0, kCkptFp8 = 1, kCkptFp4 = 2 };
 
 struct KParams {
   // sizes
@@ -32,32 +32,51 @@ struct KParams {
   float* S;
   uint8_t* S8;
   float* Sscale;
-  void* ring;          // [B][H][cap] records of rec_bytes: k (N io), v (P io), Delta, a
+  void* ring_k;        // [B][G][cap] k records of rec_k_bytes: k (N io)
+  void* ring;          // [B][H][cap] head records of rec_bytes: v (P io), Delta, a
   const void* qpack;   // [B][G][qpack_pos][N] io verify queries packed per group, or null
   const int32_t* counts_in;
   int32_t* counts_out;
   int32_t* status;
   // shared-memory layout, bytes
   int32_t num_stages, stage_bytes, stages_off;
-  int32_t rec_bytes, qpack_pos;                // ring record size; positions per qpack group
-  int32_t off_rec, off_q, off_meta;            // within a stage
-  int32_t ws_off, ws_group_bytes;          // one workspace per consumer group
-  int32_t ws_alpha, ws_sig, ws_cw, ws_wt;  // within a group's workspace
-  int32_t wt_stride;                           // row stride of the fold weight table [L][wt_stride]
+  int32_t rec_bytes, rec_k_bytes, qpack_pos;   // head / k record sizes; positions per qpack group
+  int32_t off_krec, off_rec, off_q, off_meta, off_coef;  // within a stage
+  int32_t co_alpha, co_sig, co_u, co_wt;       // within a stage's coefficient area
+  int32_t u_stride, wt_stride;                 // floats per position of u, per entry of wt (= rows_unit)
+  int32_t ws_off, ws_bytes;                    // one scratch area per coefficient warp
   int32_t smem_bytes;
 };
 
 // The pre-pass that writes this call's new entries into their ring records.
 struct PackParams {
-  int32_t B, H, G, P, N, L, cap, n_pos, hpg, rec_bytes, io_bytes, qpack_pos;
+  int32_t B, H, G, P, N, L, cap, n_pos, hpg, rec_bytes, rec_k_bytes, io_bytes, qpack_pos;
+  int32_t write_entries;  // 0: the entries are already in the ring (resident calls): pack queries only
   const void* q;
   const void* k;
   const void* v;
   const float* dt;
   const float* a;
+  void* ring_k;
   void* ring;
   void* qpack;  // null: no packing of the queries
   const int32_t* counts_in;
+};
+
+// Snapshot export / import of n listed sequences.
+struct SnapParams {
+  int32_t B, H, G, P, N, L, cap, rec_bytes, rec_k_bytes, n;
+  int64_t snap_bytes;      // bytes of one sequence's snapshot
+  const int32_t* seqs;     // [n] sequence ids (device)
+  void* snap;              // [n][snap_bytes] snapshots (device)
+  float* S;
+  uint8_t* S8;             // the read copy's codes and its scales (import re-quantises), or null
+  float* Sscale;
+  int32_t ckpt;            // kCkptFp8 / kCkptFp4: the read copy's format (import re-quantises)
+  void* ring_k;
+  void* ring;
+  int32_t* counts;         // the current half of the pointer words
+  int32_t* status;
 };
 
 }  // namespace replay

@@ -80,7 +80,8 @@ def run_decode(shape: gen.Shape, steps: int, rows, flush_at_end=True, fp8_emulat
     every step (y, flush flags); all sequences' counts checked at the end."""
     cfg, bufs, r, S0 = setup(shape)
     ref = ro.ReplayBatch(_np(S0, rows), shape.G, shape.L, ckpt="f32")
-    emu = ro.ReplayBatch(_np(S0, rows), shape.G, shape.L, ckpt="f32_fp8read") if fp8_emulation else None
+    # the oracle's emulation of the same read-copy method (FP8 or FP4), beside the FP32 oracle
+    emu = ro.ReplayBatch(_np(S0, rows), shape.G, shape.L, ckpt=shape.ckpt) if fp8_emulation else None
     if shared_fp8:  # the in-house shared-FP8 eager kernel on the same inputs, for comparison
         codes_d, scale_d = lar.quantize_rows_e4m3(S0)
     rep = Report()

@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "replay.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?(?:int|int32_t|void|char)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|int32_t|int64_t|void|char)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
@@ -26,7 +26,9 @@ def test_header_declares_the_entry_points():
     for want in ("replay_init", "replay_step", "replay_verify", "replay_rollback", "replay_flush",
                  "replay_read_counts", "replay_check_status", "replay_destroy", "eager_step",
                  "eager_step_fp8", "replay_quantize_rows_e4m3", "replay_ring_capacity", "replay_ring_record_bytes",
-                 "replay_strerror"):
+                 "replay_strerror", "replay_append_slots", "replay_step_resident", "replay_verify_resident",
+                 "replay_verify_static_scratch", "replay_snapshot_bytes", "replay_export", "replay_import",
+                 "replay_ring_k_record_bytes", "replay_quantize_rows_e2m1"):
         assert want in names
 
 
@@ -48,31 +50,50 @@ def test_ring_capacity_and_config_checks():
     assert lib.replay_ring_capacity(ctypes.byref(_cfg())) == 6  # L + max_pos
     assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=1))) == 17
     assert lib.replay_ring_capacity(ctypes.byref(_cfg(L=16, max_pos=5))) == 21
-    # record: k (N io) + v (P io) + Delta + a, padded to 16 bytes
-    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg())) == 144  # (16 + 16) * 4 + 8 -> 144
-    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 400
+    # head record: v (P io) + Delta + a, padded to 16 bytes; k record: k (N io), once per group
+    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg())) == 80  # 16 * 4 + 8 -> 80
+    assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 144  # 136 -> 144
+    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg())) == 64
+    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 256
     for bad in (dict(groups=3), dict(P=12), dict(P=0), dict(N=48), dict(N=256), dict(L=0),
-                dict(max_pos=9), dict(max_pos=5, L=4), dict(io=7), dict(ckpt=3), dict(batch=0),
+                dict(max_pos=9), dict(max_pos=5, L=4), dict(io=7), dict(ckpt=3), dict(ckpt=-1), dict(batch=0),
                 dict(P=256, N=128)):
         assert lib.replay_ring_capacity(ctypes.byref(_cfg(**bad))) == _abi.REPLAY_EINVAL, bad
         assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(**bad))) == _abi.REPLAY_EINVAL, bad
+        assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg(**bad))) == _abi.REPLAY_EINVAL, bad
+
+
+def test_snapshot_bytes():
+    lib = _abi.load()
+    # header 64 + H*P*N*4 + G*L*RK + H*L*R
+    assert lib.replay_snapshot_bytes(ctypes.byref(_cfg())) == 64 + 4 * 16 * 16 * 4 + 2 * 4 * 64 + 4 * 4 * 80
+    big = _cfg(batch=256, heads=64, groups=64, P=64, N=128, L=16, max_pos=1, io=_abi.REPLAY_BF16)
+    assert lib.replay_snapshot_bytes(ctypes.byref(big)) == 64 + 64 * 64 * 128 * 4 + 64 * 16 * 256 + 64 * 16 * 144
+    shared = _cfg(batch=256, heads=64, groups=8, P=64, N=128, L=16, max_pos=1, io=_abi.REPLAY_BF16)
+    assert lib.replay_snapshot_bytes(ctypes.byref(shared)) == 64 + 64 * 64 * 128 * 4 + 8 * 16 * 256 + 64 * 16 * 144
+    assert lib.replay_snapshot_bytes(ctypes.byref(_cfg(groups=3))) == _abi.REPLAY_EINVAL
 
 
 def test_init_rejects_bad_arguments_before_any_cuda_call():
     lib = _abi.load()
     ctx = ctypes.c_void_p()
     good = ctypes.c_void_p(0x10000)
-    bufs = _abi.CBuffers(good, None, None, good, good, good, good)
+    bufs = _abi.CBuffers(good, None, None, good, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg(groups=3)), ctypes.byref(bufs), None, ctypes.byref(ctx)) == \
         _abi.REPLAY_EINVAL
-    nulls = _abi.CBuffers(None, None, None, good, good, good, good)
+    nulls = _abi.CBuffers(None, None, None, good, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(nulls), None, ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
-    odd = _abi.CBuffers(ctypes.c_void_p(0x10008), None, None, good, good, good, good)
+    no_ring_k = _abi.CBuffers(good, None, None, None, good, good, good, good)
+    assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(no_ring_k), None, ctypes.byref(ctx)) == \
+        _abi.REPLAY_EINVAL
+    assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(nulls), None, ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
+    odd = _abi.CBuffers(ctypes.c_void_p(0x10008), None, None, good, good, good, good, good)
     assert lib.replay_init(ctypes.byref(_cfg()), ctypes.byref(odd), None, ctypes.byref(ctx)) == _abi.REPLAY_EALIGN
-    fp8_missing = _abi.CBuffers(good, None, None, good, good, good, good)
-    assert lib.replay_init(ctypes.byref(_cfg(ckpt=_abi.REPLAY_CKPT_F32_FP8READ)), ctypes.byref(fp8_missing), None,
-                           ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
-    no_qpack = _abi.CBuffers(good, None, None, good, None, good, good)
+    codes_missing = _abi.CBuffers(good, None, None, good, good, good, good, good)
+    for ckpt in (_abi.REPLAY_CKPT_F32_FP8READ, _abi.REPLAY_CKPT_F32_FP4READ):
+        assert lib.replay_init(ctypes.byref(_cfg(ckpt=ckpt)), ctypes.byref(codes_missing), None,
+                               ctypes.byref(ctx)) == _abi.REPLAY_EINVAL
+    no_qpack = _abi.CBuffers(good, None, None, good, good, None, good, good)
     assert lib.replay_init(ctypes.byref(_cfg(max_pos=2)), ctypes.byref(no_qpack), None, ctypes.byref(ctx)) == \
         _abi.REPLAY_EINVAL
     assert not ctx.value
@@ -87,6 +108,11 @@ def test_calls_on_a_null_context_are_rejected():
     assert lib.replay_flush(None, None, None) == _abi.REPLAY_EINVAL
     assert lib.replay_read_counts(None, p, None) == _abi.REPLAY_EINVAL
     assert lib.replay_check_status(None, None, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_append_slots(None, p, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_step_resident(None, p, p, None, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_verify_resident(None, 2, p, p, None, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_export(None, p, 1, p, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_import(None, p, 1, p, None) == _abi.REPLAY_EINVAL
     lib.replay_destroy(None)
 
 
@@ -100,10 +126,12 @@ def test_eager_and_quantize_argument_checks():
     assert lib.eager_step_fp8(ctypes.byref(_cfg()), p, None, p, p, p, p, p, p, None) == _abi.REPLAY_EINVAL
     assert lib.replay_quantize_rows_e4m3(p, 4, 24, p, p, None) == _abi.REPLAY_EINVAL
     assert lib.replay_quantize_rows_e4m3(p, 0, 16, p, p, None) == _abi.REPLAY_OK  # nothing to do
+    assert lib.replay_quantize_rows_e2m1(p, 4, 24, p, p, None) == _abi.REPLAY_EINVAL
+    assert lib.replay_quantize_rows_e2m1(p, 0, 16, p, p, None) == _abi.REPLAY_OK
 
 
 def test_strerror_covers_every_code():
-    for code in range(0, -8, -1):
+    for code in range(0, -9, -1):
         assert lar.strerror(code) != "unknown status"
     assert lar.strerror(-99) == "unknown status"
 

@@ -122,7 +122,7 @@ def test_fp8_init_copy_bit_exact():
     cfg, bufs, r, S0 = hx.setup(shape)
     torch.cuda.synchronize()
     codes, scale = ro.quantize_rows_e4m3(S0.cpu().numpy())
-    np.testing.assert_array_equal(bufs["S0_fp8"].cpu().numpy(), codes)
+    np.testing.assert_array_equal(bufs["S0_codes"].cpu().numpy(), codes)
     np.testing.assert_array_equal(bufs["S0_scale"].cpu().numpy(), scale)
     r.close()
 
@@ -132,6 +132,74 @@ def test_eager_fp8_small(P, N):
     shape = gen.Shape("f3", B=2, H=2, G=2, P=P, N=N, L=4, io="f32", seed=33)
     rep = hx.run_eager(shape, 12, np.arange(shape.B), fp8=True)
     assert rep.max_err <= 1e-3, rep.max_err
+
+
+# ------------------------------------------------------------------ FP4 e2m1 read copy
+
+def pack_e2m1(codes):
+    """Oracle codes (one per value) packed two per byte: element 2i low nibble, 2i+1 high."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128])
+def test_quantize_rows_e2m1_bit_exact(n):
+    g = torch.Generator(device="cuda").manual_seed(4321 + n)
+    rows = 4096
+    mags = torch.exp2(torch.randint(-30, 30, (rows, 1), generator=g, device="cuda").float())
+    x = torch.randn(rows, n, generator=g, device="cuda") * mags
+    x[7] = 0.0                       # all-zero row
+    x[9, :] = 0.0
+    x[9, 3] = -2.5                   # single non-zero
+    x[11] = torch.linspace(-6, 6, n, device="cuda")  # values on codes and between
+    x[13] = 1e-30 * torch.randn(n, generator=g, device="cuda")  # tiny magnitudes
+    # every code and every midpoint between neighbouring codes, at scale 1 (row max 6)
+    grid = torch.tensor([0, .25, .5, .75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 6], device="cuda")
+    x[15] = torch.cat([grid, -grid])[:n].repeat((n + 31) // 32)[:n] if n >= 32 else grid[:n]
+    codes, scale = lar.quantize_rows_e2m1(x)
+    want_codes, want_scale = ro.quantize_rows_e2m1(x.cpu().numpy())
+    np.testing.assert_array_equal(scale.cpu().numpy(), want_scale)
+    np.testing.assert_array_equal(codes.cpu().numpy(), pack_e2m1(want_codes))
+
+
+def test_fp4_init_copy_bit_exact():
+    shape = gen.Shape("q2", B=2, H=3, G=3, P=16, N=128, L=4, io="bf16", ckpt="f32_fp4read", seed=36)
+    cfg, bufs, r, S0 = hx.setup(shape)
+    torch.cuda.synchronize()
+    codes, scale = ro.quantize_rows_e2m1(S0.cpu().numpy())
+    np.testing.assert_array_equal(bufs["S0_codes"].cpu().numpy(), pack_e2m1(codes))
+    np.testing.assert_array_equal(bufs["S0_scale"].cpu().numpy(), scale)
+    r.close()
+
+
+def test_fp4_read_copy_decodes_every_code():
+    """The output-only route's decode of the e2m1 read copy: with a one-hot query, Delta =
+    0 and a = 1 every output is one decoded code times its row's scale, exactly; the 16
+    codes (OCP MX e2m1) in both nibble positions, against the oracle's table."""
+    shape = gen.Shape("q4", B=1, H=1, G=1, P=16, N=16, L=16, io="f32", ckpt="f32_fp4read", seed=37)
+    cfg, bufs, r, _ = hx.setup(shape)
+    codes = (np.arange(256).reshape(16, 16) % 16).astype(np.uint8)  # row p: codes 0..15
+    codes = (codes + np.arange(16)[:, None]) % 16                      # each row a rotation
+    scale = np.exp2(np.arange(16) - 8.0).astype(np.float32)
+    bufs["S0_codes"].copy_(torch.from_numpy(pack_e2m1(codes)).view(1, 1, 16, 8))
+    bufs["S0_scale"].copy_(torch.from_numpy(scale).view(1, 1, 16))
+    want = ro.e2m1_decode(codes) * scale[:, None].astype(np.float64)
+    got = np.zeros((16, 16))
+    for n in range(16):  # 16 steps, no flush (the buffer holds L = 16 entries)
+        got[:, n] = r.step(*_one_hot_step(shape, n)).cpu().numpy()[0, 0]
+    assert r.check_status() == 0
+    assert r.read_counts() == [16]
+    np.testing.assert_array_equal(got, want)
+    r.close()
+
+
+@pytest.mark.parametrize("P,N", [(32, 64), (96, 128)], ids=["one_unit", "row_blocks_64_32"])
+def test_fp4_read_copy_small(P, N):
+    shape = gen.Shape("q1", B=3, H=4, G=2, P=P, N=N, L=4, io="f32", ckpt="f32_fp4read", seed=38)
+    rep = hx.run_decode(shape, 21, np.arange(shape.B), fp8_emulation=True)
+    assert rep.max_err_fp8_emul <= 1e-3, rep.max_err_fp8_emul  # against the oracle's FP4 emulation
+    assert rep.flags_equal and rep.counts_equal
+    assert rep.ckpt_err <= hx.TOL_F32  # the master never sees FP4 rounding
 
 
 def _all_finite_e4m3_codes(P=16, N=16):
@@ -160,7 +228,7 @@ def test_fp8_read_copy_decodes_every_code():
     shape = gen.Shape("f4", B=1, H=1, G=1, P=16, N=16, L=16, io="f32", ckpt="f32_fp8read", seed=34)
     cfg, bufs, r, _ = hx.setup(shape)
     codes, scale = _all_finite_e4m3_codes()
-    bufs["S0_fp8"].copy_(torch.from_numpy(codes).view(1, 1, 16, 16))
+    bufs["S0_codes"].copy_(torch.from_numpy(codes).view(1, 1, 16, 16))
     bufs["S0_scale"].copy_(torch.from_numpy(scale).view(1, 1, 16))
     want = ro.e4m3_decode(codes) * scale[:, None].astype(np.float64)
     got = np.zeros((16, 16))
@@ -250,6 +318,38 @@ def test_mamba2_b256_decode_sampled():
     rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 8))
     _check_decode(rep)
     assert rep.max_err <= hx.TOL_BF16
+
+
+def test_mamba2_b256_groups_decode_sampled():
+    """The B=256 layer with k and q shared by groups of 8 heads (G = 8): k stored once per
+    group in the ring, k . q formed once per group; 512 steps, 6 sampled sequences against
+    the oracle every step, counts and flags of all 256 sequences bit-exact."""
+    shape = gen.SHAPES["mamba2_b256_g8"]
+    rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 6, seed=3))
+    _check_decode(rep)
+
+
+def test_mamba2_b256_fp4_sampled():
+    """The FP4 e2m1 read copy at full size over 512 steps (32 flushes), four sampled
+    sequences: per-vector parity against the oracle's emulation of the same FP4-read
+    method, the master exact, and the method's own error against the FP32 oracle reported
+    (written to fp4_error_mamba2_b256.json under REPLAY_REPORT_DIR)."""
+    shape = gen.SHAPES["mamba2_b256_fp4"].replace(steps=512)
+    rows = hx.sample_rows(shape.B, 4, seed=5)
+    rep = hx.run_decode(shape, shape.steps, rows, fp8_emulation=True, shared_fp8=False)
+    report = {"workload": shape.name, "steps": shape.steps, "sampled_sequences": [int(r) for r in rows],
+              "fp4_read_vs_fp4_emulation_max": rep.max_err_fp8_emul,
+              "fp4_read_vs_fp32_oracle_frobenius_max": rep.fro_err, "fp4_read_vs_fp32_oracle_max": rep.max_err,
+              "master_checkpoint_vs_fp32_oracle": rep.ckpt_err}
+    print(json.dumps(report))
+    out_dir = os.environ.get("REPLAY_REPORT_DIR")
+    if out_dir:
+        os.makedirs(out_dir, exist_ok=True)
+        with open(os.path.join(out_dir, "fp4_error_mamba2_b256.json"), "w") as f:
+            json.dump(report, f, indent=1)
+    assert rep.max_err_fp8_emul <= 1e-1, rep.max_err_fp8_emul
+    assert rep.flags_equal and rep.counts_equal
+    assert rep.ckpt_err <= hx.TOL_F32  # the master never sees FP4 rounding
 
 
 def _error_summary(per_vector, per_step_fro):

@@ -57,7 +57,7 @@ class Shape:
     N: int  # k-dim (columns of the per-head state)
     L: int  # window: buffer entries between two checkpoint flushes
     io: str = "bf16"  # dtype of q, k, v: "bf16" or "f32"
-    ckpt: str = "f32"  # "f32" or "f32_fp8read" (FP32 master + FP8 e4m3 read copy)
+    ckpt: str = "f32"  # "f32", "f32_fp8read" or "f32_fp4read" (FP32 master + FP8 / FP4 read copy)
     max_pos: int = 1  # query positions per verify call (1 = plain decode)
     s0: str = "gauss"  # "gauss" or "prefill"
     steps: int = 32
@@ -86,6 +86,13 @@ SHAPES = {
     "mamba2_b256_fp8": Shape("mamba2_b256_fp8", B=256, H=64, G=64, P=64, N=128, L=16,
                              io="bf16", ckpt="f32_fp8read", s0="prefill", steps=2048,
                              seed=2000),
+    # same layer, FP32 master checkpoint + FP4 e2m1 read copy
+    "mamba2_b256_fp4": Shape("mamba2_b256_fp4", B=256, H=64, G=64, P=64, N=128, L=16,
+                             io="bf16", ckpt="f32_fp4read", s0="prefill", steps=2048,
+                             seed=2500),
+    # same layer with k and q shared by groups of 8 heads (8 groups)
+    "mamba2_b256_g8": Shape("mamba2_b256_g8", B=256, H=64, G=8, P=64, N=128, L=16,
+                            io="bf16", s0="prefill", steps=512, seed=1500),
     # speculative verify + rollback, draft length 4 (5 query positions)
     "mamba2_b256_spec": Shape("mamba2_b256_spec", B=256, H=64, G=64, P=64, N=128, L=16,
                               io="bf16", max_pos=5, s0="prefill", steps=256, seed=3000),

@@ -49,6 +49,36 @@ __device__ __forceinline__ void report_error(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// A row warp's release of a stage, counted (after the warp's reads of the stage, which
+// __syncwarp orders before lane 0's fence).
+__device__ __forceinline__ void count_release(int* released, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence_block();
+    atomicAdd(released, 1);
+  }
+}
+// Waits (bounded, about two seconds) until at least `target` row-warp releases of a stage
+// have been counted; the whole warp returns the outcome.
+__device__ __forceinline__ bool wait_released(const int* released, int target, int lane) {
+  bool ok = true;
+  if (lane == 0) {
+    const volatile int* r = released;
+    if (*r < target) {
+      const long long t0 = clock64();
+      while (*r < target) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+          ok = false;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence_block();
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // barriers at the start of shared memory
 struct Bars {
   uint64_t tfull[kMaxStages];   // the unit's state tile (and FP8 scales) landed
@@ -57,6 +87,7 @@ struct Bars {
   uint64_t empty[kMaxStages];   // every row warp is done with the stage
   int abort_flag;
   int last_fill[kMaxStages];    // CTA-local index of the latest unit copied into each stage
+  int released[kMaxStages];     // row-warp releases of each stage so far (kRowWarps per use)
 };
 static_assert(sizeof(Bars) <= kHeaderBytes, "the barrier header must fit the bytes the host layout reserves");
 
@@ -570,39 +601,57 @@ __device__ __forceinline__ void coef_unit(const KParams& p, const Plan& pl, uint
     }
     output_weights<N, IO>(rec, c, n, o0, kq, alpha, cw, lane);
     __syncwarp();
-    // u_s[p] = sum_l cw[s][l] v_{o0+l}[r0 + p]: each v read once for every position, four
-    // entries in flight (cw is zero past each position's window)
-    for (int pr = lane; pr < rows; pr += 32) {
-      const uint8_t* vrow = rec.base + (size_t)(r0 + pr) * S_IO;
-      float acc[NQR];
+    // u_s[p] = sum_l cw[s][l] v_{o0+l}[r0 + p]: two rows per lane at a time (p and p + 32),
+    // each v read once for every position, eight entries in flight per row (cw is zero
+    // past each position's window)
+    for (int pr0 = lane; pr0 < rows; pr0 += 64) {
+      const int pr1 = pr0 + 32 < rows ? pr0 + 32 : pr0;  // the second row, or the first again
+      const uint8_t* vrow0 = rec.base + (size_t)(r0 + pr0) * S_IO;
+      const uint8_t* vrow1 = rec.base + (size_t)(r0 + pr1) * S_IO;
+      float acc0[NQR], acc1[NQR];
 #pragma unroll
-      for (int s = 0; s < NQR; ++s) acc[s] = 0.f;
-      for (int l0 = 0; l0 < width; l0 += 4) {
-        float vv[4];
+      for (int s = 0; s < NQR; ++s) acc0[s] = acc1[s] = 0.f;
+      for (int l0 = 0; l0 < width; l0 += 8) {
+        float v0[8], v1[8];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          vv[r] = (l0 + r < width) ? IoT<IO>::load1(vrow + (size_t)(o0 + l0 + r) * rec.R) : 0.f;
+        for (int r = 0; r < 8; ++r) {
+          const size_t off = (size_t)(o0 + (l0 + r < width ? l0 + r : 0)) * rec.R;
+          v0[r] = (l0 + r < width) ? IoT<IO>::load1(vrow0 + off) : 0.f;
+          v1[r] = (l0 + r < width) ? IoT<IO>::load1(vrow1 + off) : 0.f;
+        }
 #pragma unroll
         for (int s = 0; s < NQR; ++s) {
           if (s < n) {
-            const float4 c4 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0);
-            acc[s] = fmaf(c4.x, vv[0], fmaf(c4.y, vv[1], fmaf(c4.z, vv[2], fmaf(c4.w, vv[3], acc[s]))));
+            const float4 ca = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0);
+            const float4 cb = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0 + 4);
+            acc0[s] = fmaf(ca.x, v0[0], fmaf(ca.y, v0[1], fmaf(ca.z, v0[2], fmaf(ca.w, v0[3],
+                      fmaf(cb.x, v0[4], fmaf(cb.y, v0[5], fmaf(cb.z, v0[6], fmaf(cb.w, v0[7], acc0[s]))))))));
+            acc1[s] = fmaf(ca.x, v1[0], fmaf(ca.y, v1[1], fmaf(ca.z, v1[2], fmaf(ca.w, v1[3],
+                      fmaf(cb.x, v1[4], fmaf(cb.y, v1[5], fmaf(cb.z, v1[6], fmaf(cb.w, v1[7], acc1[s]))))))));
           }
         }
       }
 #pragma unroll
-      for (int s = 0; s < NQR; ++s)
-        if (s < n) u[s * p.u_stride + pr] = acc[s];
+      for (int s = 0; s < NQR; ++s) {
+        if (s < n) {
+          u[s * p.u_stride + pr0] = acc0[s];
+          if (pr0 + 32 < rows) u[s * p.u_stride + pr0 + 32] = acc1[s];
+        }
+      }
     }
   }
 }
 
 // The coefficient warps' loop: the units of a k/q group (its heads, each with its row
 // blocks) all go to one warp, groups in turn, so that the warp forms the group's k . q
-// once. Before a warp waits for a stage's records (rfull, phase k) it waits for the
-// stage's previous release (empty, phase k-1): the row warps were then done with the use
-// before, whose records had landed, so both parity waits are exact however far the warps
-// drift apart. Each warp takes its units in order, so no wait can close a cycle.
+// once. A warp's consecutive units may lie any distance apart, so its parity waits are
+// made exact by counting: before it waits for the k-th use of a stage it waits until the
+// row warps' releases of that stage's use k-2 have all been counted (the row warps take
+// the units in order and cannot be two uses further on, since they need this warp's
+// coefficients for use k). Then it waits for the stage's previous release (empty, phase
+// k-1), after which no one touches the stage, and for its records (rfull, phase k),
+// whose phase k-1 completed before the row warps could release use k-1. Each warp takes
+// its units in order, so no wait can close a cycle.
 template <int N, typename IO, int CKPT, int MODE, int NQ>
 __device__ void coef_loop(const KParams& p, uint8_t* stages, Bars* bars, float* kq, float* cw, int cwarp, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
@@ -617,6 +666,7 @@ __device__ void coef_loop(const KParams& p, uint8_t* stages, Bars* bars, float* 
     const int s = i % NS;
     const int k = i / NS;
     bool ready = *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
+    if (ready && k > 1) ready = wait_released(&bars->released[s], (k - 1) * kRowWarps, lane);
     if (ready && k > 0) ready = mbar_wait_bounded(&bars->empty[s], (k - 1) & 1);
     if (ready) ready = mbar_wait_bounded(&bars->rfull[s], k & 1);
     if (!__all_sync(0xffffffffu, ready)) {
@@ -828,7 +878,7 @@ __device__ void row_loop(const KParams& p, uint8_t* stages, Bars* bars, int warp
     const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, cta_unit(p, i), word, msk);
     if (pl.active) row_unit<N, IO, CKPT, MODE, NQ>(p, pl, st, warp, lane);
-    __syncwarp();
+    count_release(&bars->released[s], lane);
     mbar_arrive(&bars->empty[s]);
   }
 }
@@ -849,7 +899,10 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
       mbar_init(&bars->empty[s], kRowWarps * 32);                // every row warp's lanes
     }
     bars->abort_flag = 0;
-    for (int s = 0; s < kMaxStages; ++s) bars->last_fill[s] = -1;
+    for (int s = 0; s < kMaxStages; ++s) {
+      bars->last_fill[s] = -1;
+      bars->released[s] = 0;
+    }
     fence_mbar_init();
   }
   __syncthreads();

@@ -105,14 +105,17 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   // a unit is one row group of a head (all of it when P is smaller): its tile is at most
   // 64 rows x 128 floats, whatever P
   const int UR = P < replay::row_group_rows(N) ? P : replay::row_group_rows(N);
+  // tile stage: the unit's FP32 rows (a read copy's codes and scales fit in the same space)
   const int tile = fp8_eager ? round_up(UR * N + UR * 4, 16) : UR * N * 4;
-  p->off_krec = round_up(tile, 16);
+  p->tstage_bytes = round_up(tile, 128);
+  // record stage: k records, head records, queries, pointer word, then the coefficient
+  // area a coefficient warp writes for the row warps: alpha[kMaxPos], the fold weights
+  // [kMaxWindow] + abar, the buffer terms u[nq][UR] and the fold weight table wt[lfold][UR]
+  // (a unit's rows, zero past the head's)
+  p->off_krec = 0;
   p->off_rec = p->off_krec + jmax * p->rec_k_bytes;
   p->off_q = p->off_rec + jmax * p->rec_bytes;
   p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
-  // the stage's coefficient area, written by a coefficient warp for the row warps:
-  // alpha[kMaxPos], the fold weights [kMaxWindow] + abar, the buffer terms u[nq][UR] and
-  // the fold weight table wt[lfold][UR] (a unit's rows, zero past the head's)
   p->off_coef = p->off_meta + 16;
   p->co_alpha = 0;
   p->co_sig = replay::kMaxPos * 4;
@@ -120,19 +123,39 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->u_stride = UR;
   p->co_wt = round_up(p->co_u + nq_alloc * UR * 4, 16);
   p->wt_stride = UR;
-  p->stage_bytes = round_up(p->off_coef + p->co_wt + lfold * UR * 4, 128);
+  p->rstage_bytes = round_up(p->off_coef + p->co_wt + lfold * UR * 4, 128);
 
   // one scratch area per coefficient warp: the group's k . q products and the head's entry
   // coefficients, [nq][kMaxWindow] each
   p->ws_off = kHeaderBytes;
   p->ws_bytes = 2 * (nq_alloc > 0 ? nq_alloc : 1) * replay::kMaxWindow * 4;
-  p->stages_off = round_up(p->ws_off + replay::kCoefWarps * p->ws_bytes, 128);
-  const int avail = smem_optin - p->stages_off;
-  int ns = avail / p->stage_bytes;
-  if (ns > replay::kMaxStages) ns = replay::kMaxStages;
-  if (ns < 2) return REPLAY_EINVAL;
-  p->num_stages = ns;
-  p->smem_bytes = p->stages_off + ns * p->stage_bytes;
+  p->tstages_off = round_up(p->ws_off + replay::kCoefWarps * p->ws_bytes, 128);
+  const int avail = smem_optin - p->tstages_off;
+  // Stage counts: as many tile stages as leave room for a record ring that runs ahead of
+  // them by min(tile stages, 4) units (the lookahead that hides the coefficient warps'
+  // chain behind the tiles in flight); the eager launch needs no lookahead.
+  int nt = 0, nr = 0;
+  for (int t = replay::kMaxTileStages; t >= 2 && !nt; --t) {
+    const int want = mode == replay::kModeEager ? t : t + (t < 4 ? t : 4);
+    int r = (avail - t * p->tstage_bytes) / p->rstage_bytes;
+    if (r > replay::kMaxRecStages) r = replay::kMaxRecStages;
+    if (r >= want) {
+      nt = t;
+      nr = r;
+    }
+  }
+  if (!nt) {  // not even two tile stages with their lookahead: two and what fits
+    nt = 2;
+    nr = (avail - 2 * p->tstage_bytes) / p->rstage_bytes;
+    if (nr > replay::kMaxRecStages) nr = replay::kMaxRecStages;
+    if (nr < 2) return REPLAY_EINVAL;
+  }
+  p->num_tstages = nt;
+  p->num_rstages = nr;
+  p->lookahead = mode == replay::kModeEager ? 0 : (nr - nt < nt ? nr - nt : nt);
+  if (p->lookahead < 0) p->lookahead = 0;
+  p->rstages_off = p->tstages_off + nt * p->tstage_bytes;
+  p->smem_bytes = p->rstages_off + nr * p->rstage_bytes;
 
   p->B = c.batch;
   p->H = c.heads;
@@ -148,12 +171,18 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   if (p->row_blocks > 2) return REPLAY_EINVAL;
   p->num_bh = c.batch * c.heads;
   p->num_units = p->num_bh * p->row_blocks;
+  // heads dealt to CTAs in chunks: the largest divisor of the heads per k/q group that is
+  // at most kMaxChunkHeads, so that a chunk never spans two groups
+  int ch = p->hpg < replay::kMaxChunkHeads ? p->hpg : replay::kMaxChunkHeads;
+  while (p->hpg % ch) --ch;
+  p->chunk_heads = ch;
+  p->num_chunks = p->num_bh / ch;
   return REPLAY_OK;
 }
 
 cudaError_t launch_main(const KParams& p, const replay_config& c, int ckpt, int mode, int nq, int num_sms,
                         cudaStream_t s) {
-  const int grid = p.num_bh < num_sms ? p.num_bh : num_sms;  // every CTA holds whole heads
+  const int grid = p.num_chunks < num_sms ? p.num_chunks : num_sms;  // every CTA holds whole chunks of heads
   switch (c.N) {
     case 16: return replay::launch_replay_n16(p, c.io, ckpt, mode, nq, grid, s);
     case 32: return replay::launch_replay_n32(p, c.io, ckpt, mode, nq, grid, s);

@@ -18,11 +18,13 @@ constexpr int kProducerWarps = 1;                // the warp that fills stages, 
 constexpr int kThreads = (kWorkerWarps + kProducerWarps) * 32;
 constexpr int kMaxPos = 8;                       // query positions per verify call
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
-constexpr int kMaxStages = 8;
+constexpr int kMaxTileStages = 8;                // ring of state tiles
+constexpr int kMaxRecStages = 16;                // ring of records, queries and coefficients
+constexpr int kMaxChunkHeads = 8;                // heads of one k/q group a CTA takes in a row
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
 constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
 constexpr int kRowsPerThread = 8;                // state rows one thread covers in a unit
-constexpr int kHeaderBytes = 512;                // the mbarriers and flags at the start of shared memory
+constexpr int kHeaderBytes = 1024;               // the mbarriers and flags at the start of shared memory
 // State rows of one unit: kRowWarps warps, 128/N rows per warp pass (a row of N floats
 // takes N/4 lanes), kRowsPerThread rows per lane. A unit covers this many rows of a head
 // (or the whole head when it has fewer), so that every unit's tile is at most 32 KiB of

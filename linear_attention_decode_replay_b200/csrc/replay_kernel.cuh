@@ -81,13 +81,15 @@ __device__ __forceinline__ bool wait_released(const int* released, int target, i
 
 // barriers at the start of shared memory
 struct Bars {
-  uint64_t tfull[kMaxStages];   // the unit's state tile (and FP8 scales) landed
-  uint64_t rfull[kMaxStages];   // its ring records and queries landed, pointer word written
-  uint64_t cready[kMaxStages];  // its coefficients and buffer terms are in the stage
-  uint64_t empty[kMaxStages];   // every row warp is done with the stage
+  uint64_t tfull[kMaxTileStages];   // the unit's state tile (and read-copy scales) landed
+  uint64_t tempty[kMaxTileStages];  // every row warp is done with the tile stage
+  uint64_t rfull[kMaxRecStages];    // the unit's records and queries landed, pointer word written
+  uint64_t cready[kMaxRecStages];   // its coefficients and buffer terms are in the record stage
+  uint64_t rempty[kMaxRecStages];   // every row warp is done with the record stage
   int abort_flag;
-  int last_fill[kMaxStages];    // CTA-local index of the latest unit copied into each stage
-  int released[kMaxStages];     // row-warp releases of each stage so far (kRowWarps per use)
+  int last_tfill[kMaxTileStages];   // CTA-local index of the latest unit copied into each stage
+  int last_rfill[kMaxRecStages];
+  int released[kMaxRecStages];      // row-warp releases of each record stage so far (kRowWarps per use)
 };
 static_assert(sizeof(Bars) <= kHeaderBytes, "the barrier header must fit the bytes the host layout reserves");
 
@@ -97,23 +99,26 @@ struct Plan {
   uint32_t tile_bytes, rec_bytes;       // bulk-copied bytes completing on tfull / rfull
 };
 
-// This CTA's units, in the order its producer fills them: a contiguous range of heads
-// (sequence-major, so the heads of a k/q group follow one another), each with its row
-// blocks in a row, so that one CTA holds every unit of a head (the in-kernel append writes
-// a head's new record once, before any copy of it) and a group's heads share one
-// coefficient warp (which forms the group's k . q once).
-__device__ __forceinline__ int cta_first_head(const KParams& p) {
-  const int q = p.num_bh / (int)gridDim.x, r = p.num_bh % (int)gridDim.x;
-  return (int)blockIdx.x * q + min((int)blockIdx.x, r);
+// This CTA's units, in the order every role takes them: chunks of chunk_heads consecutive
+// heads of one k/q group (the group, or a part of it, so that its heads share one
+// coefficient warp and its k . q products), chunk c on CTA c mod gridDim.x, each head
+// with its row blocks in a row. Dealing the chunks round-robin keeps the 148 CTAs on
+// neighbouring tiles of the state at any moment, and one CTA holds every unit of a head
+// (the in-kernel append writes a head's new record once, before any copy of it).
+__device__ __forceinline__ int cta_chunks(const KParams& p) {
+  return (p.num_chunks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 }
-__device__ __forceinline__ int cta_heads(const KParams& p) {
-  return p.num_bh / (int)gridDim.x + ((int)blockIdx.x < p.num_bh % (int)gridDim.x ? 1 : 0);
+__device__ __forceinline__ int cta_units(const KParams& p) { return (cta_chunks(p) * p.chunk_heads) << p.rb_shift; }
+// the CTA's i-th head (chunk i / chunk_heads, head i mod chunk_heads within it)
+__device__ __forceinline__ int cta_head(const KParams& p, int hi) {
+  const int ck = hi / p.chunk_heads;
+  return ((int)blockIdx.x + ck * (int)gridDim.x) * p.chunk_heads + (hi - ck * p.chunk_heads);
 }
-__device__ __forceinline__ int cta_units(const KParams& p) { return cta_heads(p) << p.rb_shift; }
 __device__ __forceinline__ int cta_unit(const KParams& p, int i) {
-  const int bh = cta_first_head(p) + (i >> p.rb_shift);
-  return (bh << p.rb_shift) | (i & (p.row_blocks - 1));
+  return (cta_head(p, i >> p.rb_shift) << p.rb_shift) | (i & (p.row_blocks - 1));
 }
+// the CTA-local chunk of unit i
+__device__ __forceinline__ int unit_chunk(const KParams& p, int i) { return (i >> p.rb_shift) / p.chunk_heads; }
 
 template <int MODE, int CKPT, int S_IO>
 __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word, int msk) {
@@ -182,10 +187,10 @@ struct Records {
 // ---------------------------------------------------------------------------- append
 // This CTA's units' new entries (one position) into their ring records, slot
 // (start + c) mod cap, by the worker threads before any bulk copy is issued: each head's
-// v, then Delta and a in one 16-byte piece, and the k of each group once (by the CTA's
-// first head of the group; a group split between two CTAs has its k written by both,
-// the same bytes). The input pieces do not depend on the pointer word, so both reads are
-// in flight together.
+// v, then Delta and a in one 16-byte piece, and the group's k once per chunk (a group of
+// more than kMaxChunkHeads heads spans chunks, possibly on several CTAs, each writing the
+// same bytes before it reads them). The input pieces do not depend on the pointer word,
+// so both reads are in flight together.
 template <int S_IO>
 __device__ __forceinline__ void append_entries(const KParams& p) {
   constexpr int kPool = kWorkerWarps * 32;
@@ -193,8 +198,7 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
   const int kpe = p.N * S_IO / 16;  // 16-byte pieces of k
   const int vpe = p.P * S_IO / 16;  // of v
   const int per_unit = kpe + vpe + 1;
-  const int bh0 = cta_first_head(p);
-  const int total = cta_heads(p) * per_unit;
+  const int total = cta_chunks(p) * p.chunk_heads * per_unit;
   for (int t0 = threadIdx.x; t0 < total; t0 += kBatch * kPool) {
     uint4 val[kBatch];
     uint8_t* dst[kBatch];
@@ -206,11 +210,11 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
       if (t < total) {
         const int iu = t / per_unit;
         const int ch = t - iu * per_unit;
-        const int bh = bh0 + iu;
+        const int bh = cta_head(p, iu);
         const int b = bh / p.H;
         const int h = bh - b * p.H;
         const int g = h / p.hpg;
-        const bool k_here = (h % p.hpg) == 0 || iu == 0;  // the CTA's first head of the group
+        const bool k_here = (iu % p.chunk_heads) == 0;  // the chunk's first head writes the group's k
         const int32_t word = __ldg(p.counts_in + b);
         if (ch < kpe) {
           if (k_here)
@@ -240,14 +244,15 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
 
 // ---------------------------------------------------------------------------- producer
 // Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile (the unit's rows)
-// and 1 their read-copy row scales, completing on tfull; 2-3 the live head records and
+// and 1 their read-copy row scales, into its tile stage `tst`, completing on tfull; into
+// its record stage `rst`: 2-3 the live head records and
 // 4-5 the live k records of the head's group, [start, start + count) modulo cap in one
 // or two pieces (whole records: every row block reads all of k and its rows of v), and
 // 6 the queries, completing on rfull. Returns the bytes of copy `kind` (0 if none) and
 // its addresses.
 constexpr int kCopyKinds = 7;
 template <int MODE, int CKPT, int S_IO>
-__device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, uint8_t* st, int kind,
+__device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, uint8_t* tst, uint8_t* rst, int kind,
                                               const uint8_t*& src, uint8_t*& dst) {
   constexpr size_t kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;
   const size_t P = pl.rows, N = p.N;
@@ -270,13 +275,13 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, 
         : (kind == 4) ? ring_k + (size_t)pl.start * RK
         : (kind == 5) ? ring_k
                       : qsrc;
-  dst = (kind == 0)   ? st
-        : (kind == 1) ? st + (size_t)p.rows_unit * (N / kCodeDiv)  // the scales follow a full unit's codes
-        : (kind == 2) ? st + p.off_rec
-        : (kind == 3) ? st + p.off_rec + (size_t)first * R
-        : (kind == 4) ? st + p.off_krec
-        : (kind == 5) ? st + p.off_krec + (size_t)first * RK
-                      : st + p.off_q;
+  dst = (kind == 0)   ? tst
+        : (kind == 1) ? tst + (size_t)p.rows_unit * (N / kCodeDiv)  // the scales follow a full unit's codes
+        : (kind == 2) ? rst + p.off_rec
+        : (kind == 3) ? rst + p.off_rec + (size_t)first * R
+        : (kind == 4) ? rst + p.off_krec
+        : (kind == 5) ? rst + p.off_krec + (size_t)first * RK
+                      : rst + p.off_q;
   uint32_t bytes = 0;
   bytes = (kind == 0) ? (pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * (N / kCodeDiv))) : bytes;
   bytes = (kind == 1 && !pl.fp32_tile) ? (uint32_t)(P * 4) : bytes;
@@ -288,24 +293,32 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, 
   return pl.active ? bytes : 0u;
 }
 
-// The producer warp fills the CTA's units in order, kUnitsPerIssue at a time: it waits
-// until their stages are free, writes each unit's pointer word into its stage, arms the
-// stage's two "full" barriers with the unit's byte counts, and then one predicated
-// bulk-copy instruction issues every copy of the batch (lane = unit in batch *
-// kCopyKinds + kind). Issuing costs the warp about as much for one copy as for a whole
-// batch, so batching is what keeps the stream fed.
+// The producer warp. Step t copies the records (and queries) of unit t into its record
+// stage and the tile of unit t - D into its tile stage, D = p.lookahead: a unit's records
+// land D units before its tile, so the coefficient warps finish with them before the row
+// warps reach the unit. The tiles of the first num_tstages units go out at once (when the
+// kernel appends this call's entries itself, before the append is complete; their records
+// after it). Steps go kUnitsPerIssue at a time: the producer waits until their stages are
+// free, writes each unit's pointer word into its record stage, arms the stages' barriers
+// with the byte counts and issues every copy of the batch with one predicated bulk-copy
+// instruction (lane = step in batch * kCopyKinds + kind), which costs the warp about as
+// much as one copy. A tile's plan takes the pointer word its record stage holds (written
+// D steps before; the stage stays until the row warps are done with the unit). Waits are
+// exact: the producer visits every use of every stage in order.
 template <int MODE, int CKPT, int S_IO, bool APPEND>
-__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
+__device__ void producer_loop(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars) {
   constexpr int U = kUnitsPerIssue;
   static_assert(U * kCopyKinds <= 32 && (32 % U) == 0, "a batch's copies must fit one warp and tile 32 units");
   const int lane = threadIdx.x & 31;
-  const int NS = p.num_stages;
+  const int NT = p.num_tstages, NR = p.num_rstages, D = p.lookahead;
   const uint64_t stream_policy = l2_evict_first_policy();
   const uint64_t keep_policy = l2_evict_normal_policy();
   const int total = cta_units(p);
   auto unit_of = [&](int i) { return cta_unit(p, i); };
-  // pointer words (and flush masks) 32 units at a time, one chunk ahead: lane j of a
-  // chunk holds the word of the chunk's j-th unit
+  auto tst_of = [&](int i) { return tstages + (size_t)(i % NT) * p.tstage_bytes; };
+  auto rst_of = [&](int i) { return rstages + (size_t)(i % NR) * p.rstage_bytes; };
+  // pointer words (and flush masks) of the record units, 32 at a time, one chunk ahead:
+  // lane j of a chunk holds the word of the chunk's j-th unit
   auto load_words = [&](int i0, int32_t& w, int& msk) {
     w = 0;
     msk = 1;
@@ -315,54 +328,41 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
       if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
     }
   };
-  auto arm = [&](uint8_t* st, int s, const Plan& pl, int32_t word, int msk) {
-    reinterpret_cast<int32_t*>(st + p.off_meta)[0] = word;
-    reinterpret_cast<int32_t*>(st + p.off_meta)[1] = msk;
-    if (pl.corrupt) report_error(p.status, kErrPointer);
-    mbar_arrive_expect_tx(&bars->tfull[s], pl.tile_bytes);
-    mbar_arrive_expect_tx(&bars->rfull[s], pl.rec_bytes);
-  };
   int32_t w_cur, w_nxt;
   int m_cur, m_nxt;
   load_words(0, w_cur, m_cur);
   load_words(32, w_nxt, m_nxt);
-  const int j = lane / kCopyKinds;     // this lane's unit within the batch
+  const int j = lane / kCopyKinds;     // this lane's step within the batch
   const int kind = lane % kCopyKinds;  // and its copy
-  // When the kernel appends this call's entries itself, the first stages' state tiles
-  // (and FP8 scales) go out at once and their records and queries once the entries are
-  // in the ring; every stage is armed with its unit's byte counts either way.
-  int pre = 0;
-  if (APPEND && p.append_here) {
-    pre = min(NS, total);
-    for (int i = 0; i < pre; ++i) {
-      const int32_t word = __shfl_sync(0xffffffffu, w_cur, i & 31);
-      const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), word, 1);
-      uint8_t* st = stages + (size_t)i * p.stage_bytes;
-      if (lane == 0) arm(st, i, pl, word, 1);
-      __syncwarp();
-      const uint8_t* src;
-      uint8_t* dst;
-      uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, st, lane, src, dst);
-      if (lane > 1) bytes = 0;
-      __syncwarp();
-      if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->tfull[i], lane == 0 ? stream_policy : keep_policy);
-      if (lane == 0) bars->last_fill[i] = i;
-    }
-    group_sync(kAppendBar, kThreads);  // the entries are in the ring
+  const int pre = min(NT, total);      // tiles issued up front
+  for (int i = 0; i < pre; ++i) {
+    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), __shfl_sync(0xffffffffu, w_cur, i),
+                                               __shfl_sync(0xffffffffu, m_cur, i));
+    if (lane == 0) mbar_arrive_expect_tx(&bars->tfull[i], pl.tile_bytes);
+    __syncwarp();
+    const uint8_t* src;
+    uint8_t* dst;
+    uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, tst_of(i), rst_of(i), lane, src, dst);
+    if (lane > 1) bytes = 0;
+    __syncwarp();
+    if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->tfull[i], lane == 0 ? stream_policy : keep_policy);
+    if (lane == 0) bars->last_tfill[i] = i;
   }
-  for (int i0 = 0; i0 < total; i0 += U) {
-    if ((i0 & 31) == 0 && i0 > 0) {
+  if (APPEND && p.append_here) group_sync(kAppendBar, kThreads);  // the entries are in the ring
+  for (int t0 = 0; t0 < total + D; t0 += U) {
+    if ((t0 & 31) == 0 && t0 > 0) {
       w_cur = w_nxt;
       m_cur = m_nxt;
-      load_words(i0 + 32, w_nxt, m_nxt);
+      load_words(t0 + 32, w_nxt, m_nxt);
     }
-    // every lane waits for the batch's stages (each lane then writes into one), the
-    // warp agrees
+    // every lane waits for the batch's stages, the warp agrees
     bool ready = true;
 #pragma unroll
     for (int jj = 0; jj < U; ++jj) {
-      const int i = i0 + jj;
-      if (i < total && i >= NS) ready = ready && mbar_wait_bounded(&bars->empty[i % NS], ((i / NS) - 1) & 1);
+      const int r = t0 + jj;      // record unit
+      const int u = t0 + jj - D;  // tile unit
+      if (r < total && r >= NR) ready = ready && mbar_wait_bounded(&bars->rempty[r % NR], ((r / NR) - 1) & 1);
+      if (u >= pre && u < total && u >= NT) ready = ready && mbar_wait_bounded(&bars->tempty[u % NT], ((u / NT) - 1) & 1);
     }
     if (!__all_sync(0xffffffffu, ready)) {
       if (lane == 0) {
@@ -373,53 +373,83 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     }
     const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
     if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
-    const int i = i0 + j;
-    const bool valid = j < U && i < total;
-    const int32_t word = __shfl_sync(0xffffffffu, w_cur, i & 31);
-    const int msk = __shfl_sync(0xffffffffu, m_cur, i & 31);
-    const int s = i % NS;
-    uint8_t* st = stages + (size_t)s * p.stage_bytes;
-    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), word, msk);
-    const bool armed = i < pre;  // tile already issued, stage already armed
-    if (valid && kind == 0 && !armed) arm(st, s, pl, word, msk);
+    const int r = t0 + j;
+    const int u = t0 + j - D;
+    const bool rec_step = j < U && r < total;
+    const bool tile_step = j < U && u >= pre && u < total;
+    // record side: the unit's pointer word and flush mask from the prefetched chunk
+    const int32_t word_r = __shfl_sync(0xffffffffu, w_cur, r & 31);
+    const int msk_r = __shfl_sync(0xffffffffu, m_cur, r & 31);
+    uint8_t* rst = rst_of(r);
+    const Plan plr = make_plan<MODE, CKPT, S_IO>(p, unit_of(r), word_r, msk_r);
+    if (rec_step && kind == 2) {
+      reinterpret_cast<int32_t*>(rst + p.off_meta)[0] = word_r;
+      reinterpret_cast<int32_t*>(rst + p.off_meta)[1] = msk_r;
+      if (plr.corrupt) report_error(p.status, kErrPointer);
+      mbar_arrive_expect_tx(&bars->rfull[r % NR], plr.rec_bytes);
+    }
+    __syncwarp();  // a record stage armed in this step may hold a tile unit's word (lookahead < batch)
+    // tile side: the pointer word from the unit's record stage
+    int32_t word_u = 0;
+    int msk_u = 1;
+    if (tile_step && kind <= 1) {
+      const uint8_t* rsu = rst_of(u);
+      word_u = reinterpret_cast<const int32_t*>(rsu + p.off_meta)[0];
+      msk_u = reinterpret_cast<const int32_t*>(rsu + p.off_meta)[1];
+    }
+    uint8_t* tst = tst_of(u < 0 ? 0 : u);
+    const Plan plt = make_plan<MODE, CKPT, S_IO>(p, unit_of(u < 0 ? 0 : u), word_u, msk_u);
+    if (tile_step && kind == 0) mbar_arrive_expect_tx(&bars->tfull[u % NT], plt.tile_bytes);
     __syncwarp();
     const uint8_t* src;
     uint8_t* dst;
-    uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, st, kind, src, dst);
-    if (!valid || (armed && kind <= 1)) bytes = 0;
+    uint32_t bytes = 0;
+    if (kind <= 1) {
+      bytes = unit_copy<MODE, CKPT, S_IO>(p, plt, tst, rst, kind, src, dst);
+      if (!tile_step) bytes = 0;
+    } else {
+      bytes = unit_copy<MODE, CKPT, S_IO>(p, plr, tst, rst, kind, src, dst);
+      if (!rec_step) bytes = 0;
+    }
     __syncwarp();
     if (bytes)
-      bulk_g2s_hint(dst, src, bytes, kind <= 1 ? &bars->tfull[s] : &bars->rfull[s],
+      bulk_g2s_hint(dst, src, bytes, kind <= 1 ? &bars->tfull[u % NT] : &bars->rfull[r % NR],
                     kind == 0 ? stream_policy : keep_policy);
-    if (valid && kind == 0) bars->last_fill[s] = i;
+    if (tile_step && kind == 0) bars->last_tfill[u % NT] = u;
+    if (rec_step && kind == 2) bars->last_rfill[r % NR] = r;
   }
   // Never leave with copies in flight into this CTA's shared memory: wait (bounded) for
   // the latest fill of every stage.
   __syncwarp();
-  for (int st_i = 0; st_i < NS; ++st_i) {
-    const int i = bars->last_fill[st_i];
-    if (i < 0) continue;
-    const bool ok = mbar_wait_bounded(&bars->tfull[st_i], (i / NS) & 1) &&
-                    mbar_wait_bounded(&bars->rfull[st_i], (i / NS) & 1);
-    if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
+  bool ok = true;
+  for (int st_i = 0; st_i < NT; ++st_i) {
+    const int i = bars->last_tfill[st_i];
+    if (i >= 0) ok = mbar_wait_bounded(&bars->tfull[st_i], (i / NT) & 1) && ok;
   }
+  for (int st_i = 0; st_i < NR; ++st_i) {
+    const int i = bars->last_rfill[st_i];
+    if (i >= 0) ok = mbar_wait_bounded(&bars->rfull[st_i], (i / NR) & 1) && ok;
+  }
+  if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
 }
 
-// The eager baseline's producer: one unit at a time; the tile (and FP8 scales) by bulk
-// copy on tfull, the new token's k, v, Delta, a and q gathered with per-lane cp.async,
-// each lane arriving on rfull once its copies have landed.
+// The eager baseline's producer: one unit at a time, no lookahead (its coefficients are
+// two numbers); the tile (and FP8 scales) by bulk copy on tfull, the new token's k, v,
+// Delta, a and q gathered with per-lane cp.async into the record stage, each lane arriving
+// on rfull once its copies have landed.
 template <int CKPT, int S_IO>
-__device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bars) {
+__device__ void producer_loop_eager(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars) {
   const int lane = threadIdx.x & 31;
-  const int NS = p.num_stages;
+  const int NT = p.num_tstages, NR = p.num_rstages;
   const uint64_t stream_policy = l2_evict_first_policy();
   const size_t P = p.P, N = p.N;
   const int total = cta_units(p);
   for (int i = 0; i < total; ++i) {
     const int u = cta_unit(p, i);
-    const int s = i % NS;
-    const int k = i / NS;
-    if (k > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1))) {
+    bool ready = true;
+    if (i >= NT) ready = mbar_wait_bounded(&bars->tempty[i % NT], ((i / NT) - 1) & 1);
+    if (ready && i >= NR) ready = mbar_wait_bounded(&bars->rempty[i % NR], ((i / NR) - 1) & 1);
+    if (!__all_sync(0xffffffffu, ready)) {
       if (lane == 0) {
         report_error(p.status, kErrWaitTimeout);
         bars->abort_flag = 1;
@@ -429,27 +459,28 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bar
     const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
     if (__shfl_sync(0xffffffffu, ab, 0)) break;
     const Plan pl = make_plan<kModeEager, CKPT, S_IO>(p, u, 0, 1);
-    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint8_t* tst = tstages + (size_t)(i % NT) * p.tstage_bytes;
+    uint8_t* rst = rstages + (size_t)(i % NR) * p.rstage_bytes;
     const size_t bh = (size_t)pl.b * p.H + pl.h;
     const size_t bg = (size_t)pl.b * p.G + pl.g;
     const size_t row0 = bh * P + pl.r0;  // the unit's rows
     const uint32_t rows = (uint32_t)pl.rows;
     constexpr size_t kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;
-    uint8_t* recbuf = st + p.off_rec;
-    uint8_t* kbuf = st + p.off_krec;
-    if (lane == 0) mbar_arrive_expect_tx(&bars->tfull[s], pl.tile_bytes);
+    uint8_t* recbuf = rst + p.off_rec;
+    uint8_t* kbuf = rst + p.off_krec;
+    if (lane == 0) mbar_arrive_expect_tx(&bars->tfull[i % NT], pl.tile_bytes);
     __syncwarp();
     if (lane == 0)
-      bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + row0 * N) : (const void*)(p.S8 + row0 * (N / kCodeDiv)),
-                    pl.fp32_tile ? (uint32_t)(rows * N * 4) : (uint32_t)(rows * (N / kCodeDiv)), &bars->tfull[s],
+      bulk_g2s_hint(tst, pl.fp32_tile ? (const void*)(p.S + row0 * N) : (const void*)(p.S8 + row0 * (N / kCodeDiv)),
+                    pl.fp32_tile ? (uint32_t)(rows * N * 4) : (uint32_t)(rows * (N / kCodeDiv)), &bars->tfull[i % NT],
                     stream_policy);
     if (lane == 1 && !pl.fp32_tile)
-      bulk_g2s(st + (size_t)p.rows_unit * (N / kCodeDiv), p.Sscale + row0, rows * 4u, &bars->tfull[s]);
+      bulk_g2s(tst + (size_t)p.rows_unit * (N / kCodeDiv), p.Sscale + row0, rows * 4u, &bars->tfull[i % NT]);
     const int kpe = (int)(N * S_IO / 16);
     const int vpe = (int)(P * S_IO / 16);
     for (int idx = lane; idx < 2 * kpe + vpe; idx += 32) {
       if (idx < kpe) {
-        cp_async16(st + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
+        cp_async16(rst + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
       } else if (idx < 2 * kpe) {
         const int ch = idx - kpe;
         cp_async16(kbuf + ch * 16, static_cast<const uint8_t*>(p.k) + bg * N * S_IO + ch * 16);
@@ -460,17 +491,23 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bar
     }
     if (lane == 0) cp_async4(recbuf + P * S_IO, p.dt + bh);
     if (lane == 1) cp_async4(recbuf + P * S_IO + 4, p.a + bh);
-    cp_async_arrive(&bars->rfull[s]);
-    if (lane == 0) bars->last_fill[s] = i;
+    cp_async_arrive(&bars->rfull[i % NR]);
+    if (lane == 0) {
+      bars->last_tfill[i % NT] = i;
+      bars->last_rfill[i % NR] = i;
+    }
   }
   __syncwarp();
-  for (int st_i = 0; st_i < NS; ++st_i) {
-    const int i2 = bars->last_fill[st_i];
-    if (i2 < 0) continue;
-    const bool ok = mbar_wait_bounded(&bars->tfull[st_i], (i2 / NS) & 1) &&
-                    mbar_wait_bounded(&bars->rfull[st_i], (i2 / NS) & 1);
-    if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
+  bool ok = true;
+  for (int st_i = 0; st_i < NT; ++st_i) {
+    const int i2 = bars->last_tfill[st_i];
+    if (i2 >= 0) ok = mbar_wait_bounded(&bars->tfull[st_i], (i2 / NT) & 1) && ok;
   }
+  for (int st_i = 0; st_i < NR; ++st_i) {
+    const int i2 = bars->last_rfill[st_i];
+    if (i2 >= 0) ok = mbar_wait_bounded(&bars->rfull[st_i], (i2 / NR) & 1) && ok;
+  }
+  if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
 }
 
 // ---------------------------------------------------------------------------- coefficients
@@ -642,32 +679,30 @@ __device__ __forceinline__ void coef_unit(const KParams& p, const Plan& pl, uint
   }
 }
 
-// The coefficient warps' loop: the units of a k/q group (its heads, each with its row
-// blocks) all go to one warp, groups in turn, so that the warp forms the group's k . q
-// once. A warp's consecutive units may lie any distance apart, so its parity waits are
-// made exact by counting: before it waits for the k-th use of a stage it waits until the
-// row warps' releases of that stage's use k-2 have all been counted (the row warps take
-// the units in order and cannot be two uses further on, since they need this warp's
-// coefficients for use k). Then it waits for the stage's previous release (empty, phase
-// k-1), after which no one touches the stage, and for its records (rfull, phase k),
-// whose phase k-1 completed before the row warps could release use k-1. Each warp takes
-// its units in order, so no wait can close a cycle.
+// The coefficient warps' loop, on the record ring: the units of a chunk (heads of one k/q
+// group, each with its row blocks) all go to one warp, chunks in turn, so that the warp
+// forms the group's k . q once per chunk. A warp's consecutive units may lie any distance
+// apart, so its parity waits are made exact by counting: before it waits for the k-th use
+// of a record stage it waits until the row warps' releases of that stage's use k-2 have
+// all been counted (the row warps take the units in order and cannot be two uses further
+// on, since they need this warp's coefficients for use k). Then it waits for the stage's
+// previous release (rempty, phase k-1), after which no one else touches the stage, and
+// for its records (rfull, phase k), whose phase k-1 completed before the row warps could
+// release use k-1. Each warp takes its units in order, so no wait can close a cycle.
 template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ void coef_loop(const KParams& p, uint8_t* stages, Bars* bars, float* kq, float* cw, int cwarp, int lane) {
+__device__ void coef_loop(const KParams& p, uint8_t* rstages, Bars* bars, float* kq, float* cw, int cwarp, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  const int NS = p.num_stages;
+  const int NR = p.num_rstages;
   const int total = cta_units(p);
-  const int bh0 = cta_first_head(p);
-  const int key0 = bh0 / p.hpg;
-  int cached = -1;  // the group (b * G + g) whose k . q the warp holds in kq
+  int cached = -1;  // the CTA-local chunk whose k . q products the warp holds in kq
   for (int i = 0; i < total; ++i) {
-    const int key = (bh0 + (i >> p.rb_shift)) / p.hpg;
-    if ((key - key0) % kCoefWarps != cwarp) continue;
-    const int s = i % NS;
-    const int k = i / NS;
+    const int key = unit_chunk(p, i);
+    if (key % kCoefWarps != cwarp) continue;
+    const int s = i % NR;
+    const int k = i / NR;
     bool ready = *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
     if (ready && k > 1) ready = wait_released(&bars->released[s], (k - 1) * kRowWarps, lane);
-    if (ready && k > 0) ready = mbar_wait_bounded(&bars->empty[s], (k - 1) & 1);
+    if (ready && k > 0) ready = mbar_wait_bounded(&bars->rempty[s], (k - 1) & 1);
     if (ready) ready = mbar_wait_bounded(&bars->rfull[s], k & 1);
     if (!__all_sync(0xffffffffu, ready)) {
       if (lane == 0) {
@@ -676,7 +711,7 @@ __device__ void coef_loop(const KParams& p, uint8_t* stages, Bars* bars, float* 
       }
       break;
     }
-    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint8_t* st = rstages + (size_t)s * p.rstage_bytes;
     const int32_t word = reinterpret_cast<const int32_t*>(st + p.off_meta)[0];
     const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, cta_unit(p, i), word, msk);
@@ -715,7 +750,8 @@ __device__ void coef_loop(const KParams& p, uint8_t* stages, Bars* bars, float* 
 // x + sum_j wt[j][rows] k_j[cols] in registers, the write-back (FP32 master and/or FP8
 // codes with per-row scales), then the outputs from the fresh rows.
 template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ __forceinline__ void row_unit(const KParams& p, const Plan& pl, const uint8_t* st, int warp, int lane) {
+__device__ __forceinline__ void row_unit(const KParams& p, const Plan& pl, const uint8_t* tst, const uint8_t* st, int warp,
+                                         int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
   constexpr int TPR = N / 4;
   constexpr int RPW = 32 / TPR;  // rows per warp pass
@@ -729,7 +765,7 @@ __device__ __forceinline__ void row_unit(const KParams& p, const Plan& pl, const
   const int r0 = pl.r0;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
   const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? pl.c : 0);
-  const uint8_t* tile = st;
+  const uint8_t* tile = tst;  // the tile stage; records, queries and coefficients in the record stage `st`
   const uint8_t* qbuf = st + p.off_q;
   constexpr int kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;  // read copy: code bytes per row = N / kCodeDiv
   const Records<N, S_IO> rec{st + p.off_krec, st + p.off_rec, PH, p.rec_bytes, p.rec_k_bytes};
@@ -852,20 +888,20 @@ __device__ __forceinline__ void row_unit(const KParams& p, const Plan& pl, const
   }
 }
 
-// The row warps' loop: every row warp takes every unit of the CTA, waiting for the
-// stage's tile (tfull) and its coefficients (cready), phase k of each; the warp's own
-// wait for phase k-1 of both came first, so both parity waits are exact.
+// The row warps' loop: every row warp takes every unit of the CTA in order, waiting for
+// the unit's tile (tfull) and its coefficients (cready); the warp's own waits for the
+// uses before came first, so both parity waits are exact. Releasing a unit frees its
+// tile stage and its record stage, and counts the release for the coefficient warps.
 template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ void row_loop(const KParams& p, uint8_t* stages, Bars* bars, int warp, int lane) {
+__device__ void row_loop(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars, int warp, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  const int NS = p.num_stages;
+  const int NT = p.num_tstages, NR = p.num_rstages;
   const int total = cta_units(p);
   for (int i = 0; i < total; ++i) {
-    const int s = i % NS;
-    const int k = i / NS;  // this is the k-th use of stage s
+    const int st_t = i % NT, st_r = i % NR;
     bool ready = *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
-    if (ready) ready = mbar_wait_bounded(&bars->tfull[s], k & 1);
-    if (ready) ready = mbar_wait_bounded(&bars->cready[s], k & 1);
+    if (ready) ready = mbar_wait_bounded(&bars->tfull[st_t], (i / NT) & 1);
+    if (ready) ready = mbar_wait_bounded(&bars->cready[st_r], (i / NR) & 1);
     if (!__all_sync(0xffffffffu, ready)) {
       if (lane == 0) {
         report_error(p.status, kErrWaitTimeout);
@@ -873,13 +909,15 @@ __device__ void row_loop(const KParams& p, uint8_t* stages, Bars* bars, int warp
       }
       break;
     }
-    const uint8_t* st = stages + (size_t)s * p.stage_bytes;
-    const int32_t word = reinterpret_cast<const int32_t*>(st + p.off_meta)[0];
-    const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
+    const uint8_t* tst = tstages + (size_t)st_t * p.tstage_bytes;
+    const uint8_t* rst = rstages + (size_t)st_r * p.rstage_bytes;
+    const int32_t word = reinterpret_cast<const int32_t*>(rst + p.off_meta)[0];
+    const int msk = reinterpret_cast<const int32_t*>(rst + p.off_meta)[1];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, cta_unit(p, i), word, msk);
-    if (pl.active) row_unit<N, IO, CKPT, MODE, NQ>(p, pl, st, warp, lane);
-    count_release(&bars->released[s], lane);
-    mbar_arrive(&bars->empty[s]);
+    if (pl.active) row_unit<N, IO, CKPT, MODE, NQ>(p, pl, tst, rst, warp, lane);
+    count_release(&bars->released[st_r], lane);
+    mbar_arrive(&bars->rempty[st_r]);
+    mbar_arrive(&bars->tempty[st_t]);
   }
 }
 
@@ -888,19 +926,24 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   static_assert(kProducerWarps == 1, "stages must be filled in unit order");
   extern __shared__ __align__(128) uint8_t smem[];
   Bars* bars = reinterpret_cast<Bars*>(smem);
-  uint8_t* stages = smem + p.stages_off;
+  uint8_t* tstages = smem + p.tstages_off;
+  uint8_t* rstages = smem + p.rstages_off;
   constexpr int S_IO = IoT<IO>::bytes;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.num_stages; ++s) {
-      mbar_init(&bars->tfull[s], 1);                             // the producer's expect_tx
-      mbar_init(&bars->rfull[s], MODE == kModeEager ? 32 : 1);   // the eager gather: 32 lanes' cp.async
-      mbar_init(&bars->cready[s], 32);                           // a coefficient warp's lanes
-      mbar_init(&bars->empty[s], kRowWarps * 32);                // every row warp's lanes
+    for (int s = 0; s < p.num_tstages; ++s) {
+      mbar_init(&bars->tfull[s], 1);                  // the producer's expect_tx
+      mbar_init(&bars->tempty[s], kRowWarps * 32);    // every row warp's lanes
+    }
+    for (int s = 0; s < p.num_rstages; ++s) {
+      mbar_init(&bars->rfull[s], MODE == kModeEager ? 32 : 1);  // the eager gather: 32 lanes' cp.async
+      mbar_init(&bars->cready[s], 32);                // a coefficient warp's lanes
+      mbar_init(&bars->rempty[s], kRowWarps * 32);    // every row warp's lanes
     }
     bars->abort_flag = 0;
-    for (int s = 0; s < kMaxStages; ++s) {
-      bars->last_fill[s] = -1;
+    for (int s = 0; s < kMaxTileStages; ++s) bars->last_tfill[s] = -1;
+    for (int s = 0; s < kMaxRecStages; ++s) {
+      bars->last_rfill[s] = -1;
       bars->released[s] = 0;
     }
     fence_mbar_init();
@@ -908,8 +951,8 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   __syncthreads();
   if constexpr (MODE == kModeReplay && NQ == 1) {
     // One-position calls append their entries here rather than in a pre-pass: the row and
-    // coefficient warps write the new ring record of each of the CTA's own units (k, v,
-    // then Delta and a in one 16-byte piece), make the writes visible to the bulk copies
+    // coefficient warps write the new ring records of the CTA's heads (v, then Delta and a
+    // in one 16-byte piece; k once per chunk), make the writes visible to the bulk copies
     // that read them, and tell the producer, which meanwhile streams the first tiles.
     if (p.append_here && threadIdx.x < kWorkerWarps * 32) {
       append_entries<S_IO>(p);
@@ -921,15 +964,15 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   const int lane = threadIdx.x & 31;
   if (warp >= kWorkerWarps) {
     if constexpr (MODE == kModeEager)
-      producer_loop_eager<CKPT, S_IO>(p, stages, bars);
+      producer_loop_eager<CKPT, S_IO>(p, tstages, rstages, bars);
     else
-      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, stages, bars);
+      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, tstages, rstages, bars);
   } else if (warp >= kRowWarps) {
     const int cwarp = warp - kRowWarps;
     float* kq = reinterpret_cast<float*>(smem + p.ws_off + (size_t)cwarp * p.ws_bytes);
-    coef_loop<N, IO, CKPT, MODE, NQ>(p, stages, bars, kq, kq + p.ws_bytes / 8, cwarp, lane);
+    coef_loop<N, IO, CKPT, MODE, NQ>(p, rstages, bars, kq, kq + p.ws_bytes / 8, cwarp, lane);
   } else {
-    row_loop<N, IO, CKPT, MODE, NQ>(p, stages, bars, warp, lane);
+    row_loop<N, IO, CKPT, MODE, NQ>(p, tstages, rstages, bars, warp, lane);
   }
 }
 

@@ -13,8 +13,10 @@ struct KParams {
   int32_t B, H, G, P, N, L, cap, n_pos, hpg;
   // units: a unit is rows [rb * rows_unit, min(P, (rb + 1) * rows_unit)) of one head of one
   // sequence, u = (b * H + h) * row_blocks + rb with row_blocks = 1 << rb_shift (1 or 2);
-  // all row blocks of a head go to one CTA
+  // all row blocks of a head go to one CTA. Heads are dealt to CTAs in chunks of
+  // chunk_heads consecutive heads of one k/q group (chunk c to CTA c mod grid).
   int32_t rows_unit, row_blocks, rb_shift, num_bh, num_units;
+  int32_t chunk_heads, num_chunks;
   int32_t commit;  // replay: 1 = step (new entries committed), 0 = verify (tentative)
   int32_t fold_min;     // flush: fold only buffers holding at least this many entries (>= 1)
   int32_t flushed_or;   // replay: OR this call's fold flags into `flushed` (a flush before it wrote them)
@@ -38,10 +40,13 @@ struct KParams {
   const int32_t* counts_in;
   int32_t* counts_out;
   int32_t* status;
-  // shared-memory layout, bytes
-  int32_t num_stages, stage_bytes, stages_off;
+  // shared-memory layout, bytes: a ring of tile stages and a deeper ring of record stages
+  // (records, queries, pointer word, coefficients); a unit's records are copied
+  // `lookahead` units before its tile
+  int32_t num_tstages, tstage_bytes, tstages_off;
+  int32_t num_rstages, rstage_bytes, rstages_off, lookahead;
   int32_t rec_bytes, rec_k_bytes, qpack_pos;   // head / k record sizes; positions per qpack group
-  int32_t off_krec, off_rec, off_q, off_meta, off_coef;  // within a stage
+  int32_t off_krec, off_rec, off_q, off_meta, off_coef;  // within a record stage
   int32_t co_alpha, co_sig, co_u, co_wt;       // within a stage's coefficient area
   int32_t u_stride, wt_stride;                 // floats per position of u, per entry of wt (= rows_unit)
   int32_t ws_off, ws_bytes;                    // one scratch area per coefficient warp

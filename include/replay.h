@@ -100,7 +100,7 @@ typedef struct {
  * The buffer of recent inputs is a ring of `cap` records per sequence: one k record per
  * k/q group and one record per head. A group's heads share its k (blog, end of "Ruta
  * 'solo salida'": k and q belong to the group), so k is stored once per group. k record
- * j of (b, g): RK bytes, k (N io values). Head record j of (b, h): R bytes, v (P io values),
+ * j of (b, g): RK bytes, k (N io values) then padding. Head record j of (b, h): R bytes, v (P io values),
  * Delta (FP32), a (FP32), zero padding to a multiple of 16 bytes. Keeping an entry's pieces
  * together lets a unit's whole buffer arrive in one or two bulk copies per ring. */
 typedef struct {
@@ -128,8 +128,9 @@ int32_t replay_ring_capacity(const replay_config* cfg);
  * (FP32). Returns a negative replay_status on a bad config. */
 int32_t replay_ring_record_bytes(const replay_config* cfg);
 
-/* Bytes of one k record: N*s (a multiple of 16). Returns a negative replay_status on a
- * bad config. */
+/* Bytes of one k record: N*s + 16 (k, then 16 bytes of padding that keep consecutive
+ * records on different shared-memory banks inside the kernel). Returns a negative
+ * replay_status on a bad config. */
 int32_t replay_ring_k_record_bytes(const replay_config* cfg);
 
 /* Validates cfg and bufs, zeroes both halves of counts (every buffer empty) and the

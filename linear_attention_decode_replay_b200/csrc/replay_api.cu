@@ -60,7 +60,11 @@ int record_bytes(const replay_config& c) {
   const int s_io = c.io == REPLAY_BF16 ? 2 : 4;
   return round_up(c.P * s_io + 8, 16);
 }
-int record_k_bytes(const replay_config& c) { return c.N * (c.io == REPLAY_BF16 ? 2 : 4); }
+// k record: k (N io values), then 16 bytes of padding. The padding staggers consecutive
+// records by four shared-memory banks once a unit's records sit in a stage, so that the
+// lanes that read several entries' k at once (one entry per lane pair or quarter) spread
+// over all 32 banks; without it every record starts on the same bank.
+int record_k_bytes(const replay_config& c) { return c.N * (c.io == REPLAY_BF16 ? 2 : 4) + 16; }
 int ckpt_kind(int ckpt) {
   return ckpt == REPLAY_CKPT_F32_FP8READ ? replay::kCkptFp8 : ckpt == REPLAY_CKPT_F32_FP4READ ? replay::kCkptFp4
                                                                                               : replay::kCkptF32;
@@ -105,57 +109,35 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   // a unit is one row group of a head (all of it when P is smaller): its tile is at most
   // 64 rows x 128 floats, whatever P
   const int UR = P < replay::row_group_rows(N) ? P : replay::row_group_rows(N);
-  // tile stage: the unit's FP32 rows (a read copy's codes and scales fit in the same space)
+  // stage: the unit's FP32 rows (a read copy's codes and scales fit in the same space),
+  // then its k records, head records, queries and pointer word
   const int tile = fp8_eager ? round_up(UR * N + UR * 4, 16) : UR * N * 4;
-  p->tstage_bytes = round_up(tile, 128);
-  // record stage: k records, head records, queries, pointer word, then the coefficient
-  // area a coefficient warp writes for the row warps: alpha[kMaxPos], the fold weights
-  // [kMaxWindow] + abar, the buffer terms u[nq][UR] and the fold weight table wt[lfold][UR]
-  // (a unit's rows, zero past the head's)
-  p->off_krec = 0;
+  p->off_krec = round_up(tile, 16);
   p->off_rec = p->off_krec + jmax * p->rec_k_bytes;
   p->off_q = p->off_rec + jmax * p->rec_bytes;
   p->off_meta = p->off_q + round_up(nq_alloc * N * s_io, 16);
-  p->off_coef = p->off_meta + 16;
-  p->co_alpha = 0;
-  p->co_sig = replay::kMaxPos * 4;
-  p->co_u = round_up(p->co_sig + (replay::kMaxWindow + 1) * 4, 16);
-  p->u_stride = UR;
-  p->co_wt = round_up(p->co_u + nq_alloc * UR * 4, 16);
-  p->wt_stride = UR;
-  p->rstage_bytes = round_up(p->off_coef + p->co_wt + lfold * UR * 4, 128);
+  p->stage_bytes = round_up(p->off_meta + 32, 128);  // meta: word, mask, b, h, g, rb
 
-  // one scratch area per coefficient warp: the group's k . q products and the head's entry
-  // coefficients, [nq][kMaxWindow] each
+  // one workspace per consumer group: alpha[kMaxPos], the fold weights [kMaxWindow] +
+  // abar, the outputs' entry coefficients [kMaxPos][kMaxWindow], the raw k . q products
+  // [kMaxPos][kMaxWindow] (kept for the group's next unit of the same chunk), and the
+  // fold weights times v, [lfold][wt_stride] (a unit's rows, padded to a multiple of
+  // kRowsPerThread)
+  p->wt_stride = round_up(UR, replay::kRowsPerThread);
+  p->ws_alpha = 0;
+  p->ws_sig = p->ws_alpha + replay::kMaxPos * 4;
+  p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
+  p->ws_kq = p->ws_cw + replay::kMaxPos * replay::kMaxWindow * 4;
+  p->ws_wt = round_up(p->ws_kq + replay::kMaxPos * replay::kMaxWindow * 4, 16);
+  p->ws_group_bytes = round_up(p->ws_wt + lfold * p->wt_stride * 4, 128);
   p->ws_off = kHeaderBytes;
-  p->ws_bytes = 2 * (nq_alloc > 0 ? nq_alloc : 1) * replay::kMaxWindow * 4;
-  p->tstages_off = round_up(p->ws_off + replay::kCoefWarps * p->ws_bytes, 128);
-  const int avail = smem_optin - p->tstages_off;
-  // Stage counts: as many tile stages as leave room for a record ring that runs ahead of
-  // them by min(tile stages, 4) units (the lookahead that hides the coefficient warps'
-  // chain behind the tiles in flight); the eager launch needs no lookahead.
-  int nt = 0, nr = 0;
-  for (int t = replay::kMaxTileStages; t >= 2 && !nt; --t) {
-    const int want = mode == replay::kModeEager ? t : t + (t < 4 ? t : 4);
-    int r = (avail - t * p->tstage_bytes) / p->rstage_bytes;
-    if (r > replay::kMaxRecStages) r = replay::kMaxRecStages;
-    if (r >= want) {
-      nt = t;
-      nr = r;
-    }
-  }
-  if (!nt) {  // not even two tile stages with their lookahead: two and what fits
-    nt = 2;
-    nr = (avail - 2 * p->tstage_bytes) / p->rstage_bytes;
-    if (nr > replay::kMaxRecStages) nr = replay::kMaxRecStages;
-    if (nr < 2) return REPLAY_EINVAL;
-  }
-  p->num_tstages = nt;
-  p->num_rstages = nr;
-  p->lookahead = mode == replay::kModeEager ? 0 : (nr - nt < nt ? nr - nt : nt);
-  if (p->lookahead < 0) p->lookahead = 0;
-  p->rstages_off = p->tstages_off + nt * p->tstage_bytes;
-  p->smem_bytes = p->rstages_off + nr * p->rstage_bytes;
+  p->stages_off = round_up(p->ws_off + replay::kGroups * p->ws_group_bytes, 128);
+  const int avail = smem_optin - p->stages_off;
+  int ns = avail / p->stage_bytes;
+  if (ns > replay::kMaxStages) ns = replay::kMaxStages;
+  if (ns < 2) return REPLAY_EINVAL;
+  p->num_stages = ns;
+  p->smem_bytes = p->stages_off + ns * p->stage_bytes;
 
   p->B = c.batch;
   p->H = c.heads;

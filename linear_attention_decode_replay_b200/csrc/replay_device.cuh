@@ -10,26 +10,25 @@
 
 namespace replay {
 
-constexpr int kRowWarps = 8;                     // warps that stream a unit's state rows
-constexpr int kCoefWarps = 7;                    // warps that form the units' coefficients and buffer terms
-                                                 // (16 warps in all: 4 per scheduler, 128 registers each)
-constexpr int kWorkerWarps = kRowWarps + kCoefWarps;
+constexpr int kGroupGemvWarps = 4;               // per consumer group: warps that stream the state rows
+constexpr int kGroupWarps = kGroupGemvWarps + 1; // ... plus one warp for the decay weights and k . q
+constexpr int kGroups = 2;                       // consumer groups per CTA
+constexpr int kConsumerWarps = kGroups * kGroupWarps;
 constexpr int kProducerWarps = 1;                // the warp that fills stages, in unit order
-constexpr int kThreads = (kWorkerWarps + kProducerWarps) * 32;
+constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
 constexpr int kMaxPos = 8;                       // query positions per verify call
 constexpr int kMaxWindow = 32;                   // largest L (decay scans use one warp)
-constexpr int kMaxTileStages = 8;                // ring of state tiles
-constexpr int kMaxRecStages = 16;                // ring of records, queries and coefficients
+constexpr int kMaxStages = 8;
 constexpr int kMaxChunkHeads = 8;                // heads of one k/q group a CTA takes in a row
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
 constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
-constexpr int kRowsPerThread = 8;                // state rows one thread covers in a unit
-constexpr int kHeaderBytes = 1024;               // the mbarriers and flags at the start of shared memory
-// State rows of one unit: kRowWarps warps, 128/N rows per warp pass (a row of N floats
-// takes N/4 lanes), kRowsPerThread rows per lane. A unit covers this many rows of a head
-// (or the whole head when it has fewer), so that every unit's tile is at most 32 KiB of
-// FP32 and as many stages fit in shared memory whatever the head's P.
-constexpr int row_group_rows(int N) { return kRowWarps * (128 / N) * kRowsPerThread; }
+constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
+constexpr int kHeaderBytes = 256;                // the mbarriers and flags at the start of shared memory
+// State rows of one row group: kGroupGemvWarps warps, 128/N rows per warp pass (a row of
+// N floats takes N/4 lanes), kRowsPerThread rows per lane. A unit covers one row group of
+// a head (or the whole head when it has fewer rows), so that every unit's tile is at most
+// 32 KiB of FP32 and as many stages fit in shared memory whatever the head's P.
+constexpr int row_group_rows(int N) { return kGroupGemvWarps * (128 / N) * kRowsPerThread; }
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at the boost clock
 
 // status word bits (device-detected errors; the host reads them with replay_check_status)

@@ -19,7 +19,7 @@ constexpr int kMaxDevices = 64;
 
 template <typename IO, int CKPT, int MODE, int NQ>
 cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
-  auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ>;
+  auto kern = replay_kernel<REPLAY_N, IO, CKPT, MODE, NQ, kGroups>;  // NG: the host layout reserves one workspace per group
   // the dynamic shared-memory opt-in is per function and device; remember the largest set
   // (under a lock: calls may come from several threads, and a smaller concurrent setting
   // must not lower the limit below what another launch needs)

@@ -1,43 +1,37 @@
 // Persistent, warp-specialised kernel for the ReplaySSM decode path on sm_100a.
 //
 // One launch processes every (sequence b, head h) unit of a decode layer (a unit is one
-// group of up to 8192/N state rows of a head). Each CTA owns the heads blockIdx.x,
-// blockIdx.x + gridDim.x, ... and streams their units through a ring of shared-memory
-// stages, with three kinds of warps that hand a stage on through mbarriers:
+// group of up to 16384/N state rows of a head). Each CTA owns chunks of heads (below)
+// and streams their units through a ring of shared-memory stages:
 //   * the producer warp reads each unit's buffer pointer word (prefetched 32 units at a
-//     time) and fills a stage with 1-D bulk copies (TMA), one copy per lane and two
-//     units per instruction: the unit's live ring records (k, v, Delta, a of every
-//     buffered input and of this call's new tokens) and its queries, completing on the
-//     stage's "rfull" barrier, and the unit's checkpoint tile (FP32 master rows, or FP8
-//     codes + per-row scales), completing on "tfull";
-//   * kCoefWarps coefficient warps take alternate units as soon as their records land
-//     (long before the tile): the decay weights and k_j . q_s products, and from them
-//     the whole buffer term u_s[p] = sum_j w_{s,j} (k_j . q_s) v_j[p] of every row and
-//     position, the output decays alpha_s and, for a fold, the fold weights and the
-//     table sig_j v_j[p]; they write these into the stage and arrive on "cready";
-//   * kRowWarps row warps take every unit, each its own rows, independently of one
-//     another: the state rows' dot products with the queries and y = alpha (S q) + u,
-//     or the fold (rank-c update in registers), its write-back and the outputs from the
-//     fresh rows; they release the stage through "empty".
-// The row warps' work per unit is only what the state tile itself needs, and no barrier
-// other than the stage's own ties them to the coefficient work, so the state streams at
-// the memory's pace while the coefficient chains of later units run meanwhile.
+//     time) and fills a stage with 1-D bulk copies (TMA), one copy per lane, two units
+//     per instruction: the unit's checkpoint tile (FP32 master rows, or the FP8 / FP4
+//     read copy's codes + per-row scales), the live k records of the head's k/q group
+//     and the head's live v, Delta, a records (each in one or two pieces of the ring),
+//     and the queries; all complete on the stage's "full" mbarrier;
+//   * NG consumer groups (kGroupGemvWarps row warps + one coefficient warp each) take
+//     alternate units end to end: the coefficient warp forms the decay weights and the
+//     k_j . q_s products while the row warps stream the state rows' dot products (or the
+//     fused fold, its write-back and the outputs from the fresh rows); the group meets at
+//     its barrier for the outputs and releases the stage through its "empty" mbarrier.
+//     Two groups keep two units in flight, so one unit's short dependent chains overlap
+//     the other's, while the producer keeps the next stages' copies in flight.
 // The state is streamed exactly once per call; every other byte is small.
 //
 // What a unit computes (blog "ReplaySSM: Cachear Inputs, No Estado": routes "estado y
 // salida" and "solo salida"; arXiv 2610.13778 abstract):
 //   REPLAY (step / verify over n_pos positions): if the buffer cannot take n_pos more
 //     entries, fold it first, S0 <- abar S0 + sum_j s_j v_j k_j^T, writing the master
-//     (and the FP8 copy) once; then for each position s
+//     (and the read copy) once; then for each position s
 //       y_s = alpha_s (S q_s) + sum_{j <= c+s} w_{s,j} (k_j . q_s) v_j
 //     where S is the fresh fold (in registers) or the stored checkpoint.
 //   FLUSH: fold the buffer of the selected sequences, no output.
 //   EAGER (baseline): S <- a S + Delta v k^T, y = S q, the state read and written every
 //     call (FP32, or a shared FP8 state re-quantised every call).
 //
-// Row layout of a unit: a state row of N floats is covered by TPR = N/4 lanes, four
-// columns each; a warp covers 32/TPR rows per pass and kRowsPerThread contiguous rows
-// per lane.
+// Row layout inside a group: a state row of N floats is covered by TPR = N/4 lanes, four
+// columns each; the group covers 32/TPR rows per warp per pass, and each thread takes
+// kRowsPerThread rows of a row group.
 #pragma once
 
 #include "replay_device.cuh"
@@ -49,67 +43,38 @@ __device__ __forceinline__ void report_error(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
-// A row warp's release of a stage, counted (after the warp's reads of the stage, which
-// __syncwarp orders before lane 0's fence).
-__device__ __forceinline__ void count_release(int* released, int lane) {
-  __syncwarp();
-  if (lane == 0) {
-    __threadfence_block();
-    atomicAdd(released, 1);
-  }
-}
-// Waits (bounded, about two seconds) until at least `target` row-warp releases of a stage
-// have been counted; the whole warp returns the outcome.
-__device__ __forceinline__ bool wait_released(const int* released, int target, int lane) {
-  bool ok = true;
-  if (lane == 0) {
-    const volatile int* r = released;
-    if (*r < target) {
-      const long long t0 = clock64();
-      while (*r < target) {
-        if (clock64() - t0 > kWaitLimitCycles) {
-          ok = false;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence_block();
-  }
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
+template <int NG>
+struct Groups {
+  static constexpr int kWarps = kConsumerWarps / NG;  // warps per consumer group
+  static constexpr int kThreads = kWarps * 32;
+};
 
 // barriers at the start of shared memory
 struct Bars {
-  uint64_t tfull[kMaxTileStages];   // the unit's state tile (and read-copy scales) landed
-  uint64_t tempty[kMaxTileStages];  // every row warp is done with the tile stage
-  uint64_t rfull[kMaxRecStages];    // the unit's records and queries landed, pointer word written
-  uint64_t cready[kMaxRecStages];   // its coefficients and buffer terms are in the record stage
-  uint64_t rempty[kMaxRecStages];   // every row warp is done with the record stage
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   int abort_flag;
-  int last_tfill[kMaxTileStages];   // CTA-local index of the latest unit copied into each stage
-  int last_rfill[kMaxRecStages];
-  int released[kMaxRecStages];      // row-warp releases of each record stage so far (kRowWarps per use)
+  int last_fill[kMaxStages];  // CTA-local index of the latest unit copied into each stage
 };
 static_assert(sizeof(Bars) <= kHeaderBytes, "the barrier header must fit the bytes the host layout reserves");
 
 struct Plan {
   int b, h, g, rb, r0, rows, start, c;  // rows r0 .. r0 + rows - 1 of head h of sequence b
   bool fold, corrupt, active, fp32_tile;
-  uint32_t tile_bytes, rec_bytes;       // bulk-copied bytes completing on tfull / rfull
+  uint32_t bytes;
 };
 
-// This CTA's units, in the order every role takes them: chunks of chunk_heads consecutive
-// heads of one k/q group (the group, or a part of it, so that its heads share one
-// coefficient warp and its k . q products), chunk c on CTA c mod gridDim.x, each head
-// with its row blocks in a row. Dealing the chunks round-robin keeps the 148 CTAs on
-// neighbouring tiles of the state at any moment, and one CTA holds every unit of a head
-// (the in-kernel append writes a head's new record once, before any copy of it).
+// This CTA's units, in the order its producer fills them and its groups take them:
+// chunks of chunk_heads consecutive heads of one k/q group (the group, or a part of it),
+// chunk c on CTA c mod gridDim.x, each head with its row blocks in a row. Dealing the
+// chunks round-robin keeps the CTAs on neighbouring tiles of the state at any moment,
+// one CTA holds every unit of a head (the in-kernel append writes a head's new record
+// once, before any copy of it), and a chunk's heads share one k record write.
 __device__ __forceinline__ int cta_chunks(const KParams& p) {
   return (p.num_chunks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 }
 __device__ __forceinline__ int cta_units(const KParams& p) { return (cta_chunks(p) * p.chunk_heads) << p.rb_shift; }
-// the CTA's i-th head (chunk i / chunk_heads, head i mod chunk_heads within it)
+// the CTA's hi-th head (chunk hi / chunk_heads, head hi mod chunk_heads within it)
 __device__ __forceinline__ int cta_head(const KParams& p, int hi) {
   const int ck = hi / p.chunk_heads;
   return ((int)blockIdx.x + ck * (int)gridDim.x) * p.chunk_heads + (hi - ck * p.chunk_heads);
@@ -117,17 +82,29 @@ __device__ __forceinline__ int cta_head(const KParams& p, int hi) {
 __device__ __forceinline__ int cta_unit(const KParams& p, int i) {
   return (cta_head(p, i >> p.rb_shift) << p.rb_shift) | (i & (p.row_blocks - 1));
 }
-// the CTA-local chunk of unit i
-__device__ __forceinline__ int unit_chunk(const KParams& p, int i) { return (i >> p.rb_shift) / p.chunk_heads; }
+
+// A unit's indices: sequence b, head h, its k/q group g, row block rb. The producer works
+// them out once per unit (the divisions) and passes them to the consumers in the stage.
+struct UnitIdx {
+  int b, h, g, rb;
+};
+__device__ __forceinline__ UnitIdx unit_idx(const KParams& p, int u) {
+  UnitIdx x;
+  const int bh = u >> p.rb_shift;
+  x.rb = u & (p.row_blocks - 1);
+  x.b = bh / p.H;
+  x.h = bh - x.b * p.H;
+  x.g = x.h / p.hpg;
+  return x;
+}
 
 template <int MODE, int CKPT, int S_IO>
-__device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word, int msk) {
+__device__ __forceinline__ Plan make_plan(const KParams& p, const UnitIdx& x, int32_t word, int msk) {
   Plan pl;
-  const int bh = u >> p.rb_shift;
-  pl.rb = u & (p.row_blocks - 1);
-  pl.b = bh / p.H;
-  pl.h = bh - pl.b * p.H;
-  pl.g = pl.h / p.hpg;
+  pl.rb = x.rb;
+  pl.b = x.b;
+  pl.h = x.h;
+  pl.g = x.g;
   pl.r0 = pl.rb * p.rows_unit;
   pl.rows = min(p.rows_unit, p.P - pl.r0);
   const uint32_t P = pl.rows, N = p.N;  // the unit's rows
@@ -139,8 +116,7 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
     pl.corrupt = false;
     pl.active = true;
     pl.fp32_tile = (CKPT == kCkptF32);
-    pl.tile_bytes = pl.fp32_tile ? P * N * 4u : P * (N / kCodeDiv) + P * 4u;
-    pl.rec_bytes = 0;  // gathered with cp.async, counted as arrivals
+    pl.bytes = pl.fp32_tile ? P * N * 4u : P * (N / kCodeDiv) + P * 4u;  // bulk-copied (TMA) bytes
     return pl;
   }
   pl.start = word >> 16;
@@ -156,13 +132,12 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, int u, int32_t word,
   pl.fp32_tile = (CKPT == kCkptF32) || pl.fold;
   if (pl.corrupt || !pl.active) {
     pl.active = false;
-    pl.tile_bytes = 0;
-    pl.rec_bytes = 0;
+    pl.bytes = 0;
     return pl;
   }
   const uint32_t records = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
-  pl.tile_bytes = pl.fp32_tile ? P * N * 4u : P * (N / kCodeDiv) + P * 4u;
-  pl.rec_bytes = records * (uint32_t)(p.rec_bytes + p.rec_k_bytes) + ((MODE == kModeReplay) ? p.n_pos * N * S_IO : 0u);
+  pl.bytes = (pl.fp32_tile ? P * N * 4u : P * (N / kCodeDiv) + P * 4u) +
+             records * (uint32_t)(p.rec_bytes + p.rec_k_bytes) + ((MODE == kModeReplay) ? p.n_pos * N * S_IO : 0u);
   return pl;
 }
 
@@ -186,14 +161,14 @@ struct Records {
 
 // ---------------------------------------------------------------------------- append
 // This CTA's units' new entries (one position) into their ring records, slot
-// (start + c) mod cap, by the worker threads before any bulk copy is issued: each head's
+// (start + c) mod cap, by the consumer threads before any bulk copy is issued: each head's
 // v, then Delta and a in one 16-byte piece, and the group's k once per chunk (a group of
 // more than kMaxChunkHeads heads spans chunks, possibly on several CTAs, each writing the
 // same bytes before it reads them). The input pieces do not depend on the pointer word,
 // so both reads are in flight together.
 template <int S_IO>
 __device__ __forceinline__ void append_entries(const KParams& p) {
-  constexpr int kPool = kWorkerWarps * 32;
+  constexpr int kPool = kConsumerWarps * 32;
   constexpr int kBatch = 8;  // pieces per thread in flight
   const int kpe = p.N * S_IO / 16;  // 16-byte pieces of k
   const int vpe = p.P * S_IO / 16;  // of v
@@ -243,213 +218,260 @@ __device__ __forceinline__ void append_entries(const KParams& p) {
 }
 
 // ---------------------------------------------------------------------------- producer
-// Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile (the unit's rows)
-// and 1 their read-copy row scales, into its tile stage `tst`, completing on tfull; into
-// its record stage `rst`: 2-3 the live head records and
-// 4-5 the live k records of the head's group, [start, start + count) modulo cap in one
-// or two pieces (whole records: every row block reads all of k and its rows of v), and
-// 6 the queries, completing on rfull. Returns the bytes of copy `kind` (0 if none) and
-// its addresses.
+// Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile (the unit's rows),
+// 1 their read-copy row scales, 2-3 the head's live records and 4-5 the live k records
+// of its group, [start, start + count) modulo cap in one or two pieces (whole records:
+// every row block reads all of k and its rows of v), 6 the queries. A producer lane
+// always issues the same kind, so it works out what does not depend on the unit once:
+// its source array and the strides that place a unit in it.
 constexpr int kCopyKinds = 7;
+struct LaneCopy {
+  const uint8_t* base;       // source array (kind 0: the FP32 master)
+  const uint8_t* base_copy;  // kind 0-1 with a read copy: the codes / scales array
+  uint64_t stride, stride_copy;  // bytes per (sequence, head) [kinds 0-3] or (sequence, group) [4-6]
+  uint32_t rb_stride, rb_stride_copy;  // kinds 0-1: bytes per row block
+  uint32_t rec;              // kinds 2-5: record bytes
+  uint32_t dst_off;          // offset in the stage
+  int kind;
+};
 template <int MODE, int CKPT, int S_IO>
-__device__ __forceinline__ uint32_t unit_copy(const KParams& p, const Plan& pl, uint8_t* tst, uint8_t* rst, int kind,
+__device__ __forceinline__ LaneCopy lane_copy(const KParams& p, int kind) {
+  constexpr uint32_t kCodeDiv = (CKPT == kCkptFp4) ? 2u : 1u;
+  const uint32_t N = p.N, P = p.P, UR = p.rows_unit;
+  LaneCopy lc;
+  lc.kind = kind;
+  lc.base_copy = nullptr;
+  lc.stride_copy = 0;
+  lc.rb_stride = lc.rb_stride_copy = 0;
+  lc.rec = 0;
+  if (kind == 0) {
+    lc.base = reinterpret_cast<const uint8_t*>(p.S);
+    lc.stride = (uint64_t)P * N * 4;
+    lc.rb_stride = UR * N * 4;
+    lc.base_copy = p.S8;
+    lc.stride_copy = (uint64_t)P * (N / kCodeDiv);
+    lc.rb_stride_copy = UR * (N / kCodeDiv);
+    lc.dst_off = 0;
+  } else if (kind == 1) {
+    lc.base = reinterpret_cast<const uint8_t*>(p.Sscale);
+    lc.stride = (uint64_t)P * 4;
+    lc.rb_stride = UR * 4;
+    lc.dst_off = UR * (N / kCodeDiv);  // the scales follow a full unit's codes
+  } else if (kind <= 3) {
+    lc.base = static_cast<const uint8_t*>(p.ring);
+    lc.rec = p.rec_bytes;
+    lc.stride = (uint64_t)p.cap * lc.rec;
+    lc.dst_off = p.off_rec;
+  } else if (kind <= 5) {
+    lc.base = static_cast<const uint8_t*>(p.ring_k);
+    lc.rec = p.rec_k_bytes;
+    lc.stride = (uint64_t)p.cap * lc.rec;
+    lc.dst_off = p.off_krec;
+  } else {
+    lc.base = static_cast<const uint8_t*>(p.qpack ? p.qpack : p.q);
+    lc.stride = (uint64_t)(p.qpack ? p.qpack_pos : 1) * N * S_IO;
+    lc.dst_off = p.off_q;
+  }
+  return lc;
+}
+// Source, destination and bytes of this lane's copy of the unit with plan `pl` (0 if none).
+template <int MODE, int CKPT, int S_IO>
+__device__ __forceinline__ uint32_t unit_copy(const KParams& p, const LaneCopy& lc, const Plan& pl, uint8_t* st,
                                               const uint8_t*& src, uint8_t*& dst) {
-  constexpr size_t kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;
-  const size_t P = pl.rows, N = p.N;
-  const size_t bh = (size_t)pl.b * p.H + pl.h;
-  const size_t bg = (size_t)pl.b * p.G + pl.g;
-  const size_t row0 = bh * p.P + pl.r0;  // the unit's first state row
-  const int R = p.rec_bytes;
-  const int RK = p.rec_k_bytes;
+  constexpr uint32_t kCodeDiv = (CKPT == kCkptFp4) ? 2u : 1u;
+  const uint32_t rows = pl.rows, N = p.N;
+  const int bh = pl.b * p.H + pl.h;
+  const int bg = pl.b * p.G + pl.g;
   const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
   const int first = min(cnt, p.cap - pl.start);
-  const uint8_t* ring = static_cast<const uint8_t*>(p.ring) + bh * p.cap * R;
-  const uint8_t* ring_k = static_cast<const uint8_t*>(p.ring_k) + bg * p.cap * RK;
-  const uint8_t* qsrc = p.qpack ? static_cast<const uint8_t*>(p.qpack) + bg * p.qpack_pos * N * S_IO
-                                : static_cast<const uint8_t*>(p.q) + bg * N * S_IO;
-  const uint8_t* tsrc = pl.fp32_tile ? reinterpret_cast<const uint8_t*>(p.S + row0 * N) : p.S8 + row0 * (N / kCodeDiv);
-  src = (kind == 0)   ? tsrc
-        : (kind == 1) ? reinterpret_cast<const uint8_t*>(p.Sscale + row0)
-        : (kind == 2) ? ring + (size_t)pl.start * R
-        : (kind == 3) ? ring
-        : (kind == 4) ? ring_k + (size_t)pl.start * RK
-        : (kind == 5) ? ring_k
-                      : qsrc;
-  dst = (kind == 0)   ? tst
-        : (kind == 1) ? tst + (size_t)p.rows_unit * (N / kCodeDiv)  // the scales follow a full unit's codes
-        : (kind == 2) ? rst + p.off_rec
-        : (kind == 3) ? rst + p.off_rec + (size_t)first * R
-        : (kind == 4) ? rst + p.off_krec
-        : (kind == 5) ? rst + p.off_krec + (size_t)first * RK
-                      : rst + p.off_q;
-  uint32_t bytes = 0;
-  bytes = (kind == 0) ? (pl.fp32_tile ? (uint32_t)(P * N * 4) : (uint32_t)(P * (N / kCodeDiv))) : bytes;
-  bytes = (kind == 1 && !pl.fp32_tile) ? (uint32_t)(P * 4) : bytes;
-  bytes = (kind == 2) ? (uint32_t)(first * R) : bytes;
-  bytes = (kind == 3) ? (uint32_t)((cnt - first) * R) : bytes;
-  bytes = (kind == 4) ? (uint32_t)(first * RK) : bytes;
-  bytes = (kind == 5) ? (uint32_t)((cnt - first) * RK) : bytes;
-  bytes = (kind == 6 && MODE == kModeReplay) ? (uint32_t)(p.n_pos * N * S_IO) : bytes;
+  const bool copy = !pl.fp32_tile;  // kinds 0-1 read the read copy
+  uint32_t bytes;
+  if (lc.kind <= 1) {
+    const uint8_t* base = (lc.kind == 0 && copy) ? lc.base_copy : lc.base;
+    const uint64_t stride = (lc.kind == 0 && copy) ? lc.stride_copy : lc.stride;
+    const uint32_t rbs = (lc.kind == 0 && copy) ? lc.rb_stride_copy : lc.rb_stride;
+    src = base + (uint64_t)bh * stride + (uint64_t)pl.rb * rbs;
+    dst = st + lc.dst_off;
+    bytes = (lc.kind == 0) ? (copy ? rows * (N / kCodeDiv) : rows * N * 4u) : (copy ? rows * 4u : 0u);
+  } else if (lc.kind <= 5) {
+    const bool second = (lc.kind == 3 || lc.kind == 5);  // the piece that wrapped to slot 0
+    src = lc.base + (uint64_t)((lc.kind <= 3) ? bh : bg) * lc.stride + (second ? 0u : (uint32_t)pl.start * lc.rec);
+    dst = st + lc.dst_off + (second ? (uint32_t)first * lc.rec : 0u);
+    bytes = (uint32_t)(second ? cnt - first : first) * lc.rec;
+  } else {
+    src = lc.base + (uint64_t)bg * lc.stride;
+    dst = st + lc.dst_off;
+    bytes = (MODE == kModeReplay) ? (uint32_t)p.n_pos * N * S_IO : 0u;
+  }
   return pl.active ? bytes : 0u;
 }
 
-// The producer warp. Step t copies the records (and queries) of unit t into its record
-// stage and the tile of unit t - D into its tile stage, D = p.lookahead: a unit's records
-// land D units before its tile, so the coefficient warps finish with them before the row
-// warps reach the unit. The tiles of the first num_tstages units go out at once (when the
-// kernel appends this call's entries itself, before the append is complete; their records
-// after it). Steps go kUnitsPerIssue at a time: the producer waits until their stages are
-// free, writes each unit's pointer word into its record stage, arms the stages' barriers
-// with the byte counts and issues every copy of the batch with one predicated bulk-copy
-// instruction (lane = step in batch * kCopyKinds + kind), which costs the warp about as
-// much as one copy. A tile's plan takes the pointer word its record stage holds (written
-// D steps before; the stage stays until the row warps are done with the unit). Waits are
-// exact: the producer visits every use of every stage in order.
+// The unit's indices, pointer word and flush mask, written into its stage for the
+// consumers: int32 word, mask, b, h, g, rb.
+__device__ __forceinline__ void write_meta(uint8_t* st, const KParams& p, const UnitIdx& x, int32_t word, int msk) {
+  int4* m = reinterpret_cast<int4*>(st + p.off_meta);
+  m[0] = make_int4(word, msk, x.b, x.h);
+  m[1] = make_int4(x.g, x.rb, 0, 0);
+}
+
+// The producer warp fills the CTA's units in order, kUnitsPerIssue at a time: it waits
+// until their stages are free, the lane of kind 0 arms each stage's "full" barrier
+// with the unit's byte count, and then one predicated bulk-copy instruction issues every
+// copy of the batch (lane = unit in batch * kCopyKinds + kind). Issuing costs the warp
+// about as much for one copy as for a whole batch, so batching is what keeps the stream
+// fed; the per-unit arithmetic is kept short for the same reason (the producer's loop,
+// not the memory, bounds a stream of small tiles): every 32 units, lane L works out
+// unit L's indices (the divisions) and reads its pointer word, once, one chunk ahead.
 template <int MODE, int CKPT, int S_IO, bool APPEND>
-__device__ void producer_loop(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars) {
+__device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   constexpr int U = kUnitsPerIssue;
   static_assert(U * kCopyKinds <= 32 && (32 % U) == 0, "a batch's copies must fit one warp and tile 32 units");
   const int lane = threadIdx.x & 31;
-  const int NT = p.num_tstages, NR = p.num_rstages, D = p.lookahead;
+  const int NS = p.num_stages;
   const uint64_t stream_policy = l2_evict_first_policy();
   const uint64_t keep_policy = l2_evict_normal_policy();
   const int total = cta_units(p);
-  auto unit_of = [&](int i) { return cta_unit(p, i); };
-  auto tst_of = [&](int i) { return tstages + (size_t)(i % NT) * p.tstage_bytes; };
-  auto rst_of = [&](int i) { return rstages + (size_t)(i % NR) * p.rstage_bytes; };
-  // pointer words (and flush masks) of the record units, 32 at a time, one chunk ahead:
-  // lane j of a chunk holds the word of the chunk's j-th unit
-  auto load_words = [&](int i0, int32_t& w, int& msk) {
-    w = 0;
-    msk = 1;
-    if (i0 + lane < total) {
-      const int b = (unit_of(i0 + lane) >> p.rb_shift) / p.H;
-      w = __ldg(p.counts_in + b);
-      if (MODE == kModeFlush && p.mask) msk = __ldg(p.mask + b);
-    }
+  struct Pre {
+    UnitIdx x;
+    int32_t word;
+    int msk;
   };
-  int32_t w_cur, w_nxt;
-  int m_cur, m_nxt;
-  load_words(0, w_cur, m_cur);
-  load_words(32, w_nxt, m_nxt);
-  const int j = lane / kCopyKinds;     // this lane's step within the batch
+  auto prefetch = [&](int i0) {
+    Pre q;
+    q.x = UnitIdx{0, 0, 0, 0};
+    q.word = 0;
+    q.msk = 1;
+    if (i0 + lane < total) {
+      q.x = unit_idx(p, cta_unit(p, i0 + lane));
+      q.word = __ldg(p.counts_in + q.x.b);
+      if (MODE == kModeFlush && p.mask) q.msk = __ldg(p.mask + q.x.b);
+    }
+    return q;
+  };
+  auto fetch = [&](const Pre& q, int i) {  // unit i's entry of the chunk, from its lane
+    Pre r;
+    const int src = i & 31;
+    r.x.b = __shfl_sync(0xffffffffu, q.x.b, src);
+    r.x.h = __shfl_sync(0xffffffffu, q.x.h, src);
+    r.x.g = __shfl_sync(0xffffffffu, q.x.g, src);
+    r.x.rb = __shfl_sync(0xffffffffu, q.x.rb, src);
+    r.word = __shfl_sync(0xffffffffu, q.word, src);
+    r.msk = __shfl_sync(0xffffffffu, q.msk, src);
+    return r;
+  };
+  Pre cur = prefetch(0), nxt = prefetch(32);
+  const int j = lane / kCopyKinds;     // this lane's unit within the batch
   const int kind = lane % kCopyKinds;  // and its copy
-  const int pre = min(NT, total);      // tiles issued up front
-  for (int i = 0; i < pre; ++i) {
-    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, unit_of(i), __shfl_sync(0xffffffffu, w_cur, i),
-                                               __shfl_sync(0xffffffffu, m_cur, i));
-    if (lane == 0) mbar_arrive_expect_tx(&bars->tfull[i], pl.tile_bytes);
-    __syncwarp();
-    const uint8_t* src;
-    uint8_t* dst;
-    uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, pl, tst_of(i), rst_of(i), lane, src, dst);
-    if (lane > 1) bytes = 0;
-    __syncwarp();
-    if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->tfull[i], lane == 0 ? stream_policy : keep_policy);
-    if (lane == 0) bars->last_tfill[i] = i;
-  }
-  if (APPEND && p.append_here) group_sync(kAppendBar, kThreads);  // the entries are in the ring
-  for (int t0 = 0; t0 < total + D; t0 += U) {
-    if ((t0 & 31) == 0 && t0 > 0) {
-      w_cur = w_nxt;
-      m_cur = m_nxt;
-      load_words(t0 + 32, w_nxt, m_nxt);
-    }
-    // every lane waits for the batch's stages, the warp agrees
-    bool ready = true;
-#pragma unroll
-    for (int jj = 0; jj < U; ++jj) {
-      const int r = t0 + jj;      // record unit
-      const int u = t0 + jj - D;  // tile unit
-      if (r < total && r >= NR) ready = ready && mbar_wait_bounded(&bars->rempty[r % NR], ((r / NR) - 1) & 1);
-      if (u >= pre && u < total && u >= NT) ready = ready && mbar_wait_bounded(&bars->tempty[u % NT], ((u / NT) - 1) & 1);
-    }
-    if (!__all_sync(0xffffffffu, ready)) {
+  const LaneCopy lc = lane_copy<MODE, CKPT, S_IO>(p, kind);
+  // When the kernel appends this call's entries itself, the first stages' state tiles
+  // (and read-copy scales) go out at once and their records and queries once the entries
+  // are in the ring; every stage is armed with its unit's full byte count either way.
+  int pre = 0;
+  if (APPEND && p.append_here) {
+    pre = min(NS, total);
+    for (int i = 0; i < pre; ++i) {
+      const Pre u = fetch(cur, i);
+      const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u.x, u.word, 1);
+      uint8_t* st = stages + (size_t)i * p.stage_bytes;
       if (lane == 0) {
+        write_meta(st, p, u.x, u.word, 1);
+        if (pl.corrupt) report_error(p.status, kErrPointer);
+        mbar_arrive_expect_tx(&bars->full[i], pl.bytes);
+      }
+      __syncwarp();
+      const uint8_t* src;
+      uint8_t* dst;
+      uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, lc, pl, st, src, dst);
+      if (lane > 1) bytes = 0;
+      __syncwarp();
+      if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->full[i], lane == 0 ? stream_policy : keep_policy);
+      if (lane == 0) bars->last_fill[i] = i;
+    }
+    group_sync(kAppendBar, kThreads);  // the entries are in the ring
+  }
+  // stage and use of the batch's first unit, advanced without divisions
+  int s0 = 0, k0 = 0;
+  for (int i0 = 0; i0 < total; i0 += U) {
+    if ((i0 & 31) == 0 && i0 > 0) {
+      cur = nxt;
+      nxt = prefetch(i0 + 32);
+    }
+    // every lane waits for the batch's stages (the releases of their previous uses; a
+    // version where lane 0 alone waited and the warp followed it measured ~20% slower),
+    // and the warp follows lane 0's outcome
+    bool ready = true;
+    {
+      int s = s0, k = k0;
+#pragma unroll
+      for (int jj = 0; jj < U; ++jj) {
+        if (i0 + jj < total && k > 0) ready = mbar_wait_bounded(&bars->empty[s], (k - 1) & 1) && ready;
+        if (++s == NS) {
+          s = 0;
+          ++k;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (!ready) {
         report_error(p.status, kErrWaitTimeout);
         bars->abort_flag = 1;
       }
-      break;
+      ready = ready && *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
     }
-    const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
-    if (__shfl_sync(0xffffffffu, ab, 0)) break;  // the warp decides together
-    const int r = t0 + j;
-    const int u = t0 + j - D;
-    const bool rec_step = j < U && r < total;
-    const bool tile_step = j < U && u >= pre && u < total;
-    // record side: the unit's pointer word and flush mask from the prefetched chunk
-    const int32_t word_r = __shfl_sync(0xffffffffu, w_cur, r & 31);
-    const int msk_r = __shfl_sync(0xffffffffu, m_cur, r & 31);
-    uint8_t* rst = rst_of(r);
-    const Plan plr = make_plan<MODE, CKPT, S_IO>(p, unit_of(r), word_r, msk_r);
-    if (rec_step && kind == 2) {
-      reinterpret_cast<int32_t*>(rst + p.off_meta)[0] = word_r;
-      reinterpret_cast<int32_t*>(rst + p.off_meta)[1] = msk_r;
-      if (plr.corrupt) report_error(p.status, kErrPointer);
-      mbar_arrive_expect_tx(&bars->rfull[r % NR], plr.rec_bytes);
+    if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;  // the warp decides together
+    const int i = i0 + j;
+    const bool valid = j < U && i < total;
+    int s = s0 + (j < U ? j : 0);  // this lane's unit's stage (U <= NS)
+    if (s >= NS) s -= NS;
+    s0 += U;
+    while (s0 >= NS) {
+      s0 -= NS;
+      ++k0;
     }
-    __syncwarp();  // a record stage armed in this step may hold a tile unit's word (lookahead < batch)
-    // tile side: the pointer word from the unit's record stage
-    int32_t word_u = 0;
-    int msk_u = 1;
-    if (tile_step && kind <= 1) {
-      const uint8_t* rsu = rst_of(u);
-      word_u = reinterpret_cast<const int32_t*>(rsu + p.off_meta)[0];
-      msk_u = reinterpret_cast<const int32_t*>(rsu + p.off_meta)[1];
+    const Pre u = fetch(cur, i);
+    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint64_t* bar = &bars->full[s];
+    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u.x, u.word, u.msk);
+    const bool armed = i < pre;  // tile already issued, stage already armed
+    if (valid && kind == 0 && !armed) {
+      write_meta(st, p, u.x, u.word, u.msk);
+      if (pl.corrupt) report_error(p.status, kErrPointer);
+      mbar_arrive_expect_tx(bar, pl.bytes);
     }
-    uint8_t* tst = tst_of(u < 0 ? 0 : u);
-    const Plan plt = make_plan<MODE, CKPT, S_IO>(p, unit_of(u < 0 ? 0 : u), word_u, msk_u);
-    if (tile_step && kind == 0) mbar_arrive_expect_tx(&bars->tfull[u % NT], plt.tile_bytes);
     __syncwarp();
     const uint8_t* src;
     uint8_t* dst;
-    uint32_t bytes = 0;
-    if (kind <= 1) {
-      bytes = unit_copy<MODE, CKPT, S_IO>(p, plt, tst, rst, kind, src, dst);
-      if (!tile_step) bytes = 0;
-    } else {
-      bytes = unit_copy<MODE, CKPT, S_IO>(p, plr, tst, rst, kind, src, dst);
-      if (!rec_step) bytes = 0;
-    }
+    uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, lc, pl, st, src, dst);
+    if (!valid || (armed && kind <= 1)) bytes = 0;
     __syncwarp();
-    if (bytes)
-      bulk_g2s_hint(dst, src, bytes, kind <= 1 ? &bars->tfull[u % NT] : &bars->rfull[r % NR],
-                    kind == 0 ? stream_policy : keep_policy);
-    if (tile_step && kind == 0) bars->last_tfill[u % NT] = u;
-    if (rec_step && kind == 2) bars->last_rfill[r % NR] = r;
+    if (bytes) bulk_g2s_hint(dst, src, bytes, bar, kind == 0 ? stream_policy : keep_policy);
+    if (valid && kind == 0) bars->last_fill[s] = i;
   }
   // Never leave with copies in flight into this CTA's shared memory: wait (bounded) for
   // the latest fill of every stage.
   __syncwarp();
-  bool ok = true;
-  for (int st_i = 0; st_i < NT; ++st_i) {
-    const int i = bars->last_tfill[st_i];
-    if (i >= 0) ok = mbar_wait_bounded(&bars->tfull[st_i], (i / NT) & 1) && ok;
+  for (int st_i = 0; st_i < NS; ++st_i) {
+    const int i = bars->last_fill[st_i];
+    if (i >= 0 && !mbar_wait_bounded(&bars->full[st_i], (i / NS) & 1) && lane == 0)
+      report_error(p.status, kErrWaitTimeout);
   }
-  for (int st_i = 0; st_i < NR; ++st_i) {
-    const int i = bars->last_rfill[st_i];
-    if (i >= 0) ok = mbar_wait_bounded(&bars->rfull[st_i], (i / NR) & 1) && ok;
-  }
-  if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
 }
 
-// The eager baseline's producer: one unit at a time, no lookahead (its coefficients are
-// two numbers); the tile (and FP8 scales) by bulk copy on tfull, the new token's k, v,
-// Delta, a and q gathered with per-lane cp.async into the record stage, each lane arriving
-// on rfull once its copies have landed.
+// The eager baseline's producer: one unit at a time; the tile (and the shared FP8 state's
+// scales) by bulk copy, the new token's k, v, Delta, a and q gathered with per-lane
+// cp.async.
 template <int CKPT, int S_IO>
-__device__ void producer_loop_eager(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars) {
+__device__ void producer_loop_eager(const KParams& p, uint8_t* stages, Bars* bars) {
   const int lane = threadIdx.x & 31;
-  const int NT = p.num_tstages, NR = p.num_rstages;
+  const int NS = p.num_stages;
   const uint64_t stream_policy = l2_evict_first_policy();
   const size_t P = p.P, N = p.N;
   const int total = cta_units(p);
   for (int i = 0; i < total; ++i) {
     const int u = cta_unit(p, i);
-    bool ready = true;
-    if (i >= NT) ready = mbar_wait_bounded(&bars->tempty[i % NT], ((i / NT) - 1) & 1);
-    if (ready && i >= NR) ready = mbar_wait_bounded(&bars->rempty[i % NR], ((i / NR) - 1) & 1);
-    if (!__all_sync(0xffffffffu, ready)) {
+    const int s = i % NS;
+    const int k = i / NS;
+    if (k > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[s], (k - 1) & 1))) {
       if (lane == 0) {
         report_error(p.status, kErrWaitTimeout);
         bars->abort_flag = 1;
@@ -458,29 +480,30 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* tstages, uint8_t*
     }
     const int ab = (lane == 0) ? *reinterpret_cast<volatile int*>(&bars->abort_flag) : 0;
     if (__shfl_sync(0xffffffffu, ab, 0)) break;
-    const Plan pl = make_plan<kModeEager, CKPT, S_IO>(p, u, 0, 1);
-    uint8_t* tst = tstages + (size_t)(i % NT) * p.tstage_bytes;
-    uint8_t* rst = rstages + (size_t)(i % NR) * p.rstage_bytes;
+    const UnitIdx x = unit_idx(p, u);
+    const Plan pl = make_plan<kModeEager, CKPT, S_IO>(p, x, 0, 1);
+    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    uint64_t* bar = &bars->full[s];
     const size_t bh = (size_t)pl.b * p.H + pl.h;
     const size_t bg = (size_t)pl.b * p.G + pl.g;
     const size_t row0 = bh * P + pl.r0;  // the unit's rows
     const uint32_t rows = (uint32_t)pl.rows;
-    constexpr size_t kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;
-    uint8_t* recbuf = rst + p.off_rec;
-    uint8_t* kbuf = rst + p.off_krec;
-    if (lane == 0) mbar_arrive_expect_tx(&bars->tfull[i % NT], pl.tile_bytes);
+    uint8_t* recbuf = st + p.off_rec;
+    uint8_t* kbuf = st + p.off_krec;
+    if (lane == 0) {
+      write_meta(st, p, x, 0, 1);
+      mbar_arrive_expect_tx(bar, pl.bytes);
+    }
     __syncwarp();
     if (lane == 0)
-      bulk_g2s_hint(tst, pl.fp32_tile ? (const void*)(p.S + row0 * N) : (const void*)(p.S8 + row0 * (N / kCodeDiv)),
-                    pl.fp32_tile ? (uint32_t)(rows * N * 4) : (uint32_t)(rows * (N / kCodeDiv)), &bars->tfull[i % NT],
-                    stream_policy);
-    if (lane == 1 && !pl.fp32_tile)
-      bulk_g2s(tst + (size_t)p.rows_unit * (N / kCodeDiv), p.Sscale + row0, rows * 4u, &bars->tfull[i % NT]);
+      bulk_g2s_hint(st, pl.fp32_tile ? (const void*)(p.S + row0 * N) : (const void*)(p.S8 + row0 * N),
+                    pl.fp32_tile ? (uint32_t)(rows * N * 4) : (uint32_t)(rows * N), bar, stream_policy);
+    if (lane == 1 && !pl.fp32_tile) bulk_g2s(st + (size_t)p.rows_unit * N, p.Sscale + row0, rows * 4u, bar);
     const int kpe = (int)(N * S_IO / 16);
     const int vpe = (int)(P * S_IO / 16);
     for (int idx = lane; idx < 2 * kpe + vpe; idx += 32) {
       if (idx < kpe) {
-        cp_async16(rst + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
+        cp_async16(st + p.off_q + idx * 16, static_cast<const uint8_t*>(p.q) + bg * N * S_IO + idx * 16);
       } else if (idx < 2 * kpe) {
         const int ch = idx - kpe;
         cp_async16(kbuf + ch * 16, static_cast<const uint8_t*>(p.k) + bg * N * S_IO + ch * 16);
@@ -491,37 +514,28 @@ __device__ void producer_loop_eager(const KParams& p, uint8_t* tstages, uint8_t*
     }
     if (lane == 0) cp_async4(recbuf + P * S_IO, p.dt + bh);
     if (lane == 1) cp_async4(recbuf + P * S_IO + 4, p.a + bh);
-    cp_async_arrive(&bars->rfull[i % NR]);
-    if (lane == 0) {
-      bars->last_tfill[i % NT] = i;
-      bars->last_rfill[i % NR] = i;
-    }
+    cp_async_arrive(bar);
+    if (lane == 0) bars->last_fill[s] = i;
   }
   __syncwarp();
-  bool ok = true;
-  for (int st_i = 0; st_i < NT; ++st_i) {
-    const int i2 = bars->last_tfill[st_i];
-    if (i2 >= 0) ok = mbar_wait_bounded(&bars->tfull[st_i], (i2 / NT) & 1) && ok;
+  for (int st_i = 0; st_i < NS; ++st_i) {
+    const int i2 = bars->last_fill[st_i];
+    if (i2 >= 0 && !mbar_wait_bounded(&bars->full[st_i], (i2 / NS) & 1) && lane == 0)
+      report_error(p.status, kErrWaitTimeout);
   }
-  for (int st_i = 0; st_i < NR; ++st_i) {
-    const int i2 = bars->last_rfill[st_i];
-    if (i2 >= 0) ok = mbar_wait_bounded(&bars->rfull[st_i], (i2 / NR) & 1) && ok;
-  }
-  if (!ok && lane == 0) report_error(p.status, kErrWaitTimeout);
 }
 
-// ---------------------------------------------------------------------------- coefficients
-// What a coefficient warp forms for a unit, from its records in shared memory (all 32
-// lanes; the results go into the stage's coefficient area for the row warps):
-//  * fold weights when the unit folds (blog "Ruta 'estado y salida'"): sig_j = Delta_j
-//    prod_{j<i<c} a_i and abar = prod_{i<c} a_i (the eager baseline: its single entry,
-//    sig_0 = Delta, abar = a), and the table wt[j][p] = sig_j v_j[p] of the unit's rows;
+// ---------------------------------------------------------------------------- consumers
+// The coefficient warp's share of a unit (all 32 lanes; ws is its group's workspace):
+//  * fold weights of the c buffered entries when the unit folds (blog "Ruta 'estado y
+//    salida'"): sig_j = Delta_j prod_{j<i<c} a_i and abar = prod_{i<c} a_i (the eager
+//    baseline: its single entry, sig_0 = Delta, abar = a);
 //  * for every position s the outputs replay the entries o0 .. c+s, o0 = c after a fold
 //    and 0 otherwise (blog "Ruta 'solo salida'"):
 //        alpha_s = prod_{o0<=i<=c+s} a_i,   w_{s,j} = Delta_j prod_{j<i<=c+s} a_i,
 //        u_s[p]  = sum_{o0<=j<=c+s} w_{s,j} (k_j . q_s) v_j[p],
-//    so that the row warps only add y_s = alpha_s (S q_s) + u_s. The products of decay
-//    factors are suffix products over the window.
+//    so that y_s = alpha_s (S q_s) + u_s. The products of decay factors are suffix
+//    products over the window, one lane per entry.
 template <int N, typename IO, int MODE>
 __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& rec, int c, float* sig, int lane) {
   if (MODE == kModeEager) {
@@ -543,436 +557,564 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
   if (lane == 0) sig[kMaxWindow] = incl;
 }
 
-// k_l . q_s of the window entries l < width (entry o0 + l) for the positions s < n, into
-// kq[s][l]: four lanes per entry (a quarter row each, one shuffle pair to combine), eight
-// entries per pass. The products belong to the k/q group, so a coefficient warp forms
-// them once for all the group's heads and row blocks.
+// The coefficients of the positions s = s0, s0 + ds, ... (< n) by one warp: alpha_s and
+// cw[s][l] = w_{s,l} (k_l . q_s) with w_{s,l} = Delta_l prod_{l < i <= last_s} a_i, zero
+// past the position's last entry so that the row lanes may read whole vectors. Two
+// forms, chosen by measurement:
+//  * output_coefs_pairs, for one-position calls on the FP32 checkpoint, where one warp
+//    per group forms the coefficients while four stream the state and its chain is on
+//    the unit's critical path: a lane pair per entry, sixteen entries per pass (half of k_l . q_s per lane,
+//    the second half one 4-element chunk rotated so that the pair's reads fall in
+//    different shared-memory banks, one shuffle to combine), and each lane forms its
+//    entry's decay weight itself from broadcast reads of the a_i. Its chain is one round
+//    of shared-memory reads, the products and one shuffle.
+//  * output_coefs_quarters, for multi-position calls, where all five warps of a group
+//    form coefficients at once and the shared-memory pipe, not one warp's chain, is the
+//    limit, and for the FP8 / FP4 read copies, whose row warps (decoding the codes) rather than
+//    the coefficient warp set the pace: four lanes per entry, eight entries per pass,
+//    and the decay weights by a suffix-product scan across the lanes, which issues fewer
+//    shared-memory requests per position than the broadcast reads.
+// Both keep the raw products k_l . q_s in kqraw[s][l] (the group's workspace) and, with
+// `reuse`, take them from there: the heads of a chunk share their sequence's window and
+// their group's k and q, so a group that takes consecutive units of one chunk forms the
+// products once (blog, end of "Ruta 'solo salida'": k and q belong to the group).
 template <int N, typename IO>
-__device__ __forceinline__ void window_kq(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int o0,
-                                          int width, int n, float* kq, int lane) {
+__device__ __forceinline__ void output_coefs_quarters(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
+                                                      int n, int o0, int s0, int ds, float* alpha, float* cw,
+                                                      float* kqraw, bool reuse, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
   constexpr int QN = N / 4;  // elements of a quarter row
-  const int quarter = lane & 3;
-  for (int l0 = 0; l0 < width; l0 += 8) {
-    const int l = l0 + (lane >> 2);
-    const uint8_t* kp = rec.k(o0 + (l < width ? l : 0)) + (size_t)quarter * QN * S_IO;
-    float4 kr[QN / 4];  // the lane's quarter of k_l, read once for every position
-#pragma unroll
-    for (int e = 0; e < QN / 4; ++e) kr[e] = IoT<IO>::load4(kp + (size_t)e * 4 * S_IO);
-    for (int s = 0; s < n; ++s) {
-      const uint8_t* qq = qbuf + ((size_t)s * N + quarter * QN) * S_IO;
-      float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-      for (int e = 0; e < QN / 4; e += 2) {
-        d0 += dot4(kr[e], IoT<IO>::load4(qq + (size_t)e * 4 * S_IO));
-        if (e + 1 < QN / 4) d1 += dot4(kr[e + 1], IoT<IO>::load4(qq + (size_t)(e + 1) * 4 * S_IO));
-      }
-      float d = d0 + d1;
-      d += __shfl_xor_sync(0xffffffffu, d, 1);
-      d += __shfl_xor_sync(0xffffffffu, d, 2);
-      if (quarter == 0 && l < width) kq[s * kMaxWindow + l] = d;
-    }
-  }
-}
-
-// The output coefficients of one head from its decay factors and the group's k . q: for
-// every position s, alpha_s = prod_{l<=last_s} a_{o0+l} and cw[s][l] = w_{s,l} kq[s][l]
-// with w_{s,l} = Delta_{o0+l} prod_{l<i<=last_s} a_{o0+i}, zero past last_s (all 32 lanes
-// written, so that the buffer terms may read whole vectors); a lane per entry and a
-// suffix-product scan across the lanes per position.
-template <int N, typename IO>
-__device__ __forceinline__ void output_weights(const Records<N, IoT<IO>::bytes>& rec, int c, int n, int o0,
-                                               const float* kq, float* alpha, float* cw, int lane) {
-  const int width = c + n - o0;  // window entries (at most kMaxWindow)
+  const int width = c + n - o0;  // window entries (at most L)
   float xa = 1.f, xd = 0.f;
   if (lane < width) {
     xa = rec.a(o0 + lane);
     xd = rec.dt(o0 + lane);
   }
-  for (int s = 0; s < n; ++s) {
+  const int quarter = lane & 3;
+  const int rot = (quarter >> 1) * 4;
+  static_assert((QN & (QN - 1)) == 0, "a quarter row is a power of two elements");
+  // raw k_l . q_s into kqraw[s][l] (kept there from the group's previous unit when that
+  // unit had the same sequence and k/q group: same window, same products)
+  for (int l0 = 0; l0 < (reuse ? 0 : width); l0 += 8) {
+    const int l = l0 + (lane >> 2);
+    const uint8_t* kq = rec.k(o0 + (l < width ? l : 0)) + (size_t)quarter * QN * S_IO;
+    for (int s = s0; s < n; s += ds) {
+      const uint8_t* qq = qbuf + ((size_t)s * N + quarter * QN) * S_IO;
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < QN; e += 8) {
+        // quarters 2 and 3 start one 4-element chunk later (mod QN): with BF16 records a
+        // quarter is 16 banks wide, so quarter q and q + 2 of one entry would share banks
+        const int e0 = (e + rot) & (QN - 1), e1 = (e + 4 + rot) & (QN - 1);
+        d0 += dot4(IoT<IO>::load4(kq + (size_t)e0 * S_IO), IoT<IO>::load4(qq + (size_t)e0 * S_IO));
+        if (e + 4 < QN)
+          d1 += dot4(IoT<IO>::load4(kq + (size_t)e1 * S_IO), IoT<IO>::load4(qq + (size_t)e1 * S_IO));
+      }
+      float d = d0 + d1;
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
+      d += __shfl_xor_sync(0xffffffffu, d, 2);
+      if (quarter == 0 && l < width) kqraw[s * kMaxWindow + l] = d;
+    }
+  }
+  __syncwarp();
+  for (int s = s0; s < n; s += ds) {
     const int last = c + s - o0;  // position s replays window entries 0 .. last
     const float incl = warp_suffix_prod(lane <= last ? xa : 1.f, lane);  // prod_{lane<=i<=last} a_i
     float excl = __shfl_down_sync(0xffffffffu, incl, 1);
     if (lane == 31) excl = 1.f;
     if (lane == 0) alpha[s] = incl;
-    cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * kq[s * kMaxWindow + lane] : 0.f;
+    // w_{s,l} (k_l . q_s); zero past `last`, so that the row lanes may read whole vectors
+    const float kqv = (lane <= last) ? kqraw[s * kMaxWindow + lane] : 0.f;
+    cw[s * kMaxWindow + lane] = (lane <= last) ? xd * excl * kqv : 0.f;
   }
 }
 
 
-template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ __forceinline__ void coef_unit(const KParams& p, const Plan& pl, uint8_t* st, float* kq, float* cw,
-                                          bool kq_ready, int lane) {
+template <int N, typename IO>
+__device__ __forceinline__ void output_coefs_pairs(const Records<N, IoT<IO>::bytes>& rec, const uint8_t* qbuf, int c,
+                                                   int n, int o0, int s0, int ds, float* alpha, float* cw,
+                                                   float* kqraw, bool reuse, int lane) {
   constexpr int S_IO = IoT<IO>::bytes;
-  constexpr int NQR = NQ > 0 ? NQ : 1;
-  const Records<N, S_IO> rec{st + p.off_krec, st + p.off_rec, p.P, p.rec_bytes, p.rec_k_bytes};
-  uint8_t* co = st + p.off_coef;
-  float* alpha = reinterpret_cast<float*>(co + p.co_alpha);  // [kMaxPos]
-  float* sig = reinterpret_cast<float*>(co + p.co_sig);      // fold weights; [kMaxWindow] = abar
-  float* u = reinterpret_cast<float*>(co + p.co_u);          // [n][u_stride] buffer terms
-  float* wt = reinterpret_cast<float*>(co + p.co_wt);        // [cf][wt_stride] fold weights times v
-  const int c = pl.c;
-  const int n = (MODE == kModeReplay) ? p.n_pos : 0;
-  const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
-  const int o0 = pl.fold ? c : 0;                                // first entry the outputs replay
-  const int rows = pl.rows;
-  const int r0 = pl.r0;
-  const int wts = p.wt_stride;
-  if (cf > 0) {
-    fold_weights<N, IO, MODE>(rec, c, sig, lane);
-    __syncwarp();
-    // wt[j][p] = sig_j v_j[r0 + p], zero for the rows past the unit's (the row warps read
-    // whole vectors)
-    for (int j = 0; j < cf; ++j) {
-      const float sj = sig[j];
-      const uint8_t* vj = rec.v(j) + (size_t)r0 * S_IO;
-      for (int pp = lane; pp < wts; pp += 32)
-        wt[(size_t)j * wts + pp] = pp < rows ? sj * IoT<IO>::load1(vj + (size_t)pp * S_IO) : 0.f;
-    }
-  }
-  if (MODE == kModeReplay) {
-    const int width = c + n - o0;
-    if (!kq_ready) {
-      window_kq<N, IO>(rec, st + p.off_q, o0, width, n, kq, lane);
-      __syncwarp();
-    }
-    output_weights<N, IO>(rec, c, n, o0, kq, alpha, cw, lane);
-    __syncwarp();
-    // u_s[p] = sum_l cw[s][l] v_{o0+l}[r0 + p]: two rows per lane at a time (p and p + 32),
-    // each v read once for every position, eight entries in flight per row (cw is zero
-    // past each position's window)
-    for (int pr0 = lane; pr0 < rows; pr0 += 64) {
-      const int pr1 = pr0 + 32 < rows ? pr0 + 32 : pr0;  // the second row, or the first again
-      const uint8_t* vrow0 = rec.base + (size_t)(r0 + pr0) * S_IO;
-      const uint8_t* vrow1 = rec.base + (size_t)(r0 + pr1) * S_IO;
-      float acc0[NQR], acc1[NQR];
-#pragma unroll
-      for (int s = 0; s < NQR; ++s) acc0[s] = acc1[s] = 0.f;
-      for (int l0 = 0; l0 < width; l0 += 8) {
-        float v0[8], v1[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const size_t off = (size_t)(o0 + (l0 + r < width ? l0 + r : 0)) * rec.R;
-          v0[r] = (l0 + r < width) ? IoT<IO>::load1(vrow0 + off) : 0.f;
-          v1[r] = (l0 + r < width) ? IoT<IO>::load1(vrow1 + off) : 0.f;
-        }
-#pragma unroll
-        for (int s = 0; s < NQR; ++s) {
-          if (s < n) {
-            const float4 ca = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0);
-            const float4 cb = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0 + 4);
-            acc0[s] = fmaf(ca.x, v0[0], fmaf(ca.y, v0[1], fmaf(ca.z, v0[2], fmaf(ca.w, v0[3],
-                      fmaf(cb.x, v0[4], fmaf(cb.y, v0[5], fmaf(cb.z, v0[6], fmaf(cb.w, v0[7], acc0[s]))))))));
-            acc1[s] = fmaf(ca.x, v1[0], fmaf(ca.y, v1[1], fmaf(ca.z, v1[2], fmaf(ca.w, v1[3],
-                      fmaf(cb.x, v1[4], fmaf(cb.y, v1[5], fmaf(cb.z, v1[6], fmaf(cb.w, v1[7], acc1[s]))))))));
-          }
-        }
-      }
-#pragma unroll
-      for (int s = 0; s < NQR; ++s) {
-        if (s < n) {
-          u[s * p.u_stride + pr0] = acc0[s];
-          if (pr0 + 32 < rows) u[s * p.u_stride + pr0 + 32] = acc1[s];
-        }
-      }
-    }
-  }
-}
-
-// The coefficient warps' loop, on the record ring: the units of a chunk (heads of one k/q
-// group, each with its row blocks) all go to one warp, chunks in turn, so that the warp
-// forms the group's k . q once per chunk. A warp's consecutive units may lie any distance
-// apart, so its parity waits are made exact by counting: before it waits for the k-th use
-// of a record stage it waits until the row warps' releases of that stage's use k-2 have
-// all been counted (the row warps take the units in order and cannot be two uses further
-// on, since they need this warp's coefficients for use k). Then it waits for the stage's
-// previous release (rempty, phase k-1), after which no one else touches the stage, and
-// for its records (rfull, phase k), whose phase k-1 completed before the row warps could
-// release use k-1. Each warp takes its units in order, so no wait can close a cycle.
-template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ void coef_loop(const KParams& p, uint8_t* rstages, Bars* bars, float* kq, float* cw, int cwarp, int lane) {
-  constexpr int S_IO = IoT<IO>::bytes;
-  const int NR = p.num_rstages;
-  const int total = cta_units(p);
-  int cached = -1;  // the CTA-local chunk whose k . q products the warp holds in kq
-  for (int i = 0; i < total; ++i) {
-    const int key = unit_chunk(p, i);
-    if (key % kCoefWarps != cwarp) continue;
-    const int s = i % NR;
-    const int k = i / NR;
-    bool ready = *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
-    if (ready && k > 1) ready = wait_released(&bars->released[s], (k - 1) * kRowWarps, lane);
-    if (ready && k > 0) ready = mbar_wait_bounded(&bars->rempty[s], (k - 1) & 1);
-    if (ready) ready = mbar_wait_bounded(&bars->rfull[s], k & 1);
-    if (!__all_sync(0xffffffffu, ready)) {
-      if (lane == 0) {
-        report_error(p.status, kErrWaitTimeout);
-        bars->abort_flag = 1;
-      }
-      break;
-    }
-    uint8_t* st = rstages + (size_t)s * p.rstage_bytes;
-    const int32_t word = reinterpret_cast<const int32_t*>(st + p.off_meta)[0];
-    const int msk = reinterpret_cast<const int32_t*>(st + p.off_meta)[1];
-    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, cta_unit(p, i), word, msk);
-    if (pl.active) {
-      coef_unit<N, IO, CKPT, MODE, NQ>(p, pl, st, kq, cw, cached == key, lane);
-      if (MODE == kModeReplay) cached = key;
-    }
-    // publish the sequence's pointer word (the entries are already in the ring) and flag
-    if (MODE != kModeEager && lane == 0 && pl.h == 0 && pl.rb == 0) {
-      const int start = pl.start;
-      const int cap = p.cap;
-      if (!pl.active) {
-        p.counts_out[pl.b] = word;  // nothing folded: the pointer word carries over
-        if (MODE == kModeFlush && p.flushed && !pl.corrupt) p.flushed[pl.b] = 0;
-      } else if (MODE == kModeReplay) {
-        int start2 = pl.fold ? start + pl.c : start;
-        start2 -= (start2 >= cap) ? cap : 0;
-        const int cnt2 = (pl.fold ? 0 : pl.c) + (p.commit ? p.n_pos : 0);
-        p.counts_out[pl.b] = (start2 << 16) | cnt2;
-        if (p.flushed && (!p.flushed_or || pl.fold)) p.flushed[pl.b] = pl.fold ? 1 : 0;
+  constexpr int HN = N / 2;       // elements of half a row
+  constexpr int HC = HN / 4;      // 4-element chunks of half a row
+  constexpr int kBlock = 16;      // decay factors read per round
+  const int width = c + n - o0;   // window entries (at most kMaxWindow)
+  const int half = lane & 1;
+  for (int e0 = 0; e0 < width; e0 += 16) {
+    const int e = e0 + (lane >> 1);
+    const int er = (e < width) ? e : width - 1;  // lanes past the window read a valid record
+    const uint8_t* kh = rec.k(o0 + er) + (size_t)half * HN * S_IO;
+    const float xd = rec.dt(o0 + er);
+    for (int s = s0; s < n; s += ds) {
+      const int last = c + s - o0;  // position s replays window entries 0 .. last
+      float kq;
+      if (reuse) {  // the group's previous unit had the same sequence and k/q group
+        kq = kqraw[s * kMaxWindow + e];
       } else {
-        int start2 = start + pl.c;
-        start2 -= (start2 >= cap) ? cap : 0;
-        p.counts_out[pl.b] = start2 << 16;
-        if (p.flushed) p.flushed[pl.b] = 1;
+        const uint8_t* qh = qbuf + ((size_t)s * N + half * HN) * S_IO;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < HC; ++t) {
+          const int off = ((t + half) % HC) * 4 * S_IO;
+          const float4 kk = IoT<IO>::load4(kh + off);
+          const float4 qq = IoT<IO>::load4(qh + off);
+          d[t & 3] = fmaf(kk.x, qq.x, fmaf(kk.y, qq.y, fmaf(kk.z, qq.z, fmaf(kk.w, qq.w, d[t & 3]))));
+        }
+        kq = (d[0] + d[1]) + (d[2] + d[3]);
+        kq += __shfl_xor_sync(0xffffffffu, kq, 1);
+        if (half == 0) kqraw[s * kMaxWindow + e] = kq;
       }
+      // prod_{e < i <= last} a_i; i runs from e0 + 1 (i <= e0 never counts for this pass)
+      float w = 1.f;
+      float a_first = 1.f;  // a_{o0}, for alpha
+      for (int t0 = (e0 == 0) ? 0 : e0 + 1; t0 <= last; t0 += kBlock) {
+        float at[kBlock];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) at[r] = (t0 + r <= last) ? rec.a(o0 + t0 + r) : 1.f;
+        if (t0 == 0) a_first = at[0];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) w = (t0 + r > e) ? w * at[r] : w;
+      }
+      if (half == 0 && e < kMaxWindow) cw[s * kMaxWindow + e] = (e <= last) ? xd * w * kq : 0.f;
+      if (lane == 0 && e0 == 0) alpha[s] = a_first * w;  // prod_{0 <= i <= last} a_i
     }
-    __syncwarp();
-    mbar_arrive(&bars->cready[s]);
   }
 }
 
-// ---------------------------------------------------------------------------- rows
-// One unit's rows by one row warp (rows rbase .. rbase + kRowsPerThread - 1 of the unit
-// per lane, four columns each). Output-only: y_s = alpha_s (S q_s) + u_s. Fold: x <- abar
-// x + sum_j wt[j][rows] k_j[cols] in registers, the write-back (FP32 master and/or FP8
-// codes with per-row scales), then the outputs from the fresh rows.
-template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ __forceinline__ void row_unit(const KParams& p, const Plan& pl, const uint8_t* tst, const uint8_t* st, int warp,
-                                         int lane) {
-  constexpr int S_IO = IoT<IO>::bytes;
+// One unit, by one consumer group: kGroupGemvWarps warps stream the state rows (dot
+// products, or the fold and its write-back) while the group's coefficient warp works out
+// the decay weights and the buffer terms from the records; the two meet at the group
+// barrier before the outputs are written.
+template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
+__device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, uint8_t* st, uint8_t* ws, int gtid,
+                                             int bar_id, int gemv_bar_id, bool reuse) {
+  using Gr = Groups<NG>;
+  constexpr int GT = Gr::kThreads;    // the whole group (barriers)
+  constexpr int GW = kGroupGemvWarps;  // warps on the state rows
+  constexpr int GTG = GW * 32;
   constexpr int TPR = N / 4;
   constexpr int RPW = 32 / TPR;  // rows per warp pass
+  constexpr int RPG = GW * RPW;  // rows per group pass
   constexpr int RT = kRowsPerThread;
+  constexpr int RGR = RPG * RT;  // rows per row group
+  constexpr int S_IO = IoT<IO>::bytes;
   constexpr int NQR = NQ > 0 ? NQ : 1;
   using Red = SegReduce<RT, TPR>;
-  const int rbase = (warp * RPW + lane / TPR) * RT;
+  const int lane = gtid & 31;
+  const int gw = gtid >> 5;
+  const bool coef_warp = gw == GW;
+  // this thread's rows of a row group: rbase .. rbase + RT - 1 (contiguous, so that a
+  // fold reads their weights as four 16-byte vectors)
+  const int rbase = (gw * RPW + lane / TPR) * RT;
   const int col = (lane % TPR) * 4;
   const int P = pl.rows;  // the unit's rows: r0 .. r0 + P - 1 of the head's PH
   const int PH = p.P;
   const int r0 = pl.r0;
+  const int c = pl.c;
   const int n = (MODE == kModeReplay) ? p.n_pos : (MODE == kModeEager ? 1 : 0);
-  const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? pl.c : 0);
-  const uint8_t* tile = tst;  // the tile stage; records, queries and coefficients in the record stage `st`
+  const int cf = (MODE == kModeEager) ? 1 : (pl.fold ? c : 0);  // entries folded into the state
+  const int o0 = pl.fold ? c : 0;                                // first entry the outputs replay
+  const int wts = p.wt_stride;  // row stride of the fold weight table, >= P, multiple of RT
+  const uint8_t* tile = st;
   const uint8_t* qbuf = st + p.off_q;
   constexpr int kCodeDiv = (CKPT == kCkptFp4) ? 2 : 1;  // read copy: code bytes per row = N / kCodeDiv
-  const Records<N, S_IO> rec{st + p.off_krec, st + p.off_rec, PH, p.rec_bytes, p.rec_k_bytes};
+  const Records<N, S_IO> rec{st + p.off_krec, st + p.off_rec, PH, p.rec_bytes, p.rec_k_bytes};  // whole records: v_j[0 .. PH)
   const float* scale_tile = reinterpret_cast<const float*>(tile + (size_t)p.rows_unit * (N / kCodeDiv));
-  const uint8_t* co = st + p.off_coef;
-  const float* alpha = reinterpret_cast<const float*>(co + p.co_alpha);
-  const float* sig = reinterpret_cast<const float*>(co + p.co_sig);
-  const float* u = reinterpret_cast<const float*>(co + p.co_u);
-  const float* wt = reinterpret_cast<const float*>(co + p.co_wt);
+  float* alpha = reinterpret_cast<float*>(ws + p.ws_alpha);  // [kMaxPos]
+  float* sig = reinterpret_cast<float*>(ws + p.ws_sig);      // fold weights; [kMaxWindow] = abar
+  float* cw = reinterpret_cast<float*>(ws + p.ws_cw);        // [kMaxPos][kMaxWindow] entry coefficients
+  float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [c][wts] fold weight times v_j[p]
+  float* kqraw = reinterpret_cast<float*>(ws + p.ws_kq);     // [kMaxPos][kMaxWindow] raw k_l . q_s
   const size_t bh = (size_t)pl.b * p.H + pl.h;
+  const int ngroups = (P + RGR - 1) / RGR;
   const bool fold = pl.fold;
 
-  float4 x[RT];
-#pragma unroll
-  for (int r = 0; r < RT; ++r) {
-    const int pr = rbase + r;
-    x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (pr < P) {
-      if (pl.fp32_tile) {
-        x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
-      } else {
-        const float4 e =
-            (CKPT == kCkptFp4)
-                ? e2m1x4_to_float4(*reinterpret_cast<const unsigned short*>(tile + (size_t)pr * (N / 2) + col / 2))
-                : e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
-        if (MODE == kModeEager) {  // a shared FP8 state: dequantise
-          const float sc = scale_tile[pr];
-          x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
-        } else {  // the read copy: the row scale multiplies the dot product
-          x[r] = e;
-        }
-      }
+  if (coef_warp) {
+    // ---- the coefficient warp: fold weights first (the fold waits for them), then the
+    // outputs' buffer terms while the fold runs
+    if (fold) {
+      fold_weights<N, IO, MODE>(rec, c, sig, lane);
+      group_sync(bar_id, GT);
     }
-  }
-
-  if (fold) {
-    // ---- fold (state route) and write-back
-    const float abar = sig[kMaxWindow];
+    // the positions are spread over the group's warps: this warp takes 0, GW + 1, ...
+    if (MODE == kModeReplay) {
+      if (NQ > 1 || CKPT != kCkptF32)
+        output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, kqraw, reuse, lane);
+      else
+        output_coefs_pairs<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, kqraw, reuse, lane);
+    }
+    group_sync(bar_id, GT);
+  } else {
+    float4 qr[NQR];
 #pragma unroll
-    for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
-    // rank-cf update: per entry, k_j's four columns and the weights of the thread's RT
-    // rows (two 16-byte reads), then 4 RT FMAs; the next entry is read ahead
-    const int wb = rbase < p.wt_stride ? rbase : 0;
-    float4 kt = IoT<IO>::load4(rec.k(0) + col * S_IO);
-    float4 w0 = *reinterpret_cast<const float4*>(wt + wb);
-    float4 w1 = *reinterpret_cast<const float4*>(wt + wb + 4);
-    for (int jj = 0; jj < cf; ++jj) {
-      const int jn = min(jj + 1, cf - 1);
-      const float4 kn = IoT<IO>::load4(rec.k(jn) + col * S_IO);
-      const float4 n0 = *reinterpret_cast<const float4*>(wt + (size_t)jn * p.wt_stride + wb);
-      const float4 n1 = *reinterpret_cast<const float4*>(wt + (size_t)jn * p.wt_stride + wb + 4);
-      const float ws8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    for (int s = 0; s < NQ; ++s)
+      qr[s] = (s < n) ? IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO) : make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // state rows of one row group (the read copy keeps its row scale for the dot product)
+    auto load_rows = [&](float4 (&x)[RT], int gi, bool dequant) {
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
-        x[r].x = fmaf(ws8[r], kt.x, x[r].x);
-        x[r].y = fmaf(ws8[r], kt.y, x[r].y);
-        x[r].z = fmaf(ws8[r], kt.z, x[r].z);
-        x[r].w = fmaf(ws8[r], kt.w, x[r].w);
-      }
-      kt = kn;
-      w0 = n0;
-      w1 = n1;
-    }
-    const bool store_f32 = (MODE != kModeEager) || (CKPT == kCkptF32);
-#pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      const int pr = rbase + r;
-      const size_t row = bh * PH + r0 + pr;
-      if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + row * N + col), x[r]);
-      if (CKPT != kCkptF32) {  // re-quantise the read copy (or the shared FP8 state) from the fresh row
-        const float am = seg_allmax<TPR>(amax4(x[r]));
-        float sc, inv;
-        if (CKPT == kCkptFp4) {
-          e2m1_row_scale(am, sc, inv);
-          if (pr < P)
-            __stcs(reinterpret_cast<unsigned short*>(p.S8 + row * (N / 2) + col / 2),
-                   static_cast<unsigned short>(quant4_e2m1(x[r], inv)));
-        } else {
-          e4m3_row_scale(am, sc, inv);
-          if (pr < P) __stcs(reinterpret_cast<unsigned int*>(p.S8 + row * N + col), quant4_e4m3(x[r], inv));
+        const int pr = gi * RGR + rbase + r;
+        x[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (pr < P) {
+          if (pl.fp32_tile) {
+            x[r] = *reinterpret_cast<const float4*>(tile + ((size_t)pr * N + col) * 4);
+          } else {
+            const float4 e =
+                (CKPT == kCkptFp4)
+                    ? e2m1x4_to_float4(*reinterpret_cast<const unsigned short*>(tile + (size_t)pr * (N / 2) + col / 2))
+                    : e4m3x4_to_float4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
+            if (dequant) {  // eager on a shared FP8 state: dequantise
+              const float sc = scale_tile[pr];
+              x[r] = make_float4(e.x * sc, e.y * sc, e.z * sc, e.w * sc);
+            } else {
+              x[r] = e;
+            }
+          }
         }
-        if (pr < P && (lane % TPR) == 0) p.Sscale[row] = sc;
       }
-    }
-  }
-  if (MODE == kModeFlush) return;
+    };
+    // the row dot products of one row group, reduced: lane holds rows base .. base+kHeld
+    float dv[NQR][Red::kHeld];
+    int dbase = 0;
+    bool dwr = false;
+    auto row_dots = [&](const float4 (&x)[RT]) {
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) {
+        if (s < n) {
+          float part[RT];
+#pragma unroll
+          for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
+          dwr = Red::run(part, lane, dbase);
+#pragma unroll
+          for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
+        }
+      }
+    };
+    // Multi-position calls, where a lane ends with one row (N >= 64): the v_l[p] of the
+    // first kPre window entries and the row's scale are read into registers before the
+    // group barrier, while the group forms the coefficients; after the barrier only the
+    // coefficients are read. (One-position calls measured no gain from it.)
+    constexpr int kPre = (MODE == kModeReplay && NQ > 1 && Red::kHeld == 1) ? 16 : 0;  // 0 or 16
+    float vpre[16];  // the first kPre used
+    float scpre = 1.f;
+    auto preload = [&](int gi, bool from_copy) {
+      if constexpr (kPre > 0) {
+        const int pr = gi * RGR + rbase + dbase;
+        const bool own = dwr && pr < P;
+        const int width = c + n - o0;
+#pragma unroll
+        for (int r = 0; r < kPre; ++r)
+          vpre[r] = (own && r < width) ? IoT<IO>::load1(rec.v(o0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
+        scpre = (own && from_copy) ? scale_tile[pr] : 1.f;
+      }
+    };
+    // y_s[p] = alpha_s d + sum_l cw[s][l] v_l[p] (replay) or y[p] = d (eager), by the
+    // lanes that hold row p's dot products; each v_l[p] is read once for all positions,
+    // eight entries in flight at a time (cw is zero past each position's window, v is
+    // zero past the unit's). `pre`: the preload above ran for this row group.
+    auto emit = [&](int gi, bool from_copy, bool pre) {
+      if (MODE == kModeFlush) return;
+#pragma unroll
+      for (int i = 0; i < Red::kHeld; ++i) {
+        const int pr = gi * RGR + rbase + dbase + i;
+        if (dwr && pr < P) {
+          const float sc = (kPre > 0 && pre) ? scpre : (from_copy ? scale_tile[pr] : 1.f);
+          if (MODE == kModeReplay && NQR == 1) {
+            const int last = c - o0;  // the one position replays window entries 0 .. last
+            float b0 = 0.f, b1 = 0.f;
+            int l0 = 0;
+            if (kPre > 0 && pre) {
+              const float4* c4 = reinterpret_cast<const float4*>(cw);
+              const float4 c0 = c4[0], c1 = c4[1], c2 = c4[2], c3 = c4[3];
+              b0 = fmaf(c0.x, vpre[0], fmaf(c0.y, vpre[1], fmaf(c0.z, vpre[2], fmaf(c0.w, vpre[3],
+                   fmaf(c1.x, vpre[4], fmaf(c1.y, vpre[5], fmaf(c1.z, vpre[6], c1.w * vpre[7])))))));
+              b1 = fmaf(c2.x, vpre[8], fmaf(c2.y, vpre[9], fmaf(c2.z, vpre[10], fmaf(c2.w, vpre[11],
+                   fmaf(c3.x, vpre[12], fmaf(c3.y, vpre[13], fmaf(c3.z, vpre[14], c3.w * vpre[15])))))));
+              l0 = kPre;
+            }
+            for (; l0 <= last; l0 += 8) {
+              float vv[8];
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+                vv[r] = (l0 + r <= last) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
+#pragma unroll
+              for (int r = 0; r < 8; r += 2) {
+                if (l0 + r <= last) b0 = fmaf(cw[l0 + r], vv[r], b0);
+                if (l0 + r + 1 <= last) b1 = fmaf(cw[l0 + r + 1], vv[r + 1], b1);
+              }
+            }
+            p.y[(((size_t)pl.b * n) * p.H + pl.h) * PH + r0 + pr] = fmaf(alpha[0], dv[0][i] * sc, b0 + b1);
+          } else if (MODE == kModeReplay) {
+            const int width = c + n - o0;
+            float b[NQR];
+#pragma unroll
+            for (int s = 0; s < NQR; ++s) b[s] = 0.f;
+            int l0 = 0;
+            if (kPre > 0 && pre) {
+#pragma unroll
+              for (int h = 0; h < kPre; h += 8) {
+                if (h < width) {
+#pragma unroll
+                  for (int s = 0; s < NQR; ++s) {
+                    if (s < n) {
+                      const float4 c0 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + h);
+                      const float4 c1 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + h + 4);
+                      const float* vv = vpre + h;
+                      b[s] = fmaf(c0.x, vv[0], fmaf(c0.y, vv[1], fmaf(c0.z, vv[2], fmaf(c0.w, vv[3],
+                             fmaf(c1.x, vv[4], fmaf(c1.y, vv[5], fmaf(c1.z, vv[6], fmaf(c1.w, vv[7], b[s]))))))));
+                    }
+                  }
+                }
+              }
+              l0 = kPre;
+            }
+            for (; l0 < width; l0 += 8) {
+              float vv[8];
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+                vv[r] = (l0 + r < width) ? IoT<IO>::load1(rec.v(o0 + l0 + r) + (size_t)(r0 + pr) * S_IO) : 0.f;
+#pragma unroll
+              for (int s = 0; s < NQR; ++s) {
+                if (s < n) {
+                  const float4 c0 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0);
+                  const float4 c1 = *reinterpret_cast<const float4*>(cw + s * kMaxWindow + l0 + 4);
+                  b[s] = fmaf(c0.x, vv[0], fmaf(c0.y, vv[1], fmaf(c0.z, vv[2], fmaf(c0.w, vv[3],
+                         fmaf(c1.x, vv[4], fmaf(c1.y, vv[5], fmaf(c1.z, vv[6], fmaf(c1.w, vv[7], b[s]))))))));
+                }
+              }
+            }
+#pragma unroll
+            for (int s = 0; s < NQR; ++s)
+              if (s < n) p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * PH + r0 + pr] = fmaf(alpha[s], dv[s][i] * sc, b[s]);
+          } else {
+            p.y[bh * PH + r0 + pr] = dv[0][i] * sc;
+          }
+        }
+      }
+    };
 
-  // ---- outputs: the rows' dot products with the queries, reduced over the row's lanes
-  static_assert(RT == kRowsPerThread, "one reduction per row group");
-  float dv[NQR][Red::kHeld];
-  int dbase = 0;
-  bool dwr = false;
+    float4 x[RT];
+    if (!fold) {
+      // ---- output-only route: row group 0's dot products, then wait for the buffer
+      // terms; further row groups (P > one row group) follow with the terms in hand
+      load_rows(x, 0, false);
+      row_dots(x);
+      preload(0, !pl.fp32_tile);
+      if (NQ > 1) output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, kqraw, reuse, lane);  // positions gw+1, ...
+      group_sync(bar_id, GT);
+      emit(0, !pl.fp32_tile, true);
+      for (int gi = 1; gi < ngroups; ++gi) {
+        load_rows(x, gi, false);
+        row_dots(x);
+        preload(gi, !pl.fp32_tile);
+        emit(gi, !pl.fp32_tile, true);
+      }
+    } else {
+      // ---- fold (state route), write the state back, outputs from the fresh rows
+      load_rows(x, 0, MODE == kModeEager);
+      group_sync(bar_id, GT);  // the fold weights are in
+      // wt[j][p] = sig_j v_j[p] (zero for p >= P), a thread per (8 entries, row): every
+      // load independent, consecutive threads on consecutive rows
+      for (int job = gtid; job < wts * ((cf + 7) / 8); job += GTG) {
+        const int j8 = job / wts;
+        const int pp = job - j8 * wts;
+        const int pv = pp < P ? pp : 0;
+        float wv[8];  // all eight reads first: the table writes could alias them
 #pragma unroll
-  for (int s = 0; s < NQR; ++s) {
-    if (s < n) {
-      const float4 qs = IoT<IO>::load4(qbuf + ((size_t)s * N + col) * S_IO);
-      float part[RT];
+        for (int r = 0; r < 8; ++r) {
+          const int jj = min(j8 * 8 + r, cf - 1);
+          wv[r] = sig[jj] * IoT<IO>::load1(rec.v(jj) + (size_t)(r0 + pv) * S_IO);
+        }
 #pragma unroll
-      for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qs);
-      dwr = Red::run(part, lane, dbase);
+        for (int r = 0; r < 8; ++r) {
+          const int jj = j8 * 8 + r;
+          if (jj < cf) wt[(size_t)jj * wts + pp] = pp < P ? wv[r] : 0.f;
+        }
+      }
+      group_sync(gemv_bar_id, GTG);
+      const float abar = sig[kMaxWindow];
+      for (int gi = 0; gi < ngroups; ++gi) {
+        if (gi > 0) load_rows(x, gi, MODE == kModeEager);
 #pragma unroll
-      for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
+        for (int r = 0; r < RT; ++r) x[r] = make_float4(abar * x[r].x, abar * x[r].y, abar * x[r].z, abar * x[r].w);
+        // rank-cf update: per entry, k_j's four columns of this lane and the weights of
+        // the thread's RT rows (four 16-byte broadcasts), then 4 * RT FMAs
+        const int wbase = (gi * RGR + rbase < P) ? gi * RGR + rbase : 0;  // all-invalid threads read row 0
+        // the next entry's k and weights are read while this entry's FMAs run
+        float4 kt = IoT<IO>::load4(rec.k(0) + col * S_IO);
+        float4 wcur[RT / 4];
+#pragma unroll
+        for (int r4 = 0; r4 < RT / 4; ++r4) wcur[r4] = reinterpret_cast<const float4*>(wt + wbase)[r4];
+        for (int jj = 0; jj < cf; ++jj) {
+          const int jn = min(jj + 1, cf - 1);
+          const float4 kn = IoT<IO>::load4(rec.k(jn) + col * S_IO);
+          float4 wn[RT / 4];
+#pragma unroll
+          for (int r4 = 0; r4 < RT / 4; ++r4) wn[r4] = reinterpret_cast<const float4*>(wt + (size_t)jn * wts + wbase)[r4];
+#pragma unroll
+          for (int r4 = 0; r4 < RT / 4; ++r4) {
+            const float ws4[4] = {wcur[r4].x, wcur[r4].y, wcur[r4].z, wcur[r4].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float4& xr = x[r4 * 4 + t];
+              xr.x = fmaf(ws4[t], kt.x, xr.x);
+              xr.y = fmaf(ws4[t], kt.y, xr.y);
+              xr.z = fmaf(ws4[t], kt.z, xr.z);
+              xr.w = fmaf(ws4[t], kt.w, xr.w);
+            }
+          }
+          kt = kn;
+#pragma unroll
+          for (int r4 = 0; r4 < RT / 4; ++r4) wcur[r4] = wn[r4];
+        }
+        // write the state: FP32 master, and/or the read copy's (or the shared FP8 state's)
+        // codes with per-row scales, re-quantised from the fresh row
+        const bool store_f32 = (MODE != kModeEager) || (CKPT == kCkptF32);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const int pr = gi * RGR + rbase + r;
+          const size_t row = bh * PH + r0 + pr;
+          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + row * N + col), x[r]);
+          if (CKPT != kCkptF32) {
+            const float am = seg_allmax<TPR>(amax4(x[r]));
+            float sc, inv;
+            if (CKPT == kCkptFp4) {
+              e2m1_row_scale(am, sc, inv);
+              if (pr < P)
+                __stcs(reinterpret_cast<unsigned short*>(p.S8 + row * (N / 2) + col / 2),
+                       static_cast<unsigned short>(quant4_e2m1(x[r], inv)));
+            } else {
+              e4m3_row_scale(am, sc, inv);
+              if (pr < P) __stcs(reinterpret_cast<unsigned int*>(p.S8 + row * N + col), quant4_e4m3(x[r], inv));
+            }
+            if (pr < P && (lane % TPR) == 0) p.Sscale[row] = sc;
+          }
+        }
+        if (MODE != kModeFlush) row_dots(x);
+        if (MODE == kModeReplay && NQ > 1 && gi == 0)
+          output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, kqraw, reuse, lane);
+        if (gi == 0) group_sync(bar_id, GT);  // the outputs' buffer terms are in
+        emit(gi, false, false);
+      }
     }
   }
-#pragma unroll
-  for (int i = 0; i < Red::kHeld; ++i) {
-    const int pr = rbase + dbase + i;
-    if (dwr && pr < P) {
-      if (MODE == kModeEager) {
-        p.y[bh * PH + r0 + pr] = dv[0][i];
-      } else {
-        const float sc = pl.fp32_tile ? 1.f : scale_tile[pr];
-#pragma unroll
-        for (int s = 0; s < NQR; ++s)
-          if (s < n)
-            p.y[(((size_t)pl.b * n + s) * p.H + pl.h) * PH + r0 + pr] =
-                fmaf(alpha[s], dv[s][i] * sc, u[s * p.u_stride + pr]);
-      }
+
+  // ---- publish the pointer word (the pre-pass already wrote this call's entries)
+  const int start = pl.start;
+  const int cap = p.cap;
+  if (MODE == kModeReplay) {
+    if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
+      int start2 = fold ? start + c : start;
+      start2 -= (start2 >= cap) ? cap : 0;
+      const int base = fold ? 0 : c;
+      const int cnt2 = base + (p.commit ? n : 0);
+      p.counts_out[pl.b] = (start2 << 16) | cnt2;
+      if (p.flushed && (!p.flushed_or || fold)) p.flushed[pl.b] = fold ? 1 : 0;
+    }
+  } else if (MODE == kModeFlush) {
+    if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
+      int start2 = start + c;
+      start2 -= (start2 >= cap) ? cap : 0;
+      p.counts_out[pl.b] = start2 << 16;
+      if (p.flushed) p.flushed[pl.b] = 1;
     }
   }
 }
 
-// The row warps' loop: every row warp takes every unit of the CTA in order, waiting for
-// the unit's tile (tfull) and its coefficients (cready); the warp's own waits for the
-// uses before came first, so both parity waits are exact. Releasing a unit frees its
-// tile stage and its record stage, and counts the release for the coefficient warps.
-template <int N, typename IO, int CKPT, int MODE, int NQ>
-__device__ void row_loop(const KParams& p, uint8_t* tstages, uint8_t* rstages, Bars* bars, int warp, int lane) {
-  constexpr int S_IO = IoT<IO>::bytes;
-  const int NT = p.num_tstages, NR = p.num_rstages;
-  const int total = cta_units(p);
-  for (int i = 0; i < total; ++i) {
-    const int st_t = i % NT, st_r = i % NR;
-    bool ready = *reinterpret_cast<volatile int*>(&bars->abort_flag) == 0;
-    if (ready) ready = mbar_wait_bounded(&bars->tfull[st_t], (i / NT) & 1);
-    if (ready) ready = mbar_wait_bounded(&bars->cready[st_r], (i / NR) & 1);
-    if (!__all_sync(0xffffffffu, ready)) {
-      if (lane == 0) {
-        report_error(p.status, kErrWaitTimeout);
-        bars->abort_flag = 1;
-      }
-      break;
-    }
-    const uint8_t* tst = tstages + (size_t)st_t * p.tstage_bytes;
-    const uint8_t* rst = rstages + (size_t)st_r * p.rstage_bytes;
-    const int32_t word = reinterpret_cast<const int32_t*>(rst + p.off_meta)[0];
-    const int msk = reinterpret_cast<const int32_t*>(rst + p.off_meta)[1];
-    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, cta_unit(p, i), word, msk);
-    if (pl.active) row_unit<N, IO, CKPT, MODE, NQ>(p, pl, tst, rst, warp, lane);
-    count_release(&bars->released[st_r], lane);
-    mbar_arrive(&bars->rempty[st_r]);
-    mbar_arrive(&bars->tempty[st_t]);
-  }
-}
-
-template <int N, typename IO, int CKPT, int MODE, int NQ>
+template <int N, typename IO, int CKPT, int MODE, int NQ, int NG>
 __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_constant__ KParams p) {
+  static_assert(NG == 1 || NG == 2, "the stage protocol relies on a stage's uses two apart being one group's");
   static_assert(kProducerWarps == 1, "stages must be filled in unit order");
+  using Gr = Groups<NG>;
   extern __shared__ __align__(128) uint8_t smem[];
   Bars* bars = reinterpret_cast<Bars*>(smem);
-  uint8_t* tstages = smem + p.tstages_off;
-  uint8_t* rstages = smem + p.rstages_off;
+  uint8_t* stages = smem + p.stages_off;
   constexpr int S_IO = IoT<IO>::bytes;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.num_tstages; ++s) {
-      mbar_init(&bars->tfull[s], 1);                  // the producer's expect_tx
-      mbar_init(&bars->tempty[s], kRowWarps * 32);    // every row warp's lanes
-    }
-    for (int s = 0; s < p.num_rstages; ++s) {
-      mbar_init(&bars->rfull[s], MODE == kModeEager ? 32 : 1);  // the eager gather: 32 lanes' cp.async
-      mbar_init(&bars->cready[s], 32);                // a coefficient warp's lanes
-      mbar_init(&bars->rempty[s], kRowWarps * 32);    // every row warp's lanes
+    for (int s = 0; s < p.num_stages; ++s) {
+      // the producer's expect_tx (the eager gather adds its 32 lanes' cp.async arrivals)
+      mbar_init(&bars->full[s], MODE == kModeEager ? 1 + 32 : 1);
+      mbar_init(&bars->empty[s], Gr::kThreads);
     }
     bars->abort_flag = 0;
-    for (int s = 0; s < kMaxTileStages; ++s) bars->last_tfill[s] = -1;
-    for (int s = 0; s < kMaxRecStages; ++s) {
-      bars->last_rfill[s] = -1;
-      bars->released[s] = 0;
-    }
+    for (int s = 0; s < kMaxStages; ++s) bars->last_fill[s] = -1;
     fence_mbar_init();
   }
   __syncthreads();
   if constexpr (MODE == kModeReplay && NQ == 1) {
-    // One-position calls append their entries here rather than in a pre-pass: the row and
-    // coefficient warps write the new ring records of the CTA's heads (v, then Delta and a
-    // in one 16-byte piece; k once per chunk), make the writes visible to the bulk copies
-    // that read them, and tell the producer, which meanwhile streams the first tiles.
-    if (p.append_here && threadIdx.x < kWorkerWarps * 32) {
+    // One-position calls append their entries here rather than in a pre-pass: each CTA
+    // writes the new ring record of each of its own units (k, v, then Delta and a in one
+    // 16-byte piece), makes the writes visible to the bulk copies that read them, and
+    // tells the producer, which meanwhile streams the first state tiles.
+    if (p.append_here && threadIdx.x < kConsumerWarps * 32) {
       append_entries<S_IO>(p);
       named_arrive(kAppendBar, kThreads);
     }
   }
 
   const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (warp >= kWorkerWarps) {
+  if (warp >= kConsumerWarps) {
     if constexpr (MODE == kModeEager)
-      producer_loop_eager<CKPT, S_IO>(p, tstages, rstages, bars);
+      producer_loop_eager<CKPT, S_IO>(p, stages, bars);
     else
-      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, tstages, rstages, bars);
-  } else if (warp >= kRowWarps) {
-    const int cwarp = warp - kRowWarps;
-    float* kq = reinterpret_cast<float*>(smem + p.ws_off + (size_t)cwarp * p.ws_bytes);
-    coef_loop<N, IO, CKPT, MODE, NQ>(p, rstages, bars, kq, kq + p.ws_bytes / 8, cwarp, lane);
-  } else {
-    row_loop<N, IO, CKPT, MODE, NQ>(p, tstages, rstages, bars, warp, lane);
+      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, stages, bars);
+    return;
+  }
+  const int g = warp / Gr::kWarps;  // consumer group
+  const int gtid = threadIdx.x - g * Gr::kThreads;
+  const int bar_id = 1 + g;                 // the whole group
+  const int gemv_bar_id = 1 + NG + g;       // the group's row warps only
+  uint8_t* ws = smem + p.ws_off + (size_t)g * p.ws_group_bytes;
+  const int NS = p.num_stages;
+  const int total = cta_units(p);
+  int prev_bg = -1;  // (sequence, k/q group) of the group's previous unit, -1 if none
+  int s = g, k = 0;  // stage and use of unit i, advanced without divisions
+  while (s >= NS) {
+    s -= NS;
+    ++k;
+  }
+  for (int i = g; i < total; i += NG) {
+    // Parity waits only tell apart a phase and the one just before it, so before waiting
+    // for its own fill (phase k of "full"), a group waits for the stage's previous use to
+    // be released (phase k-1 of "empty"). That release may come from the other group;
+    // the use before it (k-2) was this group's own, already released, so both waits are
+    // exact even when the two groups drift apart.
+    bool ready = true;
+    if (k > 0) ready = mbar_wait_bounded(&bars->empty[s], (k - 1) & 1);
+    if (ready) ready = mbar_wait_bounded(&bars->full[s], k & 1);
+    const bool ok = group_all(ready, bar_id, Gr::kThreads);
+    if (!ok) {
+      if (gtid == 0) {
+        report_error(p.status, kErrWaitTimeout);
+        bars->abort_flag = 1;
+      }
+      break;
+    }
+    uint8_t* st = stages + (size_t)s * p.stage_bytes;
+    const int4 m0 = reinterpret_cast<const int4*>(st + p.off_meta)[0];  // word, mask, b, h
+    const int4 m1 = reinterpret_cast<const int4*>(st + p.off_meta)[1];  // g, rb
+    const int32_t word = m0.x;
+    const int msk = m0.y;
+    const Plan pl = make_plan<MODE, CKPT, S_IO>(p, UnitIdx{m0.z, m0.w, m1.x, m1.y}, word, msk);
+    // the group's previous unit had the same sequence and k/q group: its k . q products hold
+    const int bg = pl.b * p.G + pl.g;
+    const bool reuse = bg == prev_bg;
+    prev_bg = pl.active ? bg : -1;
+    if (pl.active) {
+      consume_unit<N, IO, CKPT, MODE, NQ, NG>(p, pl, st, ws, gtid, bar_id, gemv_bar_id, reuse);
+    } else if (pl.h == 0 && pl.rb == 0 && gtid == 0) {
+      p.counts_out[pl.b] = word;  // nothing to fold: the pointer word carries over
+      if (MODE == kModeFlush && p.flushed && !pl.corrupt) p.flushed[pl.b] = 0;
+    }
+    group_sync(bar_id, Gr::kThreads);
+    mbar_arrive(&bars->empty[s]);
+    s += NG;
+    while (s >= NS) {
+      s -= NS;
+      ++k;
+    }
   }
 }
 

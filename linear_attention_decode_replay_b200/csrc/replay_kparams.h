@@ -40,16 +40,14 @@ struct KParams {
   const int32_t* counts_in;
   int32_t* counts_out;
   int32_t* status;
-  // shared-memory layout, bytes: a ring of tile stages and a deeper ring of record stages
-  // (records, queries, pointer word, coefficients); a unit's records are copied
-  // `lookahead` units before its tile
-  int32_t num_tstages, tstage_bytes, tstages_off;
-  int32_t num_rstages, rstage_bytes, rstages_off, lookahead;
+  // shared-memory layout, bytes: a ring of stages, each holding one unit's tile, records,
+  // queries and pointer word; one workspace per consumer group
+  int32_t num_stages, stage_bytes, stages_off;
   int32_t rec_bytes, rec_k_bytes, qpack_pos;   // head / k record sizes; positions per qpack group
-  int32_t off_krec, off_rec, off_q, off_meta, off_coef;  // within a record stage
-  int32_t co_alpha, co_sig, co_u, co_wt;       // within a stage's coefficient area
-  int32_t u_stride, wt_stride;                 // floats per position of u, per entry of wt (= rows_unit)
-  int32_t ws_off, ws_bytes;                    // one scratch area per coefficient warp
+  int32_t off_krec, off_rec, off_q, off_meta;  // within a stage
+  int32_t ws_off, ws_group_bytes;              // one workspace per consumer group
+  int32_t ws_alpha, ws_sig, ws_cw, ws_kq, ws_wt;  // within a group's workspace
+  int32_t wt_stride;                           // row stride of the fold weight table [L][wt_stride]
   int32_t smem_bytes;
 };
 

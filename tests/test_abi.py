@@ -53,8 +53,8 @@ def test_ring_capacity_and_config_checks():
     # head record: v (P io) + Delta + a, padded to 16 bytes; k record: k (N io), once per group
     assert lib.replay_ring_record_bytes(ctypes.byref(_cfg())) == 80  # 16 * 4 + 8 -> 80
     assert lib.replay_ring_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 144  # 136 -> 144
-    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg())) == 64
-    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 256
+    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg())) == 64 + 16  # k, then 16 bytes of padding
+    assert lib.replay_ring_k_record_bytes(ctypes.byref(_cfg(P=64, N=128, io=_abi.REPLAY_BF16))) == 256 + 16
     for bad in (dict(groups=3), dict(P=12), dict(P=0), dict(N=48), dict(N=256), dict(L=0),
                 dict(max_pos=9), dict(max_pos=5, L=4), dict(io=7), dict(ckpt=3), dict(ckpt=-1), dict(batch=0),
                 dict(P=256, N=128)):
@@ -66,11 +66,11 @@ def test_ring_capacity_and_config_checks():
 def test_snapshot_bytes():
     lib = _abi.load()
     # header 64 + H*P*N*4 + G*L*RK + H*L*R
-    assert lib.replay_snapshot_bytes(ctypes.byref(_cfg())) == 64 + 4 * 16 * 16 * 4 + 2 * 4 * 64 + 4 * 4 * 80
+    assert lib.replay_snapshot_bytes(ctypes.byref(_cfg())) == 64 + 4 * 16 * 16 * 4 + 2 * 4 * 80 + 4 * 4 * 80
     big = _cfg(batch=256, heads=64, groups=64, P=64, N=128, L=16, max_pos=1, io=_abi.REPLAY_BF16)
-    assert lib.replay_snapshot_bytes(ctypes.byref(big)) == 64 + 64 * 64 * 128 * 4 + 64 * 16 * 256 + 64 * 16 * 144
+    assert lib.replay_snapshot_bytes(ctypes.byref(big)) == 64 + 64 * 64 * 128 * 4 + 64 * 16 * 272 + 64 * 16 * 144
     shared = _cfg(batch=256, heads=64, groups=8, P=64, N=128, L=16, max_pos=1, io=_abi.REPLAY_BF16)
-    assert lib.replay_snapshot_bytes(ctypes.byref(shared)) == 64 + 64 * 64 * 128 * 4 + 8 * 16 * 256 + 64 * 16 * 144
+    assert lib.replay_snapshot_bytes(ctypes.byref(shared)) == 64 + 64 * 64 * 128 * 4 + 8 * 16 * 272 + 64 * 16 * 144
     assert lib.replay_snapshot_bytes(ctypes.byref(_cfg(groups=3))) == _abi.REPLAY_EINVAL
 
 

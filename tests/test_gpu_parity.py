@@ -69,6 +69,9 @@ RAGGED = [
     gen.Shape("r5", B=4, H=1, G=1, P=64, N=128, L=16, io="bf16", s0="prefill", seed=15),
     # two row-block units per head (N = 64: 128 rows per unit), a group shared by two heads
     gen.Shape("r6", B=3, H=2, G=1, P=256, N=64, L=4, io="bf16", seed=16),
+    # eight heads per group: a CTA takes them in a row, and each consumer group forms the
+    # k . q products once for its units of the chunk and reuses them
+    gen.Shape("r7", B=3, H=16, G=2, P=32, N=64, L=5, io="bf16", seed=17),
 ]
 
 
@@ -91,6 +94,8 @@ SPEC = [
     gen.Shape("s3", B=2, H=2, G=1, P=64, N=128, L=16, io="bf16", max_pos=8, seed=23),
     # two row-block units per head: every unit replays the same records for its rows
     gen.Shape("s5", B=3, H=2, G=2, P=128, N=128, L=8, io="bf16", max_pos=5, seed=25),
+    # four heads per group: the products of every position are reused across a chunk
+    gen.Shape("s6", B=3, H=8, G=2, P=32, N=64, L=6, io="f32", max_pos=5, seed=26),
 ]
 
 

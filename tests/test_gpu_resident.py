@@ -34,7 +34,9 @@ def _write_records(layer, slots, x, n_pos):
         pick = (lambda t: t[:, s]) if x["k"].dim() == 4 else (lambda t: t)  # verify inputs carry n_pos
         k, v, dt, a = pick(x["k"]), pick(x["v"]), pick(x["dt"]), pick(x["a"])
         slot = ((slots.long() + s) % cap)[:, None]
-        ring_k[bi, gi, slot] = k.contiguous().view(torch.uint8).reshape(B, G, N * s_io)
+        krec = torch.zeros(B, G, ring_k.shape[3], dtype=torch.uint8, device=ring.device)  # k, then padding
+        krec[:, :, :N * s_io] = k.contiguous().view(torch.uint8).reshape(B, G, N * s_io)
+        ring_k[bi, gi, slot] = krec
         rec = torch.zeros(B, H, R, dtype=torch.uint8, device=ring.device)
         rec[:, :, :P * s_io] = v.contiguous().view(torch.uint8).reshape(B, H, P * s_io)
         rec[:, :, P * s_io:P * s_io + 8] = torch.stack([dt, a], -1).contiguous().view(torch.uint8).reshape(B, H, 8)

@@ -21,7 +21,6 @@ constexpr int kMaxWindow = 32;                   // largest L (decay scans use o
 constexpr int kMaxStages = 8;
 constexpr int kMaxChunkHeads = 8;                // heads of one k/q group a CTA takes in a row
 constexpr int kUnitsPerIssue = 2;                // units whose copies share one bulk-copy instruction
-constexpr int kAppendBar = 15;                   // named barrier: entries appended -> producer
 constexpr int kRowsPerThread = 16;               // state rows one thread covers per row group
 constexpr int kHeaderBytes = 256;                // the mbarriers and flags at the start of shared memory
 // State rows of one row group: kGroupGemvWarps warps, 128/N rows per warp pass (a row of

@@ -68,8 +68,8 @@ struct Plan {
 // chunks of chunk_heads consecutive heads of one k/q group (the group, or a part of it),
 // chunk c on CTA c mod gridDim.x, each head with its row blocks in a row. Dealing the
 // chunks round-robin keeps the CTAs on neighbouring tiles of the state at any moment,
-// one CTA holds every unit of a head (the in-kernel append writes a head's new record
-// once, before any copy of it), and a chunk's heads share one k record write.
+// and a consumer group that takes several heads of one chunk forms their k . q products
+// once.
 __device__ __forceinline__ int cta_chunks(const KParams& p) {
   return (p.num_chunks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 }
@@ -135,9 +135,13 @@ __device__ __forceinline__ Plan make_plan(const KParams& p, const UnitIdx& x, in
     pl.bytes = 0;
     return pl;
   }
-  const uint32_t records = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
+  // ring records copied: the buffered ones and, unless this call's entry comes straight
+  // from the inputs (one-position calls), the new ones the pre-pass appended
+  const bool from_inputs = MODE == kModeReplay && p.append_here;
+  const uint32_t records = pl.c + ((MODE == kModeReplay && !from_inputs) ? p.n_pos : 0);
   pl.bytes = (pl.fp32_tile ? P * N * 4u : P * (N / kCodeDiv) + P * 4u) +
-             records * (uint32_t)(p.rec_bytes + p.rec_k_bytes) + ((MODE == kModeReplay) ? p.n_pos * N * S_IO : 0u);
+             records * (uint32_t)(p.rec_bytes + p.rec_k_bytes) + ((MODE == kModeReplay) ? p.n_pos * N * S_IO : 0u) +
+             (from_inputs ? (N + (uint32_t)p.P) * S_IO : 0u);
   return pl;
 }
 
@@ -159,72 +163,17 @@ struct Records {
   }
 };
 
-// ---------------------------------------------------------------------------- append
-// This CTA's units' new entries (one position) into their ring records, slot
-// (start + c) mod cap, by the consumer threads before any bulk copy is issued: each head's
-// v, then Delta and a in one 16-byte piece, and the group's k once per chunk (a group of
-// more than kMaxChunkHeads heads spans chunks, possibly on several CTAs, each writing the
-// same bytes before it reads them). The input pieces do not depend on the pointer word,
-// so both reads are in flight together.
-template <int S_IO>
-__device__ __forceinline__ void append_entries(const KParams& p) {
-  constexpr int kPool = kConsumerWarps * 32;
-  constexpr int kBatch = 8;  // pieces per thread in flight
-  const int kpe = p.N * S_IO / 16;  // 16-byte pieces of k
-  const int vpe = p.P * S_IO / 16;  // of v
-  const int per_unit = kpe + vpe + 1;
-  const int total = cta_chunks(p) * p.chunk_heads * per_unit;
-  for (int t0 = threadIdx.x; t0 < total; t0 += kBatch * kPool) {
-    uint4 val[kBatch];
-    uint8_t* dst[kBatch];
-#pragma unroll
-    for (int r = 0; r < kBatch; ++r) {
-      const int t = t0 + r * kPool;
-      dst[r] = nullptr;
-      val[r] = make_uint4(0u, 0u, 0u, 0u);
-      if (t < total) {
-        const int iu = t / per_unit;
-        const int ch = t - iu * per_unit;
-        const int bh = cta_head(p, iu);
-        const int b = bh / p.H;
-        const int h = bh - b * p.H;
-        const int g = h / p.hpg;
-        const bool k_here = (iu % p.chunk_heads) == 0;  // the chunk's first head writes the group's k
-        const int32_t word = __ldg(p.counts_in + b);
-        if (ch < kpe) {
-          if (k_here)
-            val[r] = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.k) + ((size_t)b * p.G + g) * p.N * S_IO)[ch];
-        } else if (ch < kpe + vpe) {
-          val[r] = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.v) + ((size_t)b * p.H + h) * p.P * S_IO)[ch - kpe];
-        } else {
-          val[r].x = __float_as_uint(__ldg(p.dt + (size_t)b * p.H + h));
-          val[r].y = __float_as_uint(__ldg(p.a + (size_t)b * p.H + h));
-        }
-        const int start = word >> 16;
-        const int c = word & 0xFFFF;
-        if (!(word < 0 || c > p.L || start >= p.cap) && (ch >= kpe || k_here)) {  // a bad word is reported by the consumers
-          int slot = start + c;
-          slot -= (slot >= p.cap) ? p.cap : 0;
-          dst[r] = ch < kpe ? static_cast<uint8_t*>(p.ring_k) + (((size_t)b * p.G + g) * p.cap + slot) * p.rec_k_bytes + (size_t)ch * 16
-                            : static_cast<uint8_t*>(p.ring) + (((size_t)b * p.H + h) * p.cap + slot) * p.rec_bytes + (size_t)(ch - kpe) * 16;
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kBatch; ++r)
-      if (dst[r]) *reinterpret_cast<uint4*>(dst[r]) = val[r];
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------- producer
 // Copies of one unit, one bulk copy (TMA) per kind: 0 the state tile (the unit's rows),
 // 1 their read-copy row scales, 2-3 the head's live records and 4-5 the live k records
 // of its group, [start, start + count) modulo cap in one or two pieces (whole records:
-// every row block reads all of k and its rows of v), 6 the queries. A producer lane
-// always issues the same kind, so it works out what does not depend on the unit once:
-// its source array and the strides that place a unit in it.
-constexpr int kCopyKinds = 7;
+// every row block reads all of k and its rows of v), 6 the queries, and for one-position
+// calls the new entry straight from the inputs, 7 its k and 8 its v, into record c of the
+// stage (the producer stores its Delta and a there itself; the consumers append the
+// entry to the ring later, off the stream's path). A producer lane always issues the
+// same kind, so it works out what does not depend on the unit once: its source array and
+// the strides that place a unit in it.
+constexpr int kCopyKinds = 9;
 struct LaneCopy {
   const uint8_t* base;       // source array (kind 0: the FP32 master)
   const uint8_t* base_copy;  // kind 0-1 with a read copy: the codes / scales array
@@ -267,10 +216,20 @@ __device__ __forceinline__ LaneCopy lane_copy(const KParams& p, int kind) {
     lc.rec = p.rec_k_bytes;
     lc.stride = (uint64_t)p.cap * lc.rec;
     lc.dst_off = p.off_krec;
-  } else {
+  } else if (kind == 6) {
     lc.base = static_cast<const uint8_t*>(p.qpack ? p.qpack : p.q);
     lc.stride = (uint64_t)(p.qpack ? p.qpack_pos : 1) * N * S_IO;
     lc.dst_off = p.off_q;
+  } else if (kind == 7) {
+    lc.base = static_cast<const uint8_t*>(p.k);
+    lc.stride = (uint64_t)N * S_IO;
+    lc.rec = p.rec_k_bytes;
+    lc.dst_off = p.off_krec;
+  } else {
+    lc.base = static_cast<const uint8_t*>(p.v);
+    lc.stride = (uint64_t)P * S_IO;
+    lc.rec = p.rec_bytes;
+    lc.dst_off = p.off_rec;
   }
   return lc;
 }
@@ -282,7 +241,8 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const LaneCopy& 
   const uint32_t rows = pl.rows, N = p.N;
   const int bh = pl.b * p.H + pl.h;
   const int bg = pl.b * p.G + pl.g;
-  const int cnt = pl.c + ((MODE == kModeReplay) ? p.n_pos : 0);
+  const bool from_inputs = MODE == kModeReplay && p.append_here;
+  const int cnt = pl.c + ((MODE == kModeReplay && !from_inputs) ? p.n_pos : 0);  // ring records
   const int first = min(cnt, p.cap - pl.start);
   const bool copy = !pl.fp32_tile;  // kinds 0-1 read the read copy
   uint32_t bytes;
@@ -298,10 +258,14 @@ __device__ __forceinline__ uint32_t unit_copy(const KParams& p, const LaneCopy& 
     src = lc.base + (uint64_t)((lc.kind <= 3) ? bh : bg) * lc.stride + (second ? 0u : (uint32_t)pl.start * lc.rec);
     dst = st + lc.dst_off + (second ? (uint32_t)first * lc.rec : 0u);
     bytes = (uint32_t)(second ? cnt - first : first) * lc.rec;
-  } else {
+  } else if (lc.kind == 6) {
     src = lc.base + (uint64_t)bg * lc.stride;
     dst = st + lc.dst_off;
     bytes = (MODE == kModeReplay) ? (uint32_t)p.n_pos * N * S_IO : 0u;
+  } else {  // the new entry's k (7) or v (8), into record c
+    src = lc.base + (uint64_t)((lc.kind == 7) ? bg : bh) * lc.stride;
+    dst = st + lc.dst_off + (uint32_t)pl.c * lc.rec;
+    bytes = from_inputs ? (uint32_t)lc.stride : 0u;
   }
   return pl.active ? bytes : 0u;
 }
@@ -322,7 +286,7 @@ __device__ __forceinline__ void write_meta(uint8_t* st, const KParams& p, const 
 // fed; the per-unit arithmetic is kept short for the same reason (the producer's loop,
 // not the memory, bounds a stream of small tiles): every 32 units, lane L works out
 // unit L's indices (the divisions) and reads its pointer word, once, one chunk ahead.
-template <int MODE, int CKPT, int S_IO, bool APPEND>
+template <int MODE, int CKPT, int S_IO>
 __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   constexpr int U = kUnitsPerIssue;
   static_assert(U * kCopyKinds <= 32 && (32 % U) == 0, "a batch's copies must fit one warp and tile 32 units");
@@ -331,20 +295,28 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
   const uint64_t stream_policy = l2_evict_first_policy();
   const uint64_t keep_policy = l2_evict_normal_policy();
   const int total = cta_units(p);
+  const bool from_inputs = MODE == kModeReplay && p.append_here;  // one-position call's entry
   struct Pre {
     UnitIdx x;
     int32_t word;
     int msk;
+    float dt, a;  // the new entry's Delta and a (one-position calls)
   };
   auto prefetch = [&](int i0) {
     Pre q;
     q.x = UnitIdx{0, 0, 0, 0};
     q.word = 0;
     q.msk = 1;
+    q.dt = q.a = 0.f;
     if (i0 + lane < total) {
       q.x = unit_idx(p, cta_unit(p, i0 + lane));
       q.word = __ldg(p.counts_in + q.x.b);
       if (MODE == kModeFlush && p.mask) q.msk = __ldg(p.mask + q.x.b);
+      if (from_inputs) {
+        const size_t bh = (size_t)q.x.b * p.H + q.x.h;
+        q.dt = __ldg(p.dt + bh);
+        q.a = __ldg(p.a + bh);
+      }
     }
     return q;
   };
@@ -357,38 +329,14 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     r.x.rb = __shfl_sync(0xffffffffu, q.x.rb, src);
     r.word = __shfl_sync(0xffffffffu, q.word, src);
     r.msk = __shfl_sync(0xffffffffu, q.msk, src);
+    r.dt = __shfl_sync(0xffffffffu, q.dt, src);
+    r.a = __shfl_sync(0xffffffffu, q.a, src);
     return r;
   };
   Pre cur = prefetch(0), nxt = prefetch(32);
   const int j = lane / kCopyKinds;     // this lane's unit within the batch
   const int kind = lane % kCopyKinds;  // and its copy
   const LaneCopy lc = lane_copy<MODE, CKPT, S_IO>(p, kind);
-  // When the kernel appends this call's entries itself, the first stages' state tiles
-  // (and read-copy scales) go out at once and their records and queries once the entries
-  // are in the ring; every stage is armed with its unit's full byte count either way.
-  int pre = 0;
-  if (APPEND && p.append_here) {
-    pre = min(NS, total);
-    for (int i = 0; i < pre; ++i) {
-      const Pre u = fetch(cur, i);
-      const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u.x, u.word, 1);
-      uint8_t* st = stages + (size_t)i * p.stage_bytes;
-      if (lane == 0) {
-        write_meta(st, p, u.x, u.word, 1);
-        if (pl.corrupt) report_error(p.status, kErrPointer);
-        mbar_arrive_expect_tx(&bars->full[i], pl.bytes);
-      }
-      __syncwarp();
-      const uint8_t* src;
-      uint8_t* dst;
-      uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, lc, pl, st, src, dst);
-      if (lane > 1) bytes = 0;
-      __syncwarp();
-      if (bytes) bulk_g2s_hint(dst, src, bytes, &bars->full[i], lane == 0 ? stream_policy : keep_policy);
-      if (lane == 0) bars->last_fill[i] = i;
-    }
-    group_sync(kAppendBar, kThreads);  // the entries are in the ring
-  }
   // stage and use of the batch's first unit, advanced without divisions
   int s0 = 0, k0 = 0;
   for (int i0 = 0; i0 < total; i0 += U) {
@@ -432,17 +380,19 @@ __device__ void producer_loop(const KParams& p, uint8_t* stages, Bars* bars) {
     uint8_t* st = stages + (size_t)s * p.stage_bytes;
     uint64_t* bar = &bars->full[s];
     const Plan pl = make_plan<MODE, CKPT, S_IO>(p, u.x, u.word, u.msk);
-    const bool armed = i < pre;  // tile already issued, stage already armed
-    if (valid && kind == 0 && !armed) {
+    if (valid && kind == 0) {
       write_meta(st, p, u.x, u.word, u.msk);
       if (pl.corrupt) report_error(p.status, kErrPointer);
+      if (from_inputs && pl.active)  // the new entry's Delta, a (and zero padding) after its v
+        *reinterpret_cast<float4*>(st + p.off_rec + (size_t)pl.c * p.rec_bytes + (size_t)p.P * S_IO) =
+            make_float4(u.dt, u.a, 0.f, 0.f);
       mbar_arrive_expect_tx(bar, pl.bytes);
     }
     __syncwarp();
     const uint8_t* src;
     uint8_t* dst;
     uint32_t bytes = unit_copy<MODE, CKPT, S_IO>(p, lc, pl, st, src, dst);
-    if (!valid || (armed && kind <= 1)) bytes = 0;
+    if (!valid) bytes = 0;
     __syncwarp();
     if (bytes) bulk_g2s_hint(dst, src, bytes, bar, kind == 0 ? stream_policy : keep_policy);
     if (valid && kind == 0) bars->last_fill[s] = i;
@@ -565,9 +515,9 @@ __device__ __forceinline__ void fold_weights(const Records<N, IoT<IO>::bytes>& r
 //    per group forms the coefficients while four stream the state and its chain is on
 //    the unit's critical path: a lane pair per entry, sixteen entries per pass (half of k_l . q_s per lane,
 //    the second half one 4-element chunk rotated so that the pair's reads fall in
-//    different shared-memory banks, one shuffle to combine), and each lane forms its
-//    entry's decay weight itself from broadcast reads of the a_i. Its chain is one round
-//    of shared-memory reads, the products and one shuffle.
+//    different shared-memory banks, one shuffle to combine), and the decay weights from
+//    one suffix-product scan of the window's a_i (one read per lane, five shuffles).
+//    Its chain is one round of shared-memory reads, the products and a few shuffles.
 //  * output_coefs_quarters, for multi-position calls, where all five warps of a group
 //    form coefficients at once and the shared-memory pipe, not one warp's chain, is the
 //    limit, and for the FP8 / FP4 read copies, whose row warps (decoding the codes) rather than
@@ -637,20 +587,23 @@ __device__ __forceinline__ void output_coefs_pairs(const Records<N, IoT<IO>::byt
   constexpr int S_IO = IoT<IO>::bytes;
   constexpr int HN = N / 2;       // elements of half a row
   constexpr int HC = HN / 4;      // 4-element chunks of half a row
-  constexpr int kBlock = 16;      // decay factors read per round
   const int width = c + n - o0;   // window entries (at most kMaxWindow)
   const int half = lane & 1;
-  for (int e0 = 0; e0 < width; e0 += 16) {
-    const int e = e0 + (lane >> 1);
-    const int er = (e < width) ? e : width - 1;  // lanes past the window read a valid record
-    const uint8_t* kh = rec.k(o0 + er) + (size_t)half * HN * S_IO;
-    const float xd = rec.dt(o0 + er);
-    for (int s = s0; s < n; s += ds) {
-      const int last = c + s - o0;  // position s replays window entries 0 .. last
+  // the window's decay factors, lane l holding a_{o0+l}: read once, then one suffix-
+  // product scan per position gives every product the weights need
+  const float al = (lane < width) ? rec.a(o0 + lane) : 1.f;
+  for (int s = s0; s < n; s += ds) {
+    const int last = c + s - o0;  // position s replays window entries 0 .. last
+    const float suf = warp_suffix_prod(lane <= last ? al : 1.f, lane);  // prod_{lane <= i <= last} a_i
+    if (lane == 0) alpha[s] = suf;
+    for (int e0 = 0; e0 < width; e0 += 16) {
+      const int e = e0 + (lane >> 1);
+      const int er = (e < width) ? e : width - 1;  // lanes past the window read a valid record
       float kq;
       if (reuse) {  // the group's previous unit had the same sequence and k/q group
         kq = kqraw[s * kMaxWindow + e];
       } else {
+        const uint8_t* kh = rec.k(o0 + er) + (size_t)half * HN * S_IO;
         const uint8_t* qh = qbuf + ((size_t)s * N + half * HN) * S_IO;
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -664,20 +617,37 @@ __device__ __forceinline__ void output_coefs_pairs(const Records<N, IoT<IO>::byt
         kq += __shfl_xor_sync(0xffffffffu, kq, 1);
         if (half == 0) kqraw[s * kMaxWindow + e] = kq;
       }
-      // prod_{e < i <= last} a_i; i runs from e0 + 1 (i <= e0 never counts for this pass)
-      float w = 1.f;
-      float a_first = 1.f;  // a_{o0}, for alpha
-      for (int t0 = (e0 == 0) ? 0 : e0 + 1; t0 <= last; t0 += kBlock) {
-        float at[kBlock];
-#pragma unroll
-        for (int r = 0; r < kBlock; ++r) at[r] = (t0 + r <= last) ? rec.a(o0 + t0 + r) : 1.f;
-        if (t0 == 0) a_first = at[0];
-#pragma unroll
-        for (int r = 0; r < kBlock; ++r) w = (t0 + r > e) ? w * at[r] : w;
-      }
-      if (half == 0 && e < kMaxWindow) cw[s * kMaxWindow + e] = (e <= last) ? xd * w * kq : 0.f;
-      if (lane == 0 && e0 == 0) alpha[s] = a_first * w;  // prod_{0 <= i <= last} a_i
+      // prod_{e < i <= last} a_i: the scan's value one lane up (empty past lane 31)
+      const float up = __shfl_sync(0xffffffffu, suf, (e + 1) & 31);
+      const float w = (e + 1 < 32) ? up : 1.f;
+      if (half == 0 && e < kMaxWindow) cw[s * kMaxWindow + e] = (e <= last) ? rec.dt(o0 + er) * w * kq : 0.f;
     }
+  }
+}
+
+// One-position calls copy their new entry from the inputs into record c of each unit's
+// stage; the coefficient warp then appends it to the ring at slot (start + c) mod cap for
+// the calls that follow: the head record (v, Delta, a) once per head (row block 0), the k
+// record once per sequence and k/q group (its first head). Nothing else in the launch
+// reads that slot: every unit copies records [start, start + c) only.
+template <int S_IO>
+__device__ __forceinline__ void ring_append(const KParams& p, const Plan& pl, const uint8_t* st, int lane) {
+  if (pl.rb != 0) return;
+  int slot = pl.start + pl.c;
+  slot -= (slot >= p.cap) ? p.cap : 0;
+  const int kpe = (pl.h == pl.g * p.hpg) ? p.N * S_IO / 16 : 0;  // 16-byte pieces of k (first head)
+  const int rpe = p.rec_bytes / 16;                                // of the head record
+  const uint4* ksrc = reinterpret_cast<const uint4*>(st + p.off_krec + (size_t)pl.c * p.rec_k_bytes);
+  const uint4* rsrc = reinterpret_cast<const uint4*>(st + p.off_rec + (size_t)pl.c * p.rec_bytes);
+  uint4* kdst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.ring_k) +
+                                         (((size_t)pl.b * p.G + pl.g) * p.cap + slot) * p.rec_k_bytes);
+  uint4* rdst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.ring) +
+                                         (((size_t)pl.b * p.H + pl.h) * p.cap + slot) * p.rec_bytes);
+  for (int t = lane; t < kpe + rpe; t += 32) {
+    if (t < kpe)
+      kdst[t] = ksrc[t];
+    else
+      rdst[t - kpe] = rsrc[t - kpe];
   }
 }
 
@@ -744,6 +714,8 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
         output_coefs_pairs<N, IO>(rec, qbuf, c, n, o0, 0, GW + 1, alpha, cw, kqraw, reuse, lane);
     }
     group_sync(bar_id, GT);
+    // the new entry into the ring, while the row warps write the outputs
+    if (MODE == kModeReplay && NQ == 1 && p.append_here) ring_append<S_IO>(p, pl, st, lane);
   } else {
     float4 qr[NQR];
 #pragma unroll
@@ -1043,23 +1015,13 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     fence_mbar_init();
   }
   __syncthreads();
-  if constexpr (MODE == kModeReplay && NQ == 1) {
-    // One-position calls append their entries here rather than in a pre-pass: each CTA
-    // writes the new ring record of each of its own units (k, v, then Delta and a in one
-    // 16-byte piece), makes the writes visible to the bulk copies that read them, and
-    // tells the producer, which meanwhile streams the first state tiles.
-    if (p.append_here && threadIdx.x < kConsumerWarps * 32) {
-      append_entries<S_IO>(p);
-      named_arrive(kAppendBar, kThreads);
-    }
-  }
 
   const int warp = threadIdx.x / 32;
   if (warp >= kConsumerWarps) {
     if constexpr (MODE == kModeEager)
       producer_loop_eager<CKPT, S_IO>(p, stages, bars);
     else
-      producer_loop<MODE, CKPT, S_IO, MODE == kModeReplay && NQ == 1>(p, stages, bars);
+      producer_loop<MODE, CKPT, S_IO>(p, stages, bars);
     return;
   }
   const int g = warp / Gr::kWarps;  // consumer group

@@ -20,7 +20,7 @@ struct KParams {
   int32_t commit;  // replay: 1 = step (new entries committed), 0 = verify (tentative)
   int32_t fold_min;     // flush: fold only buffers holding at least this many entries (>= 1)
   int32_t flushed_or;   // replay: OR this call's fold flags into `flushed` (a flush before it wrote them)
-  int32_t append_here;  // replay, one position: the kernel appends the entries (no pre-pass)
+  int32_t append_here;  // replay, one position: the entry comes from the inputs; the kernel appends it (no pre-pass)
   // this call's inputs and outputs
   const void* q;
   const void* k;

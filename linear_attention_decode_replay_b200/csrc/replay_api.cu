@@ -129,7 +129,9 @@ int build_layout(KParams* p, const replay_config& c, int mode, int fp8_eager, in
   p->ws_cw = round_up(p->ws_sig + (replay::kMaxWindow + 4) * 4, 16);
   p->ws_kq = p->ws_cw + replay::kMaxPos * replay::kMaxWindow * 4;
   p->ws_wt = round_up(p->ws_kq + replay::kMaxPos * replay::kMaxWindow * 4, 16);
-  p->ws_group_bytes = round_up(p->ws_wt + lfold * p->wt_stride * 4, 128);
+  // ... and the inverse scales of a row group's rows, for the fold's re-quantisation
+  p->ws_inv = round_up(p->ws_wt + lfold * p->wt_stride * 4, 16);
+  p->ws_group_bytes = round_up(p->ws_inv + replay::row_group_rows(N) * 4, 128);
   p->ws_off = kHeaderBytes;
   p->stages_off = round_up(p->ws_off + replay::kGroups * p->ws_group_bytes, 128);
   const int avail = smem_optin - p->stages_off;

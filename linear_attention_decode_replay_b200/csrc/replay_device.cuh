@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -258,6 +259,48 @@ __device__ __forceinline__ void e2m1_row_scale(float amax, float& scale, float& 
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
+// Read-copy codes for the dot products: four e4m3 (byte i = element i) or e2m1 codes as
+// two f16x2 words (elements 0,1 and 2,3), the first step of the conversions above
+// without the widening to f32.
+__device__ __forceinline__ uint2 e4m3x4_to_half4(uint32_t w) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+__device__ __forceinline__ uint2 e2m1x4_to_half4(uint32_t w16) {
+  uint32_t h01, h23;
+  asm("{\n\t.reg .b8 lo, hi;\n\t"
+      "mov.b16 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, hi;\n\t}"
+      : "=r"(h01), "=r"(h23)
+      : "h"(static_cast<unsigned short>(w16)));
+  return make_uint2(h01, h23);
+}
+// four floats (exactly representable in f16: BF16 inputs in f16's range) as two f16x2 words
+__device__ __forceinline__ uint2 float4_to_half4(float4 v) {
+  const __half2 lo = __floats2half2_rn(v.x, v.y);
+  const __half2 hi = __floats2half2_rn(v.z, v.w);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+// a.x b.x + (a.y b.y + (a.z b.z + a.w b.w)) of f16 operands, accumulated in f32 by the
+// mixed-precision FMA (f16 x f16 -> f32): every product is exact in f32, so the result
+// equals dot4 of the operands widened to f32, without the widening conversions.
+__device__ __forceinline__ float dot4_h(uint2 a, uint2 b) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {a2, a3}, %2;\n\t"
+      "mov.b32 {b0, b1}, %3;\n\t"
+      "mov.b32 {b2, b3}, %4;\n\t"
+      "fma.rn.f32.f16 %0, a3, b3, 0f00000000;\n\t"
+      "fma.rn.f32.f16 %0, a2, b2, %0;\n\t"
+      "fma.rn.f32.f16 %0, a1, b1, %0;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\t}"
+      : "=f"(d)
+      : "r"(a.x), "r"(a.y), "r"(b.x), "r"(b.y));
+  return d;
+}
 __device__ __forceinline__ float amax4(float4 a) {
   return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
 }
@@ -292,8 +335,10 @@ __device__ __forceinline__ float seg_allmax(float v) {
 // row it covers); afterwards lane l holds complete row sums for R/TPR rows (or one row,
 // replicated over TPR/R lanes, when R < TPR). Costs about R + log2(TPR) shuffles
 // instead of R * log2(TPR). `base` returns the index of the first row held in v[0].
-template <int R, int OFF>
+// (MAX: the same with the maximum in place of the sum.)
+template <int R, int OFF, bool MAX = false>
 struct SegTranspose {
+  __device__ __forceinline__ static float op(float a, float b) { return MAX ? fmaxf(a, b) : a + b; }
   __device__ __forceinline__ static void run(float* v, int lane, int& base) {
     if constexpr (OFF >= 1) {
       if constexpr (R > 1) {
@@ -303,13 +348,13 @@ struct SegTranspose {
         for (int i = 0; i < H; ++i) {
           const float send = up ? v[i] : v[i + H];
           const float keep = up ? v[i + H] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+          v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, OFF));
         }
         if (up) base += H;
-        SegTranspose<H, OFF / 2>::run(v, lane, base);
+        SegTranspose<H, OFF / 2, MAX>::run(v, lane, base);
       } else {
-        v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
-        SegTranspose<1, OFF / 2>::run(v, lane, base);
+        v[0] = op(v[0], __shfl_xor_sync(0xffffffffu, v[0], OFF));
+        SegTranspose<1, OFF / 2, MAX>::run(v, lane, base);
       }
     }
   }
@@ -323,13 +368,13 @@ struct SegLog2<1> {
   static constexpr int value = 0;
 };
 
-template <int R, int TPR>
+template <int R, int TPR, bool MAX = false>
 struct SegReduce {
   static constexpr int kHeld = (R >= TPR) ? R / TPR : 1;  // row sums each lane ends with
   // returns true for the lanes that should write their v[0..kHeld)
   __device__ __forceinline__ static bool run(float* v, int lane, int& base) {
     base = 0;
-    SegTranspose<R, TPR / 2>::run(v, lane, base);
+    SegTranspose<R, TPR / 2, MAX>::run(v, lane, base);
     if constexpr (R >= TPR) {
       return true;
     } else {

@@ -695,6 +695,7 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
   float* cw = reinterpret_cast<float*>(ws + p.ws_cw);        // [kMaxPos][kMaxWindow] entry coefficients
   float* wt = reinterpret_cast<float*>(ws + p.ws_wt);        // [c][wts] fold weight times v_j[p]
   float* kqraw = reinterpret_cast<float*>(ws + p.ws_kq);     // [kMaxPos][kMaxWindow] raw k_l . q_s
+  float* sinv = reinterpret_cast<float*>(ws + p.ws_inv);     // [row group] inverse row scales (fold)
   const size_t bh = (size_t)pl.b * p.H + pl.h;
   const int ngroups = (P + RGR - 1) / RGR;
   const bool fold = pl.fold;
@@ -757,6 +758,36 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
           float part[RT];
 #pragma unroll
           for (int r = 0; r < RT; ++r) part[r] = dot4(x[r], qr[s]);
+          dwr = Red::run(part, lane, dbase);
+#pragma unroll
+          for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
+        }
+      }
+    };
+    // The read copy with BF16 inputs: the codes stay f16 (one conversion per two codes)
+    // and meet the queries, as f16, in mixed-precision FMAs that accumulate in f32; the
+    // products are exact, so the dot products equal those of row_dots on widened values.
+    constexpr bool kHalfDots = (CKPT != kCkptF32) && (S_IO == 2) && (MODE == kModeReplay);
+    uint2 qh[kHalfDots ? NQR : 1];
+#pragma unroll
+    for (int s = 0; s < (kHalfDots ? NQR : 1); ++s) qh[s] = float4_to_half4(qr[s]);
+    auto rows_dots_half = [&](int gi) {
+      uint2 xc[RT];
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const int pr = gi * RGR + rbase + r;
+        xc[r] = make_uint2(0u, 0u);
+        if (pr < P)
+          xc[r] = (CKPT == kCkptFp4)
+                      ? e2m1x4_to_half4(*reinterpret_cast<const unsigned short*>(tile + (size_t)pr * (N / 2) + col / 2))
+                      : e4m3x4_to_half4(*reinterpret_cast<const uint32_t*>(tile + (size_t)pr * N + col));
+      }
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) {
+        if (s < n) {
+          float part[RT];
+#pragma unroll
+          for (int r = 0; r < RT; ++r) part[r] = dot4_h(xc[r], qh[s]);
           dwr = Red::run(part, lane, dbase);
 #pragma unroll
           for (int i = 0; i < Red::kHeld; ++i) dv[s][i] = part[i];
@@ -870,15 +901,23 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
     if (!fold) {
       // ---- output-only route: row group 0's dot products, then wait for the buffer
       // terms; further row groups (P > one row group) follow with the terms in hand
-      load_rows(x, 0, false);
-      row_dots(x);
+      if (kHalfDots && !pl.fp32_tile) {
+        rows_dots_half(0);
+      } else {
+        load_rows(x, 0, false);
+        row_dots(x);
+      }
       preload(0, !pl.fp32_tile);
       if (NQ > 1) output_coefs_quarters<N, IO>(rec, qbuf, c, n, o0, gw + 1, GW + 1, alpha, cw, kqraw, reuse, lane);  // positions gw+1, ...
       group_sync(bar_id, GT);
       emit(0, !pl.fp32_tile, true);
       for (int gi = 1; gi < ngroups; ++gi) {
-        load_rows(x, gi, false);
-        row_dots(x);
+        if (kHalfDots && !pl.fp32_tile) {
+          rows_dots_half(gi);
+        } else {
+          load_rows(x, gi, false);
+          row_dots(x);
+        }
         preload(gi, !pl.fp32_tile);
         emit(gi, !pl.fp32_tile, true);
       }
@@ -946,21 +985,46 @@ __device__ __forceinline__ void consume_unit(const KParams& p, const Plan& pl, u
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           const int pr = gi * RGR + rbase + r;
-          const size_t row = bh * PH + r0 + pr;
-          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + row * N + col), x[r]);
-          if (CKPT != kCkptF32) {
-            const float am = seg_allmax<TPR>(amax4(x[r]));
-            float sc, inv;
-            if (CKPT == kCkptFp4) {
-              e2m1_row_scale(am, sc, inv);
-              if (pr < P)
+          if (store_f32 && pr < P) __stcs(reinterpret_cast<float4*>(p.S + (bh * PH + r0 + pr) * N + col), x[r]);
+        }
+        if constexpr (CKPT != kCkptF32) {
+          // the rows' scales: their largest magnitudes by the transposing reduction (a lane
+          // ends with kHeld whole rows), each row's scale and inverse worked out once, by
+          // the lane that holds the row, and the inverses read back from the workspace by
+          // the row's lanes (a warp's rows are its own)
+          using RedMax = SegReduce<RT, TPR, true>;
+          float m[RT];
+#pragma unroll
+          for (int r = 0; r < RT; ++r) m[r] = amax4(x[r]);
+          int mbase = 0;
+          const bool mwr = RedMax::run(m, lane, mbase);
+          if (mwr) {
+#pragma unroll
+            for (int i = 0; i < RedMax::kHeld; ++i) {
+              const int rr = rbase + mbase + i;
+              const int pr = gi * RGR + rr;
+              float sc, inv;
+              if (CKPT == kCkptFp4)
+                e2m1_row_scale(m[i], sc, inv);
+              else
+                e4m3_row_scale(m[i], sc, inv);
+              sinv[rr] = inv;
+              if (pr < P) p.Sscale[bh * PH + r0 + pr] = sc;
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const int pr = gi * RGR + rbase + r;
+            const float inv = sinv[rbase + r];
+            const size_t row = bh * PH + r0 + pr;
+            if (pr < P) {
+              if (CKPT == kCkptFp4)
                 __stcs(reinterpret_cast<unsigned short*>(p.S8 + row * (N / 2) + col / 2),
                        static_cast<unsigned short>(quant4_e2m1(x[r], inv)));
-            } else {
-              e4m3_row_scale(am, sc, inv);
-              if (pr < P) __stcs(reinterpret_cast<unsigned int*>(p.S8 + row * N + col), quant4_e4m3(x[r], inv));
+              else
+                __stcs(reinterpret_cast<unsigned int*>(p.S8 + row * N + col), quant4_e4m3(x[r], inv));
             }
-            if (pr < P && (lane % TPR) == 0) p.Sscale[row] = sc;
           }
         }
         if (MODE != kModeFlush) row_dots(x);

@@ -46,7 +46,7 @@ struct KParams {
   int32_t rec_bytes, rec_k_bytes, qpack_pos;   // head / k record sizes; positions per qpack group
   int32_t off_krec, off_rec, off_q, off_meta;  // within a stage
   int32_t ws_off, ws_group_bytes;              // one workspace per consumer group
-  int32_t ws_alpha, ws_sig, ws_cw, ws_kq, ws_wt;  // within a group's workspace
+  int32_t ws_alpha, ws_sig, ws_cw, ws_kq, ws_wt, ws_inv;  // within a group's workspace
   int32_t wt_stride;                           // row stride of the fold weight table [L][wt_stride]
   int32_t smem_bytes;
 };

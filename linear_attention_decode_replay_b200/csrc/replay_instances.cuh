@@ -36,8 +36,21 @@ cudaError_t launch_one(const KParams& p, int grid, cudaStream_t s) {
       if (dev >= 0 && dev < kMaxDevices) configured[dev] = p.smem_bytes;
     }
   }
-  kern<<<grid, kThreads, p.smem_bytes, s>>>(p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: this grid's CTAs may be scheduled while the previous
+  // kernel on the stream drains (an SM takes one as soon as its previous CTA exits); the
+  // kernel waits for that kernel's completion (griddepcontrol.wait) before it reads any
+  // memory, so only its set-up overlaps the previous kernel's tail.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 constexpr int kVerifyPosSmall = 5;  // positions of the smaller multi-position instance

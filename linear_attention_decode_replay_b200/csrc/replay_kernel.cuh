@@ -1068,6 +1068,9 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
   uint8_t* stages = smem + p.stages_off;
   constexpr int S_IO = IoT<IO>::bytes;
 
+  // this CTA lets the next kernel on the stream be scheduled (see the launch), and sets
+  // up its barriers before waiting for the previous kernel to complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.num_stages; ++s) {
       // the producer's expect_tx (the eager gather adds its 32 lanes' cp.async arrivals)
@@ -1079,6 +1082,7 @@ __global__ void __launch_bounds__(kThreads, 1) replay_kernel(const __grid_consta
     fence_mbar_init();
   }
   __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's writes are visible
 
   const int warp = threadIdx.x / 32;
   if (warp >= kConsumerWarps) {

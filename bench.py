@@ -44,13 +44,12 @@ FALLBACK_HBM_GBS = 6650.0
 # window) of the workload it was captured on, from an ncu capture, and the hash of the
 # kernel sources it applies to. For another workload, or once the sources change, the
 # figure does not apply and is reported as null. "captured_on" is the hash of the sources
-# of the capture itself; the sources have since changed only in the dispatch of
-# multi-position verify calls (host code and a second verify instance), which leaves the
-# replay_step kernel as it was captured.
+# of the capture itself. Measured on the fold launch and an 8-entry output-only launch:
+# (fold + 15 x output-only) / 16.
 NCU_TRAFFIC = {"workload": "mamba2_b256",
-               "sources_sha256": "a0dcf23f3dd3b5f62340d4de902044d00a902427b2957326c531345116907711",
-               "captured_on": "02e754b9f0ac5f3f23f0ef3b60c8386e72f01b065fcf05a98a712ee408d5eafb",
-               "bytes_per_launch": 597.3e6}
+               "sources_sha256": "e21d8dddf37eccd0f0edeb00f8e98d6b152826fcde7bec1dd8fcedccd8204fe7",
+               "captured_on": "e21d8dddf37eccd0f0edeb00f8e98d6b152826fcde7bec1dd8fcedccd8204fe7",
+               "bytes_per_launch": 646.1e6}
 
 
 def kernel_sources_hash() -> str:

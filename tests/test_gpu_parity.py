@@ -25,6 +25,21 @@ def _check_decode(rep, tol=hx.TOL_F32):
     assert rep.ckpt_err <= tol, rep.ckpt_err
 
 
+def _report_errors(name, rep):
+    """With REPLAY_REPORT_DIR set, records the measured errors of a passing parity run in
+    parity_errors.json there (one entry per workload)."""
+    out_dir = os.environ.get("REPLAY_REPORT_DIR")
+    if not out_dir:
+        return
+    os.makedirs(out_dir, exist_ok=True)
+    path = os.path.join(out_dir, "parity_errors.json")
+    data = json.load(open(path)) if os.path.exists(path) else {}
+    data[name] = {"max_rel_err_outputs": float(rep.max_err), "max_rel_err_checkpoint": float(rep.ckpt_err),
+                  "flags_equal": bool(rep.flags_equal), "counts_equal": bool(rep.counts_equal)}
+    with open(path, "w") as f:
+        json.dump(data, f, indent=1)
+
+
 # ------------------------------------------------------------------ FP8 quantiser, bit-exact
 
 @pytest.mark.parametrize("n", [16, 32, 64, 128])
@@ -49,6 +64,7 @@ def test_quantize_rows_bit_exact(n):
 def test_tiny_replay_matches_oracle_every_step():
     rep = hx.run_decode(gen.SHAPES["tiny"], 32, np.arange(2))
     _check_decode(rep)
+    _report_errors("tiny", rep)
 
 
 def test_tiny_eager_matches_oracle_every_step():
@@ -360,6 +376,7 @@ def test_mamba2_b256_decode_sampled():
     rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 8))
     _check_decode(rep)
     assert rep.max_err <= hx.TOL_BF16
+    _report_errors(shape.name, rep)
 
 
 def test_mamba2_b256_groups_decode_sampled():
@@ -369,6 +386,7 @@ def test_mamba2_b256_groups_decode_sampled():
     shape = gen.SHAPES["mamba2_b256_g8"]
     rep = hx.run_decode(shape, shape.steps, hx.sample_rows(shape.B, 6, seed=3))
     _check_decode(rep)
+    _report_errors(shape.name, rep)
 
 
 def test_mamba2_b256_fp4_sampled():
@@ -438,6 +456,7 @@ def test_mamba2_b256_spec_sampled():
     shape = gen.SHAPES["mamba2_b256_spec"]
     rep = hx.run_spec(shape, shape.steps, hx.sample_rows(shape.B, 6))
     _check_decode(rep)
+    _report_errors(shape.name, rep)
 
 
 SWEEP = [s for s in gen.sweep_shapes() if (s.B, s.L) in ((1, 4), (16, 32), (1024, 16), (64, 8))]

@@ -8,12 +8,15 @@
 //     per instruction: the unit's checkpoint tile (FP32 master rows, or the FP8 / FP4
 //     read copy's codes + per-row scales), the live k records of the head's k/q group
 //     and the head's live v, Delta, a records (each in one or two pieces of the ring),
-//     and the queries; all complete on the stage's "full" mbarrier;
+//     the queries and, for one-position calls, the new entry's k and v straight from the
+//     inputs; all complete on the stage's "full" mbarrier;
 //   * NG consumer groups (kGroupGemvWarps row warps + one coefficient warp each) take
 //     alternate units end to end: the coefficient warp forms the decay weights and the
 //     k_j . q_s products while the row warps stream the state rows' dot products (or the
 //     fused fold, its write-back and the outputs from the fresh rows); the group meets at
-//     its barrier for the outputs and releases the stage through its "empty" mbarrier.
+//     its barrier for the outputs, the coefficient warp appends a one-position call's new
+//     entry to the ring meanwhile, and the group releases the stage through its "empty"
+//     mbarrier.
 //     Two groups keep two units in flight, so one unit's short dependent chains overlap
 //     the other's, while the producer keeps the next stages' copies in flight.
 // The state is streamed exactly once per call; every other byte is small.

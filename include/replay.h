@@ -23,6 +23,10 @@
  *    library never allocates device memory. A replay_ctx holds host metadata only.
  *  - Work is queued asynchronously on the given stream. Only replay_read_counts and
  *    replay_check_status synchronise (that stream only).
+ *  - The decode kernel is launched with programmatic stream serialization: its blocks may
+ *    be scheduled while the previous kernel on the stream drains, but they read and write
+ *    no global memory before that kernel has completed (griddepcontrol.wait), so stream
+ *    order holds as for any launch; work queued after it waits for it as usual.
  *  - Invalid arguments return a negative replay_status at once and queue nothing.
  *    Errors found on the device are OR-ed into the caller's status word; read them
  *    with replay_check_status. No kernel traps.

@@ -45,10 +45,10 @@ FALLBACK_HBM_GBS = 6650.0
 # kernel sources it applies to. For another workload, or once the sources change, the
 # figure does not apply and is reported as null. "captured_on" is the hash of the sources
 # of the capture itself (they differ from the current ones only in the kernel's header
-# comment). Measured on the fold launch and an 8-entry output-only launch:
-# (fold + 15 x output-only) / 16.
+# comment and in two unused device helpers since removed). Measured on the fold launch
+# and an 8-entry output-only launch: (fold + 15 x output-only) / 16.
 NCU_TRAFFIC = {"workload": "mamba2_b256",
-               "sources_sha256": "6f35a16b7781f9225785ae9db02a5280cb5815e66aa2b671f6b69dea3e68716b",
+               "sources_sha256": "ca5c0a8c8f3c97581a3b95deec93766a80041e023cd01d3a2fcda67ef3bd8f8a",
                "captured_on": "e21d8dddf37eccd0f0edeb00f8e98d6b152826fcde7bec1dd8fcedccd8204fe7",
                "bytes_per_launch": 646.1e6}
 

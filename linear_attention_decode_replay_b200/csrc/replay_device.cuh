@@ -141,10 +141,6 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 __device__ __forceinline__ void group_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-// Arrive on named barrier `id` (of `count` threads) without waiting.
-__device__ __forceinline__ void named_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 // Group barrier with an AND-vote across the group's threads.
 __device__ __forceinline__ bool group_all(bool v, int id, int count) {
   uint32_t r;
@@ -317,13 +313,7 @@ __device__ __forceinline__ float warp_suffix_prod(float x, int lane) {
 }
 
 // ---------------------------------------------------------------- segment reductions
-// Sum over the TPR lanes of an aligned lane segment (all lanes get the total).
-template <int TPR>
-__device__ __forceinline__ float seg_allsum(float v) {
-#pragma unroll
-  for (int off = TPR / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
+// Maximum over the TPR lanes of an aligned lane segment (all lanes get it).
 template <int TPR>
 __device__ __forceinline__ float seg_allmax(float v) {
 #pragma unroll
